@@ -1,0 +1,282 @@
+"""Seeded synthetic inputs for split-KV decode attention.
+
+This module draws inputs only; it holds none of the attention arithmetic.
+The test harness, the benchmark and the fp64 oracle all take their inputs
+from here, so both sides of a parity check see the same bf16 bytes.
+
+Every tensor element is a pure function of (stream seed, element index):
+the SplitMix64 counter generator of ``fdgen.c`` followed by Box-Muller and
+round-to-nearest-even to bf16.  bf16 tensors are held as ``numpy.uint16``
+bit patterns.
+
+Workload shapes follow the decode workload the Flash-Decoding write-up
+discusses (one query token per sequence against a long cached history,
+CodeLlama-34B at batch 1 over 512 to 64K tokens: slavadubrov.com, "What is
+Flash-Decoding, and when does it speed up LLMs?", sections "Why decode needs
+a different schedule" and "Interpret the reported result") plus the 256K
+context of "Faster Than Flash" (abstract).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import subprocess
+from dataclasses import dataclass, field
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC_PATH = os.path.join(_HERE, "fdgen.c")
+_LIB_PATH = os.path.join(_HERE, "libfdgen.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile fdgen.c into libfdgen.so next to it."""
+    if (force or not os.path.exists(_LIB_PATH)
+            or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC_PATH)):
+        subprocess.check_call(["gcc", "-O2", "-Wall", "-Wextra", "-shared", "-fPIC",
+                               "-pthread", _SRC_PATH, "-o", _LIB_PATH, "-lm"])
+    return _LIB_PATH
+
+BF16_NAN = np.uint16(0x7FC0)
+
+# Stream indices: each tensor of a workload draws from its own stream, whose
+# seed is draw number <index> of the workload's base stream.
+STREAM_Q, STREAM_K, STREAM_V, STREAM_SEQLENS, STREAM_PERM, STREAM_POS = range(6)
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        u64 = ctypes.c_uint64
+        lib.fdgen_u64.argtypes = [u64, u64, u64, ctypes.c_void_p]
+        lib.fdgen_u64.restype = None
+        lib.fdgen_normal_f64.argtypes = [u64, u64, u64, ctypes.c_void_p]
+        lib.fdgen_normal_f64.restype = None
+        lib.fdgen_normal_bf16.argtypes = [u64, u64, u64, ctypes.c_void_p, ctypes.c_int]
+        lib.fdgen_normal_bf16.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    return max(1, min(64, os.cpu_count() or 1))
+
+
+def u64(seed: int, n: int, offset: int = 0) -> np.ndarray:
+    out = np.empty(n, dtype=np.uint64)
+    if n:
+        _load().fdgen_u64(seed, offset, n, out.ctypes.data)
+    return out
+
+
+def normal_f64(seed: int, n: int, offset: int = 0) -> np.ndarray:
+    out = np.empty(n, dtype=np.float64)
+    if n:
+        _load().fdgen_normal_f64(seed, offset, n, out.ctypes.data)
+    return out
+
+
+def normal_bf16(seed: int, shape, offset: int = 0, out: Optional[np.ndarray] = None,
+                nthreads: Optional[int] = None) -> np.ndarray:
+    """bf16 bit patterns of N(0,1) draws, element i = draw (offset + i)."""
+    n = int(np.prod(shape)) if len(shape) else 1
+    if out is None:
+        out = np.empty(shape, dtype=np.uint16)
+    assert out.dtype == np.uint16 and out.flags.c_contiguous and out.size == n
+    if n:
+        _load().fdgen_normal_bf16(seed, offset, n, out.ctypes.data,
+                                  nthreads or default_threads())
+    return out
+
+
+def stream_seed(base_seed: int, stream: int) -> int:
+    return int(u64(base_seed, 1, offset=stream)[0])
+
+
+def uniform_int(seed: int, n: int, lo: int, hi: int) -> np.ndarray:
+    """n integers in [lo, hi]: lo + (draw mod (hi - lo + 1))."""
+    r = u64(seed, n)
+    return (np.int64(lo) + (r % np.uint64(hi - lo + 1)).astype(np.int64)).astype(np.int32)
+
+
+def permutation(seed: int, n: int) -> np.ndarray:
+    """Fisher-Yates: for i = n-1 .. 1, swap a[i] with a[draw_k mod (i+1)], k = n-1-i."""
+    a = np.arange(n, dtype=np.int64)
+    r = u64(seed, max(n - 1, 0))
+    for k, i in enumerate(range(n - 1, 0, -1)):
+        j = int(r[k] % np.uint64(i + 1))
+        a[i], a[j] = a[j], a[i]
+    return a.astype(np.int32)
+
+
+def distinct_positions(seed: int, count: int, n: int) -> np.ndarray:
+    """`count` distinct integers of [0, n): the first `count` steps of a
+    forward Fisher-Yates shuffle of 0..n-1 (swap a[i] with a[i + draw_i mod (n-i)])."""
+    r = u64(seed, count)
+    swapped: dict = {}
+    out = []
+    for i in range(count):
+        j = i + int(r[i] % np.uint64(n - i))
+        ai, aj = swapped.get(i, i), swapped.get(j, j)
+        swapped[i], swapped[j] = aj, ai
+        out.append(aj)
+    return np.array(out, dtype=np.int32)
+
+
+def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """fp64 -> fp32 (nearest even) -> bf16 (nearest even), as bit patterns."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + np.uint64(0x7FFF) + ((u >> np.uint64(16)) & np.uint64(1))) >> np.uint64(16)
+    return u.astype(np.uint16)
+
+
+def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
+    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+@dataclass
+class Workload:
+    """One decode-attention problem held on the host.
+
+    q: [B, Hq, D] bf16 bits.  Contiguous cache: k, v [B, Hkv, max_len, D].
+    Paged cache: k, v [num_blocks, Hkv, block_size, D] with
+    block_table [B, max_blocks_per_seq] int32.  seqlens: [B] int32 or None
+    (None means every sequence holds max_len tokens)."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    D: int
+    max_len: int
+    q: np.ndarray
+    k: np.ndarray
+    v: np.ndarray
+    scale: float
+    seqlens: Optional[np.ndarray] = None
+    block_size: int = 0
+    block_table: Optional[np.ndarray] = None
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def G(self) -> int:
+        return self.Hq // self.Hkv
+
+    @property
+    def paged(self) -> bool:
+        return self.block_table is not None
+
+    @property
+    def num_blocks(self) -> int:
+        return int(self.k.shape[0]) if self.paged else 0
+
+    @property
+    def max_blocks_per_seq(self) -> int:
+        return int(self.block_table.shape[1]) if self.paged else 0
+
+    def lengths(self) -> np.ndarray:
+        if self.seqlens is None:
+            return np.full(self.B, self.max_len, dtype=np.int64)
+        return np.clip(self.seqlens.astype(np.int64), 0, self.max_len)
+
+    def kv_bytes(self) -> int:
+        """Algorithmic K+V bytes: valid tokens x Hkv x D x 2 bytes x 2 tensors."""
+        return int(self.lengths().sum()) * self.Hkv * self.D * 4
+
+    def logical_kv(self, b: int, h: int):
+        """K, V rows [n, D] (bf16 bits) of sequence b, KV head h, in token order."""
+        n = int(self.lengths()[b])
+        if not self.paged:
+            return self.k[b, h, :n], self.v[b, h, :n]
+        bs = self.block_size
+        npages = (n + bs - 1) // bs
+        pages = self.block_table[b, :npages].astype(np.int64)
+        kk = self.k[pages, h].reshape(-1, self.D)[:n]
+        vv = self.v[pages, h].reshape(-1, self.D)[:n]
+        return kk, vv
+
+
+def make_problem(B: int, Hq: int, Hkv: int, D: int, max_len: int, seed: int,
+                 seqlens=None, nan_pad: bool = False, block_size: int = 0,
+                 num_blocks: Optional[int] = None, name: str = "custom",
+                 nthreads: Optional[int] = None) -> Workload:
+    """Build a workload with i.i.d. N(0,1) bf16 q, K, V from base `seed`.
+
+    Contiguous cache when block_size == 0.  Paged cache otherwise: the
+    physical pool holds `num_blocks` pages (default: exactly enough for every
+    sequence) and the block table is a seeded permutation of the pool,
+    reshaped [B, max_len / block_size]."""
+    q = normal_bf16(stream_seed(seed, STREAM_Q), (B, Hq, D), nthreads=nthreads)
+    if block_size:
+        assert max_len % block_size == 0
+        per_seq = max_len // block_size
+        nb = num_blocks if num_blocks is not None else B * per_seq
+        assert nb >= B * per_seq
+        perm = permutation(stream_seed(seed, STREAM_PERM), nb)
+        table = perm[: B * per_seq].reshape(B, per_seq).copy()
+        shape = (nb, Hkv, block_size, D)
+    else:
+        table = None
+        shape = (B, Hkv, max_len, D)
+    k = normal_bf16(stream_seed(seed, STREAM_K), shape, nthreads=nthreads)
+    v = normal_bf16(stream_seed(seed, STREAM_V), shape, nthreads=nthreads)
+    sl = None if seqlens is None else np.asarray(seqlens, dtype=np.int32)
+    if nan_pad and sl is not None:
+        assert not block_size
+        for b in range(B):
+            k[b, :, int(sl[b]):, :] = BF16_NAN
+            v[b, :, int(sl[b]):, :] = BF16_NAN
+    return Workload(name=name, B=B, Hq=Hq, Hkv=Hkv, D=D, max_len=max_len, q=q, k=k, v=v,
+                    scale=float(np.float32(1.0 / math.sqrt(D))), seqlens=sl,
+                    block_size=block_size, block_table=table)
+
+
+def plant_dominant_keys(w: Workload, count: int, seed: int, magnitude: float = 4.0) -> np.ndarray:
+    """Overwrite `count` seeded distinct positions of every KV head with the key
+    magnitude * q/|q| * sqrt(D), q being the group's first query head of that
+    KV head (batch entry 0 .. B-1 alike), computed in fp64 and rounded to bf16.
+    Returns the positions."""
+    assert not w.paged
+    pos = distinct_positions(stream_seed(seed, STREAM_POS), count, w.max_len)
+    G = w.G
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            q0 = bf16_bits_to_f64(w.q[b, h * G])
+            key = magnitude * q0 / np.linalg.norm(q0) * math.sqrt(w.D)
+            w.k[b, h, pos, :] = f64_to_bf16_bits(key)[None, :]
+    w.meta["dominant_positions"] = pos
+    return pos
+
+
+# --- the five workloads -------------------------------------------------------
+
+CONFIG_SEED_BASE = 20260000
+CONFIG2_LENGTHS = (512, 2048, 8192, 16384, 32768, 65536)
+
+
+def config(idx: int, L: Optional[int] = None, nthreads: Optional[int] = None) -> Workload:
+    """Full-size workload `idx` (1..5).  Config 2 takes its cache length L."""
+    seed = CONFIG_SEED_BASE + idx
+    if idx == 1:
+        return make_problem(1, 8, 8, 64, 512, seed, name="tiny-mha-L512", nthreads=nthreads)
+    if idx == 2:
+        L = 65536 if L is None else int(L)
+        return make_problem(1, 64, 8, 128, L, seed, name=f"codellama34b-gqa8-L{L}",
+                            nthreads=nthreads)
+    if idx == 3:
+        sl = uniform_int(stream_seed(seed, STREAM_SEQLENS), 32, 1024, 32768)
+        return make_problem(32, 32, 8, 128, 32768, seed, seqlens=sl, nan_pad=True,
+                            name="varlen-B32", nthreads=nthreads)
+    if idx == 4:
+        return make_problem(8, 32, 8, 128, 131072, seed, block_size=16,
+                            name="paged-B8-L128K-bs16", nthreads=nthreads)
+    if idx == 5:
+        w = make_problem(1, 32, 8, 128, 262144, seed, name="peaked-L256K", nthreads=nthreads)
+        plant_dominant_keys(w, 64, seed)
+        return w
+    raise ValueError(f"no workload {idx}")
