@@ -1,0 +1,171 @@
+/*
+ * fd.h — C ABI of the B200 (sm_100a) split-KV decode attention library
+ * (libfd.so).
+ *
+ * The operation is Flash-Decoding ("What is Flash-Decoding, and when does it
+ * speed up LLMs?", slavadubrov.com: the opening paragraph and the section
+ * "Why decode needs a different schedule"). One new query token per
+ * sequence attends over that sequence's long cached K/V history. The history
+ * is split into chunks. Each chunk gives a partial output and a log-sum-exp,
+ * and a reduction merges the partials into the exact attention over the
+ * whole history:
+ *
+ *     out[b, h, :] = softmax_j(scale * q[b, h, :] . K[b, kv, j, :]) @ V[b, kv, j, :]
+ *     lse[b, h]    = ln sum_j exp(scale * q[b, h, :] . K[b, kv, j, :])
+ *
+ * Here kv = h / (Hq / Hkv), which covers grouped-query attention, and j runs
+ * over the seqlens[b] valid cached tokens.
+ *
+ * Conventions shared by every entry point:
+ *  - Tensor pointers are DEVICE pointers owned by the caller. The library
+ *    keeps no pointer and allocates nothing; the workspace is caller-supplied.
+ *  - Element types: q, K, V and out are bf16; lse, the workspace and scale
+ *    are fp32; seqlens and block_table are int32.
+ *  - Errors are return codes. No entry point aborts, throws or prints.
+ *    Argument checks run on the host before anything is launched; an invalid
+ *    call launches nothing.
+ *  - Work is asynchronous on the caller's stream. A fault inside a kernel
+ *    surfaces at the caller's next synchronisation.
+ *  - There is no CPU fallback. The kernels are built for sm_100a only.
+ */
+#ifndef FD_H_
+#define FD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FD_API __attribute__((visibility("default")))
+#else
+#define FD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t (struct CUstream_st*); NULL is the legacy default
+ * stream. */
+typedef struct CUstream_st* fd_stream_t;
+
+typedef enum fd_status {
+  FD_OK = 0,
+  /* Null pointer, non-positive size, Hq % Hkv != 0, a tensor pointer not
+   * 16-byte aligned (lse: 4-byte), num_splits outside [1, 1024], scale not
+   * finite and positive, seqlen-independent shape limits exceeded. */
+  FD_ERR_INVALID_ARGUMENT = -1,
+  /* Head dim D not in {64, 128}, group size Hq/Hkv not in {1, 2, 4, 8, 16},
+   * block_size not a power of two in [8, 256], or the device is not sm_100. */
+  FD_ERR_UNSUPPORTED = -2,
+  /* The chosen split count needs a workspace, and the one passed is NULL or
+   * smaller than fd_workspace_bytes() reports. */
+  FD_ERR_WORKSPACE = -3,
+  /* A CUDA runtime or driver call failed (launch error, tensor-map encode). */
+  FD_ERR_CUDA = -4,
+  /* A kernel gave up on a bounded wait. Its outputs are not valid. */
+  FD_ERR_DEVICE_TIMEOUT = -5
+} fd_status;
+
+/* Shape of one decode-attention call.
+ *   B           sequences in the batch (1 .. 65535)
+ *   Hq, Hkv     query heads and KV heads (Hkv .. 65535, Hq % Hkv == 0)
+ *   D           head dimension (64 or 128)
+ *   max_len     contiguous cache: rows held per (sequence, KV head);
+ *               paged cache: the longest sequence the block table can hold
+ *               (<= max_blocks_per_seq * block_size)
+ *   block_size  0 for a contiguous cache; otherwise tokens per page
+ *   num_blocks  paged cache: pages in the pool (ignored when contiguous)
+ *   max_blocks_per_seq  paged cache: row length of block_table */
+typedef struct fd_problem {
+  int32_t B;
+  int32_t Hq;
+  int32_t Hkv;
+  int32_t D;
+  int32_t max_len;
+  int32_t block_size;
+  int32_t num_blocks;
+  int32_t max_blocks_per_seq;
+} fd_problem;
+
+/* Split-count planner.
+ * Follows the same page's section "Why decode needs a different schedule".
+ * Splitting the history creates extra work units when the batch supplies too
+ * few. For a short history the partials and the reduction can cost more than
+ * they save, and a large batch already supplies the work.
+ * Returns S >= 1 for fd_decode's num_splits, chosen for the current device's
+ * SM count. Returns 1 when B*Hkv already fills the device or the history is
+ * short. Returns a negative fd_status for invalid or unsupported shapes.
+ * Host only and deterministic. It reads the SM count of the current device
+ * once per device and caches it. */
+FD_API int fd_plan(int B, int Hq, int Hkv, int D, int max_len, int block_size);
+
+/* The same planner with the SM count given explicitly. Pure function: no
+ * CUDA call. */
+FD_API int fd_plan_sm(int num_sms, int B, int Hq, int Hkv, int D, int max_len,
+               int block_size);
+
+/* Tokens per split for a given split count. This is ceil(max_len /
+ * num_splits) rounded up to the 64-token tile. Split s covers tokens
+ * [s*chunk, (s+1)*chunk) of every sequence, and splits past a sequence's end
+ * are empty. Returns a negative fd_status for invalid arguments. */
+FD_API int fd_split_chunk(int max_len, int num_splits);
+
+/* Workspace bytes that fd_decode needs for num_splits splits. This is 0
+ * when num_splits == 1. Otherwise it is the fp32 partial outputs
+ * [B, Hq, S, D] followed by the fp32 partial log-sum-exps [B, Hq, S], each
+ * part rounded up to 256 bytes, with S = num_splits. The effective split
+ * count never exceeds num_splits, so this size is always enough for the call.
+ * Returns 0 for invalid arguments. */
+FD_API size_t fd_workspace_bytes(int B, int Hq, int D, int num_splits);
+
+/* Decode attention for one query token per sequence.
+ *   p            shape (see fd_problem)
+ *   q            [B, Hq, D] bf16, 16-byte aligned
+ *   k_cache, v_cache
+ *                contiguous: [B, Hkv, max_len, D] bf16;
+ *                paged:      [num_blocks, Hkv, block_size, D] bf16;
+ *                16-byte aligned
+ *   seqlens      [B] int32 valid tokens per sequence, or NULL (all max_len).
+ *                Values are clamped to [0, max_len]. Rows at or past a
+ *                sequence's length are never summed; they may hold anything,
+ *                NaN included. A length of 0 gives out = 0 and lse = -inf.
+ *   block_table  paged only: [B, max_blocks_per_seq] int32; token t of
+ *                sequence b sits in page block_table[b, t / block_size], row
+ *                t % block_size. Entries are read only for pages that hold
+ *                valid tokens. A page id outside [0, num_blocks) reads zeros.
+ *                NULL selects the contiguous layout and needs block_size == 0.
+ *   scale        softmax scale (finite, > 0), typically 1/sqrt(D)
+ *   num_splits   requested split count in [1, 1024], normally fd_plan's
+ *                result. The effective count is ceil(max_len / chunk).
+ *   out          [B, Hq, D] bf16, round-to-nearest-even, 16-byte aligned
+ *   lse          [B, Hq] fp32 natural-log log-sum-exp of the scaled logits,
+ *                or NULL to skip it
+ *   workspace    fp32 scratch of at least fd_workspace_bytes(B, Hq, D, S)
+ *                bytes for the effective split count S (the num_splits
+ *                passed is always enough), 16-byte aligned. It may be NULL
+ *                when S == 1. Its
+ *                contents on entry do not matter, and it must not be shared
+ *                by calls that overlap on the GPU.
+ *   stream       the stream to run on
+ * Results are bit-identical across repeated calls with the same inputs and
+ * the same num_splits. The paged and contiguous layouts of the same logical
+ * cache also give bit-identical results. */
+FD_API fd_status fd_decode(const fd_problem* p, const void* q, const void* k_cache,
+                    const void* v_cache, const int32_t* seqlens,
+                    const int32_t* block_table, float scale, int num_splits,
+                    void* out, float* lse, void* workspace,
+                    size_t workspace_bytes, fd_stream_t stream);
+
+/* Waits for `stream`, then reads and clears the current device's error word.
+ * A kernel sets that word when one of its bounded waits runs out. Returns
+ * FD_OK, FD_ERR_DEVICE_TIMEOUT, or FD_ERR_CUDA. */
+FD_API fd_status fd_check_device_error(fd_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+FD_API const char* fd_status_string(fd_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FD_H_ */

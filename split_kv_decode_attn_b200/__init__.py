@@ -1,1 +1,177 @@
-"""B200-native split-KV decode attention (Flash-Decoding)."""
+"""B200-native split-KV decode attention (Flash-Decoding).
+
+Python binding of libfd.so.  Every function here marshals arguments for the C
+ABI declared in ``include/fd.h`` and calls it; all arithmetic runs in the
+library's CUDA kernels.  There is no fallback: if libfd.so is missing or a
+call fails, an exception is raised.
+
+The functions named ``fd_*`` mirror the C entry points one to one and take
+raw device pointers (ints) or torch tensors.  ``decode`` is a convenience
+wrapper that allocates the outputs and workspace with torch and calls
+``fd_decode`` on the current stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfd.so")
+
+FD_OK = 0
+FD_ERR_INVALID_ARGUMENT = -1
+FD_ERR_UNSUPPORTED = -2
+FD_ERR_WORKSPACE = -3
+FD_ERR_CUDA = -4
+FD_ERR_DEVICE_TIMEOUT = -5
+
+# Entry points declared in include/fd.h.
+EXPORTS = ("fd_plan", "fd_plan_sm", "fd_split_chunk", "fd_workspace_bytes", "fd_decode",
+           "fd_check_device_error", "fd_status_string")
+
+
+class FdError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {fd_status_string(status)} ({status})" if what
+                         else f"{fd_status_string(status)} ({status})")
+
+
+class fd_problem(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
+                ("D", ctypes.c_int32), ("max_len", ctypes.c_int32),
+                ("block_size", ctypes.c_int32), ("num_blocks", ctypes.c_int32),
+                ("max_blocks_per_seq", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libfd.so (raises if it is not built: there is no fallback path)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise ImportError(f"{path} is missing; build it with __graft_entry__.build()")
+        lib = ctypes.CDLL(path)
+        I, vp, sz, F = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float
+        lib.fd_plan.argtypes = [I] * 6
+        lib.fd_plan.restype = I
+        lib.fd_plan_sm.argtypes = [I] * 7
+        lib.fd_plan_sm.restype = I
+        lib.fd_split_chunk.argtypes = [I, I]
+        lib.fd_split_chunk.restype = I
+        lib.fd_workspace_bytes.argtypes = [I, I, I, I]
+        lib.fd_workspace_bytes.restype = sz
+        lib.fd_decode.argtypes = [ctypes.POINTER(fd_problem), vp, vp, vp, vp, vp, F, I, vp, vp,
+                                  vp, sz, vp]
+        lib.fd_decode.restype = I
+        lib.fd_check_device_error.argtypes = [vp]
+        lib.fd_check_device_error.restype = I
+        lib.fd_status_string.argtypes = [I]
+        lib.fd_status_string.restype = ctypes.c_char_p
+        _lib = lib
+    return _lib
+
+
+def _ptr(x) -> Optional[int]:
+    """Device address of a torch tensor, an int address, or None."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x or None
+    return x.data_ptr() or None
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream or None
+    if isinstance(stream, int):
+        return stream or None
+    return stream.cuda_stream or None
+
+
+# ---- one-to-one mirrors of the C entry points --------------------------------
+
+def fd_status_string(status: int) -> str:
+    return load_library().fd_status_string(int(status)).decode()
+
+
+def fd_plan(B: int, Hq: int, Hkv: int, D: int, max_len: int, block_size: int = 0) -> int:
+    return int(load_library().fd_plan(B, Hq, Hkv, D, max_len, block_size))
+
+
+def fd_plan_sm(num_sms: int, B: int, Hq: int, Hkv: int, D: int, max_len: int,
+               block_size: int = 0) -> int:
+    return int(load_library().fd_plan_sm(num_sms, B, Hq, Hkv, D, max_len, block_size))
+
+
+def fd_split_chunk(max_len: int, num_splits: int) -> int:
+    return int(load_library().fd_split_chunk(max_len, num_splits))
+
+
+def fd_workspace_bytes(B: int, Hq: int, D: int, num_splits: int) -> int:
+    return int(load_library().fd_workspace_bytes(B, Hq, D, num_splits))
+
+
+def fd_decode(problem: fd_problem, q, k_cache, v_cache, seqlens, block_table, scale: float,
+              num_splits: int, out, lse, workspace, workspace_bytes: int, stream=None) -> int:
+    """Call the C fd_decode; returns its status code."""
+    return int(load_library().fd_decode(
+        ctypes.byref(problem), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens),
+        _ptr(block_table), ctypes.c_float(scale), int(num_splits), _ptr(out), _ptr(lse),
+        _ptr(workspace), int(workspace_bytes), _stream(stream)))
+
+
+def fd_check_device_error(stream=None) -> int:
+    return int(load_library().fd_check_device_error(_stream(stream)))
+
+
+# ---- convenience wrapper -----------------------------------------------------
+
+def make_problem(B, Hq, Hkv, D, max_len, block_size=0, num_blocks=0, max_blocks_per_seq=0):
+    return fd_problem(B, Hq, Hkv, D, max_len, block_size, num_blocks, max_blocks_per_seq)
+
+
+def decode(q, k_cache, v_cache, seqlens=None, block_table=None, *, max_len: Optional[int] = None,
+           block_size: int = 0, scale: Optional[float] = None, num_splits: Optional[int] = None,
+           out=None, lse=None, workspace=None, stream=None):
+    """Decode attention on torch CUDA tensors.
+
+    q [B, Hq, D] bf16; contiguous caches [B, Hkv, max_len, D] bf16, or paged
+    caches [num_blocks, Hkv, block_size, D] with block_table [B, max_blocks]
+    int32; seqlens [B] int32 or None.  Returns (out [B, Hq, D] bf16,
+    lse [B, Hq] fp32).  num_splits defaults to fd_plan's choice."""
+    import torch
+    B, Hq, D = q.shape
+    if block_table is None:
+        _, Hkv, L, _ = k_cache.shape
+        max_len = L if max_len is None else max_len
+        prob = make_problem(B, Hq, Hkv, D, max_len)
+    else:
+        nb, Hkv, bs, _ = k_cache.shape
+        block_size = bs
+        mbps = block_table.shape[1]
+        max_len = mbps * bs if max_len is None else max_len
+        prob = make_problem(B, Hq, Hkv, D, max_len, bs, nb, mbps)
+    if scale is None:
+        scale = 1.0 / (D ** 0.5)
+    if num_splits is None:
+        num_splits = fd_plan(B, Hq, Hkv, D, max_len, block_size)
+        if num_splits < 0:
+            raise FdError(num_splits, "fd_plan")
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    wbytes = fd_workspace_bytes(B, Hq, D, num_splits)
+    if workspace is None and wbytes:
+        workspace = torch.empty(wbytes // 4, dtype=torch.float32, device=q.device)
+    have = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = fd_decode(prob, q, k_cache, v_cache, seqlens, block_table, scale, num_splits, out, lse,
+                   workspace, have, stream)
+    if st != FD_OK:
+        raise FdError(st, "fd_decode")
+    return out, lse

@@ -1,0 +1,415 @@
+// fd_api.cu — host side of libfd.so: argument checks, the split-count
+// planner, TMA tensor-map encoding and kernel launches on the caller's
+// stream.  See include/fd.h for the contract of every entry point.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fd.h"
+#include "fd_kernels.cuh"
+
+namespace {
+
+constexpr int kMaxSplits = 1024;
+constexpr int kMaxDevices = 64;
+
+// ---------------------------------------------------------------- planner
+
+// Cost model of one call, in microseconds, used to pick the split count.
+// Constants are measured on B200 (see the planner notes in the design doc):
+//   kHbmGBs     sustained K/V streaming rate of the whole device
+//   kCtaGBs     streaming rate one CTA reaches on its own (pipeline depth /
+//               memory latency)
+//   kCtaFixedUs per-CTA fixed cost: launch, first-tile latency, epilogue
+//   kCombineUs  second kernel of a split call, before its bytes
+struct PlanModel {
+  static constexpr double kHbmGBs = 6500.0;
+  static constexpr double kCtaGBs = 45.0;
+  static constexpr double kCtaFixedUs = 1.5;
+  static constexpr double kCombineUs = 2.0;
+};
+
+int tile_round_up(long long x) {
+  return static_cast<int>((x + fd::kTile - 1) / fd::kTile * fd::kTile);
+}
+
+int chunk_for(int max_len, int num_splits) {
+  const long long per = (static_cast<long long>(max_len) + num_splits - 1) / num_splits;
+  const int c = tile_round_up(per);
+  return c < fd::kTile ? fd::kTile : c;
+}
+
+int effective_splits(int max_len, int chunk) {
+  if (max_len <= 0) return 1;
+  return static_cast<int>((static_cast<long long>(max_len) + chunk - 1) / chunk);
+}
+
+double model_time_us(int num_sms, int B, int Hq, int Hkv, int D, int max_len, int S) {
+  const int chunk = chunk_for(max_len, S);
+  const int s_eff = effective_splits(max_len, chunk);
+  const double units = static_cast<double>(B) * Hkv * s_eff;
+  const double slots = static_cast<double>(num_sms) * fd::kCtasPerSm;
+  const double chunk_tok = std::min<double>(chunk, max_len);
+  const double cta_bytes = chunk_tok * D * 4.0;
+  const double full_waves = std::floor(units / slots);
+  const double rem = units - full_waves * slots;
+  const double hbm = PlanModel::kHbmGBs * 1e3;   // bytes per microsecond
+  const double cta = PlanModel::kCtaGBs * 1e3;
+  double t = 0.0;
+  if (full_waves > 0)
+    t += full_waves * (std::max(cta_bytes * slots / hbm, cta_bytes / cta) + PlanModel::kCtaFixedUs);
+  if (rem > 0) t += std::max(cta_bytes * rem / hbm, cta_bytes / cta) + PlanModel::kCtaFixedUs;
+  if (s_eff > 1) {
+    const double ws = static_cast<double>(B) * Hq * s_eff * (D + 1) * 4.0;
+    t += PlanModel::kCombineUs + 2.0 * ws / hbm;
+  }
+  return t;
+}
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int ilog2(int x) {
+  int r = 0;
+  while ((1 << r) < x) ++r;
+  return r;
+}
+
+fd_status check_shape(int B, int Hq, int Hkv, int D, int max_len, int block_size) {
+  if (B < 1 || B > 65535 || Hq < 1 || Hkv < 1 || Hkv > 65535 || max_len < 0)
+    return FD_ERR_INVALID_ARGUMENT;
+  if (Hq % Hkv != 0) return FD_ERR_INVALID_ARGUMENT;
+  if (D != 64 && D != 128) return FD_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return FD_ERR_UNSUPPORTED;
+  if (block_size != 0 && (!is_pow2(block_size) || block_size < 8 || block_size > 256))
+    return FD_ERR_UNSUPPORTED;
+  if (block_size < 0) return FD_ERR_INVALID_ARGUMENT;
+  return FD_OK;
+}
+
+// --------------------------------------------------------- device queries
+
+struct DeviceInfo {
+  std::atomic<int> sms{0};
+  std::atomic<int> sm100{-1};
+};
+DeviceInfo g_dev[kMaxDevices];
+
+fd_status current_device(int* dev) {
+  if (cudaGetDevice(dev) != cudaSuccess) return FD_ERR_CUDA;
+  if (*dev < 0 || *dev >= kMaxDevices) return FD_ERR_CUDA;
+  return FD_OK;
+}
+
+fd_status device_sms(int dev, int* sms) {
+  int v = g_dev[dev].sms.load();
+  if (v == 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return FD_ERR_CUDA;
+    g_dev[dev].sms.store(v);
+  }
+  *sms = v;
+  return FD_OK;
+}
+
+fd_status device_is_sm100(int dev) {
+  int v = g_dev[dev].sm100.load();
+  if (v < 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return FD_ERR_CUDA;
+    v = (major == 10 && minor == 0) ? 1 : 0;
+    g_dev[dev].sm100.store(v);
+  }
+  return v ? FD_OK : FD_ERR_UNSUPPORTED;
+}
+
+// ------------------------------------------------------------ tensor maps
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+fd_status encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
+  std::call_once(g_encode_once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                         cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  *fn = g_encode;
+  return g_encode ? FD_OK : FD_ERR_CUDA;
+}
+
+// 3-D view {D, rows, planes} of a bf16 cache, box {64, box_rows, 1}, 128-byte
+// swizzle, zero fill outside the tensor.
+fd_status make_cache_map(CUtensorMap* tm, const void* base, int D, long long rows,
+                         long long planes, int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  if (encoder(&enc) != FD_OK) return FD_ERR_CUDA;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(planes)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                           static_cast<cuuint64_t>(rows) * D * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FD_OK : FD_ERR_CUDA;
+}
+
+// --------------------------------------------------------------- launches
+
+template <int D, int NB, int MODE, bool PAGED>
+fd_status launch_split(const CUtensorMap& tk, const CUtensorMap& tv, const fd::SplitArgs& a,
+                       int n_splits, int Hkv, int B, cudaStream_t stream) {
+  constexpr int STAGES = D == 128 ? 3 : 6;
+  using L = fd::SplitSmem<D, STAGES>;
+  auto kern = fd::fd_split_kernel<D, NB, MODE, PAGED, STAGES>;
+  // The shared-memory opt-in is per device; remember which devices have it.
+  static std::atomic<unsigned long long> attr_done{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FD_ERR_CUDA;
+  const unsigned long long bit = 1ull << dev;
+  if (!(attr_done.load() & bit)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             L::kDynamicBytes) != cudaSuccess)
+      return FD_ERR_CUDA;
+    attr_done.fetch_or(bit);
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(n_splits), static_cast<unsigned>(Hkv),
+                     static_cast<unsigned>(B));
+  cfg.blockDim = dim3(fd::kThreads);
+  cfg.dynamicSmemBytes = L::kDynamicBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, tk, tv, a) != cudaSuccess) return FD_ERR_CUDA;
+  return FD_OK;
+}
+
+template <int D>
+fd_status launch_combine(const fd::CombineArgs& c, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg{};
+  const int rows = c.B * c.Hq;
+  cfg.gridDim = dim3(static_cast<unsigned>((rows + 3) / 4));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, fd::fd_combine_kernel<D>, c) != cudaSuccess) return FD_ERR_CUDA;
+  return FD_OK;
+}
+
+template <int D, bool PAGED>
+fd_status dispatch_split(int G, const CUtensorMap& tk, const CUtensorMap& tv,
+                         const fd::SplitArgs& a, int n_splits, int Hkv, int B,
+                         cudaStream_t s) {
+  if (G <= 4) return launch_split<D, 1, fd::kDup, PAGED>(tk, tv, a, n_splits, Hkv, B, s);
+  if (G == 8) return launch_split<D, 1, fd::kHiLo, PAGED>(tk, tv, a, n_splits, Hkv, B, s);
+  return launch_split<D, 2, fd::kHiLo, PAGED>(tk, tv, a, n_splits, Hkv, B, s);
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+
+extern "C" {
+
+const char* fd_status_string(fd_status status) {
+  switch (status) {
+    case FD_OK: return "FD_OK";
+    case FD_ERR_INVALID_ARGUMENT: return "FD_ERR_INVALID_ARGUMENT";
+    case FD_ERR_UNSUPPORTED: return "FD_ERR_UNSUPPORTED";
+    case FD_ERR_WORKSPACE: return "FD_ERR_WORKSPACE";
+    case FD_ERR_CUDA: return "FD_ERR_CUDA";
+    case FD_ERR_DEVICE_TIMEOUT: return "FD_ERR_DEVICE_TIMEOUT";
+  }
+  return "FD_ERR_UNKNOWN";
+}
+
+int fd_split_chunk(int max_len, int num_splits) {
+  if (max_len < 0 || num_splits < 1 || num_splits > kMaxSplits) return FD_ERR_INVALID_ARGUMENT;
+  return chunk_for(max_len, num_splits);
+}
+
+int fd_plan_sm(int num_sms, int B, int Hq, int Hkv, int D, int max_len, int block_size) {
+  if (num_sms < 1) return FD_ERR_INVALID_ARGUMENT;
+  const fd_status st = check_shape(B, Hq, Hkv, D, max_len, block_size);
+  if (st != FD_OK) return st;
+  const long long tiles = (static_cast<long long>(max_len) + fd::kTile - 1) / fd::kTile;
+  if (tiles <= 1) return 1;
+  // Enough (sequence, KV head) units to fill every CTA slot: no split.
+  if (static_cast<long long>(B) * Hkv >= static_cast<long long>(num_sms) * fd::kCtasPerSm) return 1;
+  const int s_max = static_cast<int>(std::min<long long>(tiles, kMaxSplits));
+  int best = 1;
+  double best_t = model_time_us(num_sms, B, Hq, Hkv, D, max_len, 1);
+  int last_eff = 1;
+  for (int S = 2; S <= s_max; ++S) {
+    const int eff = effective_splits(max_len, chunk_for(max_len, S));
+    if (eff == last_eff) continue;  // same chunking as a smaller S
+    last_eff = eff;
+    const double t = model_time_us(num_sms, B, Hq, Hkv, D, max_len, S);
+    if (t < best_t * 0.98) {  // prefer fewer splits unless clearly faster
+      best_t = t;
+      best = S;
+    }
+  }
+  return best;
+}
+
+int fd_plan(int B, int Hq, int Hkv, int D, int max_len, int block_size) {
+  const fd_status st = check_shape(B, Hq, Hkv, D, max_len, block_size);
+  if (st != FD_OK) return st;
+  int dev = 0, sms = 0;
+  if (current_device(&dev) != FD_OK || device_sms(dev, &sms) != FD_OK) return FD_ERR_CUDA;
+  return fd_plan_sm(sms, B, Hq, Hkv, D, max_len, block_size);
+}
+
+size_t fd_workspace_bytes(int B, int Hq, int D, int num_splits) {
+  if (B < 1 || Hq < 1 || D < 1 || num_splits < 1 || num_splits > kMaxSplits) return 0;
+  if (num_splits == 1) return 0;
+  const size_t rows = static_cast<size_t>(B) * Hq * num_splits;
+  return round256(rows * D * sizeof(float)) + round256(rows * sizeof(float));
+}
+
+fd_status fd_decode(const fd_problem* p, const void* q, const void* k_cache,
+                    const void* v_cache, const int32_t* seqlens, const int32_t* block_table,
+                    float scale, int num_splits, void* out, float* lse, void* workspace,
+                    size_t workspace_bytes, fd_stream_t stream) {
+  // ---- host-side checks: nothing is launched for an invalid call
+  if (!p || !q || !k_cache || !v_cache || !out) return FD_ERR_INVALID_ARGUMENT;
+  const fd_status st = check_shape(p->B, p->Hq, p->Hkv, p->D, p->max_len, p->block_size);
+  if (st != FD_OK) return st;
+  const bool paged = p->block_size != 0;
+  if (paged != (block_table != nullptr)) return FD_ERR_INVALID_ARGUMENT;
+  if (paged) {
+    if (p->num_blocks < 1 || p->max_blocks_per_seq < 1) return FD_ERR_INVALID_ARGUMENT;
+    if (static_cast<long long>(p->max_blocks_per_seq) * p->block_size < p->max_len)
+      return FD_ERR_INVALID_ARGUMENT;
+  }
+  if (!std::isfinite(scale) || !(scale > 0.f)) return FD_ERR_INVALID_ARGUMENT;
+  if (num_splits < 1 || num_splits > kMaxSplits) return FD_ERR_INVALID_ARGUMENT;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+      !aligned(lse, 4) || !aligned(workspace, 16) || !aligned(seqlens, 4) ||
+      !aligned(block_table, 4))
+    return FD_ERR_INVALID_ARGUMENT;
+
+  const int B = p->B, Hq = p->Hq, Hkv = p->Hkv, D = p->D, G = Hq / Hkv;
+  const int chunk = chunk_for(p->max_len, num_splits);
+  const int n_splits = effective_splits(p->max_len, chunk);
+  float* part_o = nullptr;
+  float* part_lse = nullptr;
+  if (n_splits > 1) {
+    const size_t need = fd_workspace_bytes(B, Hq, D, n_splits);
+    if (!workspace || workspace_bytes < need) return FD_ERR_WORKSPACE;
+    part_o = static_cast<float*>(workspace);
+    part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                        round256(static_cast<size_t>(B) * Hq * n_splits * D * 4));
+  }
+
+  int dev = 0;
+  if (current_device(&dev) != FD_OK) return FD_ERR_CUDA;
+  const fd_status arch = device_is_sm100(dev);
+  if (arch != FD_OK) return arch;
+
+  // ---- tensor maps over the caches
+  CUtensorMap tk, tv;
+  if (!paged) {
+    const long long planes = static_cast<long long>(B) * Hkv;
+    const long long rows = p->max_len > 0 ? p->max_len : 1;
+    if (make_cache_map(&tk, k_cache, D, rows, planes, fd::kTile) != FD_OK ||
+        make_cache_map(&tv, v_cache, D, rows, planes, fd::kTile) != FD_OK)
+      return FD_ERR_CUDA;
+  } else {
+    const long long planes = static_cast<long long>(p->num_blocks) * Hkv;
+    const int box_rows = std::min(p->block_size, fd::kTile);
+    if (make_cache_map(&tk, k_cache, D, p->block_size, planes, box_rows) != FD_OK ||
+        make_cache_map(&tv, v_cache, D, p->block_size, planes, box_rows) != FD_OK)
+      return FD_ERR_CUDA;
+  }
+
+  fd::SplitArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.seqlens = seqlens;
+  a.block_table = block_table;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.lse = lse;
+  a.part_o = part_o;
+  a.part_lse = part_lse;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.G = G;
+  a.max_len = p->max_len;
+  a.block_size = paged ? p->block_size : 0;
+  a.log2_block_size = paged ? ilog2(p->block_size) : 0;
+  a.max_blocks_per_seq = paged ? p->max_blocks_per_seq : 0;
+  a.chunk = chunk;
+  a.n_splits = n_splits;
+  a.scale_log2 = scale * 1.4426950408889634074f;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  fd_status r;
+  if (D == 128)
+    r = paged ? dispatch_split<128, true>(G, tk, tv, a, n_splits, Hkv, B, s)
+              : dispatch_split<128, false>(G, tk, tv, a, n_splits, Hkv, B, s);
+  else
+    r = paged ? dispatch_split<64, true>(G, tk, tv, a, n_splits, Hkv, B, s)
+              : dispatch_split<64, false>(G, tk, tv, a, n_splits, Hkv, B, s);
+  if (r != FD_OK) return r;
+
+  if (n_splits > 1) {
+    fd::CombineArgs c{};
+    c.part_o = part_o;
+    c.part_lse = part_lse;
+    c.seqlens = seqlens;
+    c.out = static_cast<__nv_bfloat16*>(out);
+    c.lse = lse;
+    c.B = B;
+    c.Hq = Hq;
+    c.max_len = p->max_len;
+    c.chunk = chunk;
+    c.n_splits = n_splits;
+    r = D == 128 ? launch_combine<128>(c, s) : launch_combine<64>(c, s);
+    if (r != FD_OK) return r;
+  }
+  return FD_OK;
+}
+
+fd_status fd_check_device_error(fd_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return FD_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, fd::g_error_word, sizeof word) != cudaSuccess)
+    return FD_ERR_CUDA;
+  if (word) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(fd::g_error_word, &zero, sizeof zero) != cudaSuccess)
+      return FD_ERR_CUDA;
+    return FD_ERR_DEVICE_TIMEOUT;
+  }
+  return FD_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,536 @@
+// fd_kernels.cuh — sm_100a kernels of split-KV decode attention.
+//
+// Split kernel: one CTA per (split, KV head, sequence).  It streams the
+// split's K/V tiles from HBM through a multi-stage shared-memory pipeline
+// fed by TMA tensor loads (128-byte swizzle), and runs the scores and the
+// P.V product for all G query heads of the KV head on the tensor cores
+// (bf16 mma.sync, fp32 accumulation), with an online softmax in between.
+// Each split ends with a partial output and a log-sum-exp ("What is
+// Flash-Decoding, and when does it speed up LLMs?", slavadubrov.com, section
+// "Why decode needs a different schedule").  The running maximum and
+// normaliser of the online softmax follow the FlashAttention-style streaming
+// described in the last abstract of scifaro.com's "Related papers:
+// INT-FlashAttention" list.
+//
+// Combine kernel: merges the partials of every (sequence, query head) with
+// the log-sum-exp weights m = max_s lse_s, O = sum_s e^(lse_s - m) O_s /
+// sum_s e^(lse_s - m), lse = m + ln sum_s e^(lse_s - m).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "fd_ptx.cuh"
+
+namespace fd {
+
+constexpr int kTile = 64;           // tokens per pipeline stage
+constexpr int kConsumerWarps = 4;   // each takes 16 tokens of every tile
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kCtasPerSm = 2;       // occupancy the split kernel is sized for
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
+
+// How the softmax weights P enter the bf16 P.V contraction.
+//  kDup : G <= 4.  Query heads fill columns 0..3 of the n=8 MMA and are
+//         duplicated into columns 4..7.  Columns 0..3 carry bf16(p), columns
+//         4..7 carry the rounding residual p - bf16(p); their sum restores p
+//         to ~16 bits at no extra MMA.
+//  kHiLo: G = 8 per column block.  A second P.V MMA adds the residual.
+//  kHi  : G = 8 per column block, bf16(p) only.
+enum PMode { kDup = 0, kHiLo = 1, kHi = 2 };
+
+// Device error word: set when a bounded wait runs out.
+__device__ unsigned int g_error_word;
+
+struct SplitArgs {
+  const __nv_bfloat16* q;       // [B, Hq, D]
+  const int32_t* seqlens;       // [B] or null
+  const int32_t* block_table;   // [B, max_blocks_per_seq] or null
+  __nv_bfloat16* out;           // [B, Hq, D]          (one split)
+  float* lse;                   // [B, Hq] or null     (one split)
+  float* part_o;                // [B, Hq, S, D]       (several splits)
+  float* part_lse;              // [B, Hq, S]          (several splits)
+  int Hq, Hkv, G;
+  int max_len;
+  int block_size, log2_block_size;
+  int max_blocks_per_seq;
+  int chunk;                    // tokens per split, a multiple of kTile
+  int n_splits;                 // effective split count = gridDim.x
+  float scale_log2;             // scale * log2(e)
+};
+
+struct CombineArgs {
+  const float* part_o;
+  const float* part_lse;
+  const int32_t* seqlens;
+  __nv_bfloat16* out;
+  float* lse;
+  int B, Hq, max_len, chunk, n_splits;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float round_to_bf16(float x) {
+  return __bfloat162float(__float2bfloat16_rn(x));
+}
+
+__device__ __forceinline__ int seq_length(const int32_t* seqlens, int b, int max_len) {
+  int n = seqlens ? seqlens[b] : max_len;
+  return n < 0 ? 0 : (n > max_len ? max_len : n);
+}
+
+__device__ __forceinline__ void raise_device_error(unsigned int code) {
+  atomicOr(&g_error_word, code);
+}
+
+template <int D, int STAGES>
+struct SplitSmem {
+  static constexpr int kHalves = D / 64;               // 128-byte swizzle rows
+  static constexpr int kHalfBytes = kTile * 128;       // one 64-column half tile
+  static constexpr int kTileBytes = kHalves * kHalfBytes;
+  static constexpr int kStageBytes = 2 * kTileBytes;   // K tile + V tile
+  static constexpr int kBarOffset = STAGES * kStageBytes;
+  static constexpr int kBytes = kBarOffset + 2 * STAGES * 8 + 16;
+  static constexpr int kDynamicBytes = kBytes + 1024;  // room to align to 1 KB
+};
+
+template <int D, int NB, int MODE, bool PAGED, int STAGES>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    fd_split_kernel(const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const SplitArgs a) {
+  using L = SplitSmem<D, STAGES>;
+  constexpr int KSTEPS = D / 16;   // k-steps of the score MMA (over D)
+  constexpr int DBLK = D / 16;     // m-blocks of the P.V MMA (over D)
+  constexpr int NCOL = NB * 8;     // MMA columns (query heads, maybe doubled)
+  static_assert(MODE != kDup || NB == 1, "duplicated columns need one column block");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t smem_base = smem_u32(smem);
+  const uint32_t bar_full = smem_base + L::kBarOffset;
+  const uint32_t bar_empty = bar_full + STAGES * 8;
+  volatile int* cta_error = reinterpret_cast<volatile int*>(smem + L::kBarOffset + 2 * STAGES * 8);
+
+  const int split = blockIdx.x;
+  const int kvh = blockIdx.y;
+  const int b = blockIdx.z;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, kConsumerWarps);
+    }
+    *cta_error = 0;
+    fence_mbar_init();
+  }
+  if (warp == kConsumerWarps && lane == 0) {
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmV);
+  }
+  __syncthreads();
+
+  // Inputs may be produced by the previous kernel on the stream.
+  grid_dependency_wait();
+  grid_dependents_launch();
+
+  const int n = seq_length(a.seqlens, b, a.max_len);
+  const int start = split * a.chunk;
+  const int end = min(start + a.chunk, n);
+  const int h0 = kvh * a.G;
+
+  if (start >= end) {
+    // Empty split.  With several splits the combine kernel skips it; with one
+    // split the sequence is empty: out = 0, lse = -inf.
+    if (a.n_splits == 1) {
+      for (int i = threadIdx.x; i < a.G * D; i += kThreads)
+        a.out[(static_cast<size_t>(b) * a.Hq + h0) * D + i] = __float2bfloat16_rn(0.f);
+      if (a.lse && threadIdx.x < a.G) a.lse[static_cast<size_t>(b) * a.Hq + h0 + threadIdx.x] = -INFINITY;
+    }
+    return;
+  }
+  const int n_tiles = (end - start + kTile - 1) / kTile;
+
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------- producer
+    const uint64_t policy = policy_evict_first();
+    int issued = 0;
+    bool ok = true;
+    if constexpr (!PAGED) {
+      const int plane = b * a.Hkv + kvh;
+      for (int it = 0; it < n_tiles; ++it) {
+        const int s = it % STAGES, k = it / STAGES;
+        if (k > 0 && !mbar_wait(bar_empty + 8 * s, (k - 1) & 1, kWaitLimitNs)) { ok = false; break; }
+        if (lane == 0) {
+          const int t0 = start + it * kTile;
+          const uint32_t dk = smem_base + s * L::kStageBytes;
+          const uint32_t dv = dk + L::kTileBytes;
+          mbar_arrive_expect_tx(bar_full + 8 * s, L::kStageBytes);
+#pragma unroll
+          for (int hf = 0; hf < L::kHalves; ++hf) {
+            tma_load_3d(dk + hf * L::kHalfBytes, &tmK, bar_full + 8 * s, hf * 64, t0, plane, policy);
+            tma_load_3d(dv + hf * L::kHalfBytes, &tmV, bar_full + 8 * s, hf * 64, t0, plane, policy);
+          }
+        }
+        ++issued;
+        __syncwarp();
+      }
+    } else {
+      const int bs = a.block_size, lbs = a.log2_block_size;
+      const int rows = bs < kTile ? bs : kTile;            // rows per TMA box
+      const int pages_per_tile = bs < kTile ? kTile / bs : 1;
+      const int n_pages = (n + bs - 1) >> lbs;
+      const int32_t* bt = a.block_table + static_cast<size_t>(b) * a.max_blocks_per_seq;
+      // A window of 32 page ids, one per lane, plus the next window in flight.
+      int win = start >> lbs;
+      int cur = (win + lane < n_pages) ? __ldg(bt + win + lane) : 0;
+      int nxt = (win + 32 + lane < n_pages) ? __ldg(bt + win + 32 + lane) : 0;
+      for (int it = 0; it < n_tiles; ++it) {
+        const int s = it % STAGES, k = it / STAGES;
+        if (k > 0 && !mbar_wait(bar_empty + 8 * s, (k - 1) & 1, kWaitLimitNs)) { ok = false; break; }
+        const int t0 = start + it * kTile;
+        const int pg = t0 >> lbs;
+        if (pg >= win + 32) {
+          win += 32;
+          cur = nxt;
+          nxt = (win + 32 + lane < n_pages) ? __ldg(bt + win + 32 + lane) : 0;
+        }
+        const int row0 = bs > kTile ? (t0 & (bs - 1)) : 0;
+        const int valid_pages = min(pages_per_tile, n_pages - pg);
+        const uint32_t dk = smem_base + s * L::kStageBytes;
+        const uint32_t dv = dk + L::kTileBytes;
+        int pid[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) pid[j] = __shfl_sync(0xffffffffu, cur, (pg - win + j) & 31);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar_full + 8 * s,
+                                valid_pages * rows * 128 * L::kHalves * 2);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (j < valid_pages) {
+              const int plane = pid[j] * a.Hkv + kvh;
+#pragma unroll
+              for (int hf = 0; hf < L::kHalves; ++hf) {
+                const uint32_t off = hf * L::kHalfBytes + j * rows * 128;
+                tma_load_3d(dk + off, &tmK, bar_full + 8 * s, hf * 64, row0, plane, policy);
+                tma_load_3d(dv + off, &tmV, bar_full + 8 * s, hf * 64, row0, plane, policy);
+              }
+            }
+          }
+        }
+        ++issued;
+        __syncwarp();
+      }
+    }
+    if (!ok && lane == 0) {
+      raise_device_error(1u);
+      *cta_error = 1;
+    }
+    // No copy may still be landing in shared memory when the CTA retires.
+    if (lane == 0) {
+      for (int it = issued > STAGES ? issued - STAGES : 0; it < issued; ++it)
+        if (!mbar_wait(bar_full + 8 * (it % STAGES), (it / STAGES) & 1, kWaitLimitNs))
+          raise_device_error(2u);
+    }
+    return;
+  }
+
+  // --------------------------------------------------------------- consumers
+  // B fragments of Q^T (k = head dim, n = query head), loaded once.
+  uint32_t qf[NB][KSTEPS][2];
+  {
+    const int ncol = lane >> 2;
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      const int head = MODE == kDup ? (ncol & 3) : nb * 8 + ncol;
+      const bool live = head < a.G;
+      const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+          a.q + (static_cast<size_t>(b) * a.Hq + h0 + (live ? head : 0)) * D);
+#pragma unroll
+      for (int ks = 0; ks < KSTEPS; ++ks) {
+        qf[nb][ks][0] = live ? qrow[ks * 8 + (lane & 3)] : 0u;
+        qf[nb][ks][1] = live ? qrow[ks * 8 + 4 + (lane & 3)] : 0u;
+      }
+    }
+  }
+
+  float m_run[NB][2], l_run[NB][2];
+  float acc[NB][DBLK][4];
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) {
+    m_run[nb][0] = m_run[nb][1] = -INFINITY;
+    l_run[nb][0] = l_run[nb][1] = 0.f;
+#pragma unroll
+    for (int db = 0; db < DBLK; ++db)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[nb][db][i] = 0.f;
+  }
+
+  // Row of the 16-token slice this lane addresses for ldmatrix, and its
+  // 128-byte swizzle phase (row mod 8).
+  const uint32_t rowK = warp * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+  const uint32_t rowV = warp * 16 + (lane >> 4) * 8 + (lane & 7);
+  const uint32_t x7 = lane & 7;
+  const int r_lo = warp * 16 + (lane >> 2);   // token rows of the C fragment
+  const int r_hi = r_lo + 8;
+  const float sl2 = a.scale_log2;
+  bool failed = false;
+
+  for (int it = 0; it < n_tiles; ++it) {
+    const int s = it % STAGES, k = it / STAGES;
+    if (!mbar_wait(bar_full + 8 * s, k & 1, kWaitLimitNs)) {
+      failed = true;
+      break;
+    }
+    const uint32_t kbase = smem_base + s * L::kStageBytes;
+    const uint32_t vbase = kbase + L::kTileBytes;
+    const int tile_valid = min(kTile, end - (start + it * kTile));
+    const bool partial = tile_valid < kTile;
+
+    // S^T = K Q^T for this warp's 16 tokens (two chains for ILP).
+    float sc[NB][2][4];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sc[nb][c][i] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < KSTEPS; ++ks) {
+      const uint32_t chunk16 = ((ks & 3) << 1) + (lane >> 4);
+      const uint32_t addr = kbase + (ks >> 2) * L::kHalfBytes + rowK * 128 + ((chunk16 ^ x7) << 4);
+      uint32_t af[4];
+      ldmatrix_x4(addr, af[0], af[1], af[2], af[3]);
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) mma_bf16_16816(sc[nb][ks & 1], af, qf[nb][ks][0], qf[nb][ks][1]);
+    }
+
+    // Online softmax in the log2 domain; this lane holds tokens r_lo, r_hi
+    // and columns 2*(lane&3), 2*(lane&3)+1.
+    uint32_t pb[NB][2];
+    uint32_t plo[NB][2];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      float t[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) t[i] = (sc[nb][0][i] + sc[nb][1][i]) * sl2;
+      if (partial) {
+        if (r_lo >= tile_valid) t[0] = t[1] = -INFINITY;
+        if (r_hi >= tile_valid) t[2] = t[3] = -INFINITY;
+      }
+      float mx0 = fmaxf(t[0], t[2]), mx1 = fmaxf(t[1], t[3]);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+      }
+      const float mn0 = fmaxf(m_run[nb][0], mx0), mn1 = fmaxf(m_run[nb][1], mx1);
+      const float mu0 = mn0 == -INFINITY ? 0.f : mn0;
+      const float mu1 = mn1 == -INFINITY ? 0.f : mn1;
+      const float al0 = ex2(m_run[nb][0] - mu0), al1 = ex2(m_run[nb][1] - mu1);
+      const float p0 = ex2(t[0] - mu0), p1 = ex2(t[1] - mu1);
+      const float p2 = ex2(t[2] - mu0), p3 = ex2(t[3] - mu1);
+      l_run[nb][0] = l_run[nb][0] * al0 + (p0 + p2);
+      l_run[nb][1] = l_run[nb][1] * al1 + (p1 + p3);
+      m_run[nb][0] = mn0;
+      m_run[nb][1] = mn1;
+      if (__any_sync(0xffffffffu, (al0 != 1.f) | (al1 != 1.f))) {
+#pragma unroll
+        for (int db = 0; db < DBLK; ++db) {
+          acc[nb][db][0] *= al0;
+          acc[nb][db][1] *= al1;
+          acc[nb][db][2] *= al0;
+          acc[nb][db][3] *= al1;
+        }
+      }
+      if constexpr (MODE == kDup) {
+        // Columns 4..7 (lanes with lane&3 >= 2) carry the bf16 residual.
+        const bool lo_lane = (lane & 2) != 0;
+        const float e0 = lo_lane ? p0 - round_to_bf16(p0) : p0;
+        const float e1 = lo_lane ? p1 - round_to_bf16(p1) : p1;
+        const float e2 = lo_lane ? p2 - round_to_bf16(p2) : p2;
+        const float e3 = lo_lane ? p3 - round_to_bf16(p3) : p3;
+        pb[nb][0] = movmatrix_trans(pack_bf16x2(e0, e1));
+        pb[nb][1] = movmatrix_trans(pack_bf16x2(e2, e3));
+      } else {
+        pb[nb][0] = movmatrix_trans(pack_bf16x2(p0, p1));
+        pb[nb][1] = movmatrix_trans(pack_bf16x2(p2, p3));
+        if constexpr (MODE == kHiLo) {
+          plo[nb][0] = movmatrix_trans(
+              pack_bf16x2(p0 - round_to_bf16(p0), p1 - round_to_bf16(p1)));
+          plo[nb][1] = movmatrix_trans(
+              pack_bf16x2(p2 - round_to_bf16(p2), p3 - round_to_bf16(p3)));
+        }
+      }
+    }
+
+    // O^T += V^T P^T for this warp's 16 tokens.
+    uint32_t vmask_lo = 0xffffffffu, vmask_hi = 0xffffffffu;
+    if (partial) {
+      const int tk = warp * 16 + 2 * (lane & 3);
+      vmask_lo = (tk < tile_valid ? 0x0000ffffu : 0u) | (tk + 1 < tile_valid ? 0xffff0000u : 0u);
+      vmask_hi = (tk + 8 < tile_valid ? 0x0000ffffu : 0u) | (tk + 9 < tile_valid ? 0xffff0000u : 0u);
+    }
+#pragma unroll
+    for (int db = 0; db < DBLK; ++db) {
+      const uint32_t chunk16 = ((db & 3) << 1) + ((lane >> 3) & 1);
+      const uint32_t addr = vbase + (db >> 2) * L::kHalfBytes + rowV * 128 + ((chunk16 ^ x7) << 4);
+      uint32_t vf[4];
+      ldmatrix_x4_trans(addr, vf[0], vf[1], vf[2], vf[3]);
+      // Rows past the valid length may hold anything (NaN included): zero them
+      // so that 0 * NaN never reaches the accumulator.
+      vf[0] &= vmask_lo;
+      vf[1] &= vmask_lo;
+      vf[2] &= vmask_hi;
+      vf[3] &= vmask_hi;
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        mma_bf16_16816(acc[nb][db], vf, pb[nb][0], pb[nb][1]);
+        if constexpr (MODE == kHiLo) mma_bf16_16816(acc[nb][db], vf, plo[nb][0], plo[nb][1]);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_empty + 8 * s);
+  }
+
+  if (failed) {
+    if (lane == 0) {
+      raise_device_error(1u);
+      *cta_error = 1;
+    }
+  }
+
+  // Row sums: lanes sharing a column hold disjoint tokens.
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1)
+        l_run[nb][j] += __shfl_xor_sync(0xffffffffu, l_run[nb][j], off);
+
+  // Every consumer warp is past its last shared-memory read of the pipeline.
+  named_barrier_sync(1, kConsumerWarps * 32);
+  if (*cta_error) return;
+
+  // Merge the four warps' partial softmax states through shared memory
+  // (the pipeline buffers are free: every issued tile has landed and been read).
+  float* red_acc = reinterpret_cast<float*>(smem);                 // [warp][NCOL][D]
+  float* red_m = red_acc + kConsumerWarps * NCOL * D;               // [warp][NCOL]
+  float* red_l = red_m + kConsumerWarps * NCOL;                     // [warp][NCOL]
+  {
+    const int j0 = 2 * (lane & 3);
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      float* base = red_acc + (warp * NCOL + nb * 8 + j0) * D;
+#pragma unroll
+      for (int db = 0; db < DBLK; ++db) {
+        const int d = db * 16 + (lane >> 2);
+        base[d] = acc[nb][db][0];
+        base[D + d] = acc[nb][db][1];
+        base[d + 8] = acc[nb][db][2];
+        base[D + d + 8] = acc[nb][db][3];
+      }
+      if (lane < 4) {
+        red_m[warp * NCOL + nb * 8 + j0] = m_run[nb][0];
+        red_m[warp * NCOL + nb * 8 + j0 + 1] = m_run[nb][1];
+        red_l[warp * NCOL + nb * 8 + j0] = l_run[nb][0];
+        red_l[warp * NCOL + nb * 8 + j0 + 1] = l_run[nb][1];
+      }
+    }
+  }
+  named_barrier_sync(1, kConsumerWarps * 32);
+
+  const int t = threadIdx.x;
+  for (int idx = t; idx < a.G * D; idx += kConsumerWarps * 32) {
+    const int g = idx / D, d = idx - (idx / D) * D;
+    const int col = g;  // head g lives in column g (kDup adds column g + 4)
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red_m[w * NCOL + col]);
+    float Lsum = 0.f, O = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      const float wt = ex2(red_m[w * NCOL + col] - M);
+      Lsum += wt * red_l[w * NCOL + col];
+      float v = red_acc[(w * NCOL + col) * D + d];
+      if constexpr (MODE == kDup) v += red_acc[(w * NCOL + col + 4) * D + d];
+      O += wt * v;
+    }
+    O = O / Lsum;
+    const float lse_val = (M + log2f(Lsum)) * 0.69314718055994530942f;
+    const size_t row = static_cast<size_t>(b) * a.Hq + h0 + g;
+    if (a.n_splits == 1) {
+      a.out[row * D + d] = __float2bfloat16_rn(O);
+      if (d == 0 && a.lse) a.lse[row] = lse_val;
+    } else {
+      a.part_o[(row * a.n_splits + split) * D + d] = O;
+      if (d == 0) a.part_lse[row * a.n_splits + split] = lse_val;
+    }
+  }
+}
+
+// One warp per (sequence, query head); lanes cover D with vector loads.
+template <int D>
+__global__ void __launch_bounds__(128) fd_combine_kernel(const CombineArgs a) {
+  constexpr int VPL = D / 32;  // values per lane (4 or 2)
+  grid_dependency_wait();      // partials come from the split kernel
+  const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= a.B * a.Hq) return;
+  const int b = row / a.Hq;
+  const int n = seq_length(a.seqlens, b, a.max_len);
+  int ns = (n + a.chunk - 1) / a.chunk;
+  ns = ns < a.n_splits ? ns : a.n_splits;
+  __nv_bfloat16* orow = a.out + static_cast<size_t>(row) * D + lane * VPL;
+  if (ns == 0) {
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) orow[i] = __float2bfloat16_rn(0.f);
+    if (a.lse && lane == 0) a.lse[row] = -INFINITY;
+    return;
+  }
+  const float* pl = a.part_lse + static_cast<size_t>(row) * a.n_splits;
+  const float* po = a.part_o + static_cast<size_t>(row) * a.n_splits * D + lane * VPL;
+  float mx = -INFINITY;
+  for (int s = lane; s < ns; s += 32) mx = fmaxf(mx, pl[s]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  constexpr float kLog2e = 1.4426950408889634074f;
+  float accv[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) accv[i] = 0.f;
+  float W = 0.f;
+#pragma unroll 4
+  for (int s = 0; s < ns; ++s) {
+    const float w = ex2((pl[s] - mx) * kLog2e);
+    W += w;
+    if constexpr (VPL == 4) {
+      const float4 o = *reinterpret_cast<const float4*>(po + static_cast<size_t>(s) * D);
+      accv[0] += w * o.x;
+      accv[1] += w * o.y;
+      accv[2] += w * o.z;
+      accv[3] += w * o.w;
+    } else {
+      const float2 o = *reinterpret_cast<const float2*>(po + static_cast<size_t>(s) * D);
+      accv[0] += w * o.x;
+      accv[1] += w * o.y;
+    }
+  }
+  const float inv = 1.f / W;
+  if constexpr (VPL == 4) {
+    uint2 pk;
+    pk.x = pack_bf16x2(accv[0] * inv, accv[1] * inv);
+    pk.y = pack_bf16x2(accv[2] * inv, accv[3] * inv);
+    *reinterpret_cast<uint2*>(orow) = pk;
+  } else {
+    *reinterpret_cast<uint32_t*>(orow) = pack_bf16x2(accv[0] * inv, accv[1] * inv);
+  }
+  if (a.lse && lane == 0) a.lse[row] = mx + logf(W);
+}
+
+}  // namespace fd

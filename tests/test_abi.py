@@ -1,0 +1,168 @@
+"""The C-ABI library on the host: it loads, exports every entry point that
+include/fd.h declares, and its host logic (planner, chunking, workspace
+sizing, argument checks) behaves as documented.  No kernel is launched here:
+every fd_decode call below is invalid for a reason the host checks before any
+CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import split_kv_decode_attn_b200 as fd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_entry_points():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"FD_API\s+[\w\s\*]*?\b(fd_\w+)\s*\(", text)
+    return names
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_entry_points()
+    assert len(names) >= 7
+    lib = fd.load_library()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(fd.EXPORTS)
+
+
+def test_status_strings():
+    assert fd.fd_status_string(fd.FD_OK) == "FD_OK"
+    assert fd.fd_status_string(fd.FD_ERR_WORKSPACE) == "FD_ERR_WORKSPACE"
+    assert fd.fd_status_string(fd.FD_ERR_DEVICE_TIMEOUT) == "FD_ERR_DEVICE_TIMEOUT"
+    assert fd.fd_status_string(12345) == "FD_ERR_UNKNOWN"
+
+
+@pytest.mark.parametrize("L,S,chunk", [(512, 1, 512), (512, 2, 256), (512, 8, 64), (512, 64, 64),
+                                       (1000, 3, 384), (65536, 37, 1792), (1, 1, 64),
+                                       (0, 4, 64), (262144, 37, 7104)])
+def test_split_chunk(L, S, chunk):
+    assert fd.fd_split_chunk(L, S) == chunk
+    assert chunk % 64 == 0
+
+
+def test_split_chunk_invalid():
+    assert fd.fd_split_chunk(-1, 2) == fd.FD_ERR_INVALID_ARGUMENT
+    assert fd.fd_split_chunk(100, 0) == fd.FD_ERR_INVALID_ARGUMENT
+    assert fd.fd_split_chunk(100, 1025) == fd.FD_ERR_INVALID_ARGUMENT
+
+
+def test_workspace_bytes():
+    assert fd.fd_workspace_bytes(1, 64, 128, 1) == 0
+    B, Hq, D, S = 1, 64, 128, 37
+    rows = B * Hq * S
+    expect = (rows * D * 4 + 255) // 256 * 256 + (rows * 4 + 255) // 256 * 256
+    assert fd.fd_workspace_bytes(B, Hq, D, S) == expect
+    assert fd.fd_workspace_bytes(0, 64, 128, 2) == 0
+    assert fd.fd_workspace_bytes(1, 64, 128, 0) == 0
+
+
+B200_SMS = 148
+
+
+def test_plan_large_batch_does_not_split():
+    # B*Hkv = 256 + 64 units >= 2 CTAs per SM on 148 SMs: enough work already
+    assert fd.fd_plan_sm(B200_SMS, 40, 32, 8, 128, 32768, 0) == 1
+
+
+def test_plan_short_history_does_not_split():
+    assert fd.fd_plan_sm(B200_SMS, 1, 64, 8, 128, 64, 0) == 1
+    assert fd.fd_plan_sm(B200_SMS, 1, 64, 8, 128, 1, 0) == 1
+    assert fd.fd_plan_sm(B200_SMS, 1, 64, 8, 128, 0, 0) == 1
+
+
+def test_plan_long_history_fills_the_device():
+    for L in (16384, 32768, 65536, 262144):
+        S = fd.fd_plan_sm(B200_SMS, 1, 64, 8, 128, L, 0)
+        chunk = fd.fd_split_chunk(L, S)
+        s_eff = -(-L // chunk)
+        ctas = 8 * s_eff
+        assert ctas >= 0.9 * B200_SMS, (L, S, ctas)
+        assert ctas <= 4 * 2 * B200_SMS, (L, S, ctas)
+
+
+def test_plan_splits_grow_with_length_and_are_deterministic():
+    prev = 1
+    for L in (512, 2048, 8192, 16384, 65536):
+        S = fd.fd_plan_sm(B200_SMS, 1, 64, 8, 128, L, 0)
+        assert S >= 1 and S == fd.fd_plan_sm(B200_SMS, 1, 64, 8, 128, L, 0)
+        assert S >= prev or S > 8
+        prev = S
+
+
+def test_plan_invalid_and_unsupported():
+    assert fd.fd_plan_sm(B200_SMS, 1, 6, 4, 128, 100, 0) == fd.FD_ERR_INVALID_ARGUMENT
+    assert fd.fd_plan_sm(B200_SMS, 0, 8, 8, 128, 100, 0) == fd.FD_ERR_INVALID_ARGUMENT
+    assert fd.fd_plan_sm(B200_SMS, 1, 8, 8, 96, 100, 0) == fd.FD_ERR_UNSUPPORTED
+    assert fd.fd_plan_sm(B200_SMS, 1, 24, 1, 128, 100, 0) == fd.FD_ERR_UNSUPPORTED  # G = 24
+    assert fd.fd_plan_sm(B200_SMS, 1, 8, 8, 128, 100, 24) == fd.FD_ERR_UNSUPPORTED
+    assert fd.fd_plan_sm(B200_SMS, 1, 8, 8, 128, 100, 4) == fd.FD_ERR_UNSUPPORTED
+    assert fd.fd_plan_sm(0, 1, 8, 8, 128, 100, 0) == fd.FD_ERR_INVALID_ARGUMENT
+
+
+# fd_decode rejections.  Fake, never-dereferenced addresses (16-byte aligned).
+Q, K, V, O, W = 0x10000, 0x20000, 0x30000, 0x40000, 0x50000
+
+
+def decode(prob, q=Q, k=K, v=V, seqlens=None, table=None, scale=0.125, S=1, out=O, lse=None,
+           ws=None, wsb=0):
+    return fd.load_library().fd_decode(
+        ctypes.byref(prob) if prob is not None else None, q, k, v, seqlens, table,
+        ctypes.c_float(scale), S, out, lse, ws, wsb, None)
+
+
+def P(B=1, Hq=8, Hkv=8, D=128, L=512, bs=0, nb=0, mb=0):
+    return fd.make_problem(B, Hq, Hkv, D, L, bs, nb, mb)
+
+
+def test_decode_rejects_nulls():
+    assert decode(None) == fd.FD_ERR_INVALID_ARGUMENT
+    assert decode(P(), q=None) == fd.FD_ERR_INVALID_ARGUMENT
+    assert decode(P(), k=None) == fd.FD_ERR_INVALID_ARGUMENT
+    assert decode(P(), out=None) == fd.FD_ERR_INVALID_ARGUMENT
+
+
+def test_decode_rejects_bad_shapes():
+    assert decode(P(Hq=12, Hkv=8)) == fd.FD_ERR_INVALID_ARGUMENT
+    assert decode(P(B=0)) == fd.FD_ERR_INVALID_ARGUMENT
+    assert decode(P(L=-1)) == fd.FD_ERR_INVALID_ARGUMENT
+    assert decode(P(D=256)) == fd.FD_ERR_UNSUPPORTED
+    assert decode(P(Hq=64, Hkv=2)) == fd.FD_ERR_UNSUPPORTED  # G = 32
+
+
+def test_decode_rejects_bad_paging():
+    # a block table without a block size, and a block size without a table
+    assert decode(P(), table=0x60000) == fd.FD_ERR_INVALID_ARGUMENT
+    assert decode(P(bs=16, nb=64, mb=32)) == fd.FD_ERR_INVALID_ARGUMENT
+    # table too short for max_len
+    assert decode(P(bs=16, nb=64, mb=8, L=512), table=0x60000) == fd.FD_ERR_INVALID_ARGUMENT
+    assert decode(P(bs=12, nb=64, mb=64), table=0x60000) == fd.FD_ERR_UNSUPPORTED
+
+
+def test_decode_rejects_bad_scalars():
+    assert decode(P(), scale=0.0) == fd.FD_ERR_INVALID_ARGUMENT
+    assert decode(P(), scale=-1.0) == fd.FD_ERR_INVALID_ARGUMENT
+    assert decode(P(), scale=float("nan")) == fd.FD_ERR_INVALID_ARGUMENT
+    assert decode(P(), scale=float("inf")) == fd.FD_ERR_INVALID_ARGUMENT
+    assert decode(P(), S=0) == fd.FD_ERR_INVALID_ARGUMENT
+    assert decode(P(), S=1025) == fd.FD_ERR_INVALID_ARGUMENT
+
+
+def test_decode_rejects_misaligned_pointers():
+    assert decode(P(), q=Q + 2) == fd.FD_ERR_INVALID_ARGUMENT
+    assert decode(P(), k=K + 8) == fd.FD_ERR_INVALID_ARGUMENT
+    assert decode(P(), out=O + 4) == fd.FD_ERR_INVALID_ARGUMENT
+    assert decode(P(), lse=0x70002) == fd.FD_ERR_INVALID_ARGUMENT
+
+
+def test_decode_rejects_missing_workspace():
+    # 8 splits of a 512-token history need partials
+    assert decode(P(), S=8) == fd.FD_ERR_WORKSPACE
+    need = fd.fd_workspace_bytes(1, 8, 128, 8)
+    assert decode(P(), S=8, ws=W, wsb=need - 1) == fd.FD_ERR_WORKSPACE
