@@ -1,0 +1,491 @@
+#!/usr/bin/env python
+"""Benchmark of split-KV decode attention on B200.
+
+One step is one fd_decode call (split kernel plus combine kernel) over one
+batch: by default the CodeLlama-34B-shaped per-layer decode (B=1, Hq=64,
+Hkv=8, D=128, bf16 cache of 65,536 tokens) with the planner's split count.
+The timed region holds exactly --steps calls, bracketed by a barrier and a
+device synchronisation, timed with CUDA events on the launching stream.
+Cache copies rotate between steps so that L2 never serves K/V.
+
+Reported (one JSON line from rank 0):
+  value        KV-read GB/s summed over ranks (algorithmic K+V bytes / time)
+  us_per_call  microseconds per fd_decode call
+  roofline     achieved GB/s of the call against the measured HBM copy peak
+  e2e          the same metric through the C ABI from pinned host buffers,
+               host<->device copies inside the timed region
+  cpu_baseline the fp64 oracle on this host's cores, on a bounded sample
+  sweep        the same call at cache lengths 512 .. 64K
+
+Multi-GPU (torchrun, one rank per GPU): every rank decodes its own batch
+(independent sequences; the path needs no collective), weak scaling.
+
+--impl reference times the fp64 CPU oracle instead (the slow reference of
+what the method computes), on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attention µs/call and KV-read GB/s (fraction of B200 HBM roofline)"
+FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0
+
+WORKLOADS = {
+    # name: (config index, cache length)
+    "codellama34b": (2, 65536),
+    "tiny": (1, None),
+    "varlen": (3, None),
+    "paged": (4, None),
+    "peaked": (5, None),
+}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40000)
+    ap.add_argument("--warmup", type=int, default=500)
+    ap.add_argument("--impl", choices=["fd", "reference"], default="fd")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="codellama34b")
+    ap.add_argument("--L", type=int, default=None, help="cache length of the codellama34b workload")
+    ap.add_argument("--splits", type=int, default=None, help="override the planner's split count")
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="CPU time budget of the oracle baseline sample")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- helpers
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "split_kv_decode_attn_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str):
+    """Per-launch DRAM bytes of the split kernel from the committed ncu summary,
+    if it was taken on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        if j.get("source_hash") != kernel_source_hash():
+            return None
+        entry = j.get("workloads", {}).get(workload)
+        return None if entry is None else float(entry["bytes_per_call"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        import torch
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            gid = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            gid = None
+        self.gid = gid
+
+    def start(self):
+        if not self.gid:
+            return
+        fd_, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd_)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gid}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.strip().split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"samples": 0}
+        sm = [float(r[0]) for r in rows]
+        mx = [float(r[1]) for r in rows]
+        util = [float(r[3]) if r[3].replace(".", "").isdigit() else 0.0 for r in rows]
+        loaded = [s for s, u in zip(sm, util) if u > 0] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx), "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[2]) for r in rows)}
+
+
+# ------------------------------------------------------------- our arm
+
+def dev_bf16(torch, a, device):
+    import numpy as np
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(torch.bfloat16)
+
+
+class Call:
+    """Device buffers and a bound fd_decode call for one workload; `copies`
+    rotating cache copies keep L2 from serving K/V."""
+
+    def __init__(self, torch, fd, w, device, num_splits=None, copies=1):
+        self.torch, self.fd, self.w = torch, fd, w
+        self.q = dev_bf16(torch, w.q, device)
+        k = dev_bf16(torch, w.k, device)
+        v = dev_bf16(torch, w.v, device)
+        self.ks = [k] + [k.clone() for _ in range(copies - 1)]
+        self.vs = [v] + [v.clone() for _ in range(copies - 1)]
+        self.seqlens = None if w.seqlens is None else torch.from_numpy(w.seqlens).to(device)
+        self.table = None if w.block_table is None else torch.from_numpy(w.block_table).to(device)
+        self.prob = fd.make_problem(w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size, w.num_blocks,
+                                    w.max_blocks_per_seq)
+        self.S = num_splits or fd.fd_plan(w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size)
+        assert self.S >= 1, fd.fd_status_string(self.S)
+        chunk = fd.fd_split_chunk(w.max_len, self.S)
+        self.s_eff = max(1, -(-w.max_len // chunk)) if w.max_len else 1
+        self.out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=device)
+        self.wbytes = fd.fd_workspace_bytes(w.B, w.Hq, w.D, self.S)
+        self.ws = torch.empty(max(self.wbytes, 4) // 4, dtype=torch.float32, device=device)
+        self.stream = torch.cuda.current_stream(device).cuda_stream
+        self.i = 0
+        self.launches_per_call = 2 if self.s_eff > 1 else 1
+
+    def __call__(self, k=None, v=None, q=None):
+        c = self.i % len(self.ks)
+        self.i += 1
+        st = self.fd.fd_decode(self.prob, q if q is not None else self.q,
+                               k if k is not None else self.ks[c], v if v is not None else self.vs[c],
+                               self.seqlens, self.table, self.w.scale, self.S, self.out, self.lse,
+                               self.ws, self.wbytes, self.stream)
+        if st != 0:
+            raise RuntimeError(f"fd_decode: {self.fd.fd_status_string(st)}")
+
+
+def timed(torch, fn, steps, warmup, barrier=None):
+    for _ in range(warmup):
+        fn()
+    if barrier:
+        barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    return e0.elapsed_time(e1)  # ms
+
+
+def copies_for(torch, nbytes, device):
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    return max(2, math.ceil(4 * l2 / max(nbytes, 1))), l2
+
+
+def make_workload(name, L, rank, nthreads=None):
+    from split_kv_decode_attn_b200 import workloads as wl
+    idx, default_L = WORKLOADS[name]
+    if idx == 2:
+        w = wl.config(2, L=L or default_L, nthreads=nthreads)
+    else:
+        w = wl.config(idx, nthreads=nthreads)
+    if rank:
+        # replicas: each rank decodes its own sequences (same shapes)
+        w2 = wl.make_problem(w.B, w.Hq, w.Hkv, w.D, w.max_len, wl.CONFIG_SEED_BASE + 1000 * rank + idx,
+                             seqlens=w.seqlens, nan_pad=w.seqlens is not None and not w.paged,
+                             block_size=w.block_size, name=w.name, nthreads=nthreads)
+        w = w2
+    return w
+
+
+def cpu_baseline(w, seconds):
+    """The fp64 oracle, as it stands, on this host's cores: one sequence per
+    oracle call (all its query heads, threads over heads), cycling through
+    the batch until `seconds` of wall time have passed.  GB/s of algorithmic
+    K+V bytes."""
+    import numpy as np
+    import oracle
+    cores = os.cpu_count() or 1
+    threads = min(cores, w.Hq)
+    lengths = w.lengths()
+    t0 = time.perf_counter()
+    done = 0
+    calls = 0
+    while True:
+        b = calls % w.B
+        n = int(lengths[b])
+        if w.paged:
+            kv = [w.logical_kv(b, h) for h in range(w.Hkv)]
+            k = np.stack([x[0] for x in kv])[None]
+            v = np.stack([x[1] for x in kv])[None]
+        else:
+            k, v = w.k[b:b + 1, :, :n], w.v[b:b + 1, :, :n]
+        oracle.decode(w.q[b:b + 1], np.ascontiguousarray(k), np.ascontiguousarray(v), w.scale,
+                      nthreads=threads)
+        done += n * w.Hkv * w.D * 4
+        calls += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(done / dt / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{calls} oracle calls, each one whole sequence of the workload "
+                      f"({w.Hq} query heads over its full history), {dt:.1f} s wall"}
+
+
+def run_fd(args):
+    import torch
+    import split_kv_decode_attn_b200 as fd
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+        barrier = lambda: dist.barrier(device_ids=[local])  # noqa: E731
+    else:
+        barrier = None
+        torch.cuda.set_device(0)
+    device = torch.device("cuda", torch.cuda.current_device())
+    fd.load_library()
+
+    w = make_workload(args.workload, args.L, rank)
+    kvb = w.kv_bytes()
+    copies, l2 = copies_for(torch, (w.k.nbytes + w.v.nbytes), device)
+    call = Call(torch, fd, w, device, args.splits, copies)
+
+    sampler = ClockSampler(device.index)
+    sampler.start()
+    ms = timed(torch, call, args.steps, args.warmup, barrier)
+    clocks = sampler.stop()
+    assert fd.fd_check_device_error() == 0
+
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    per_call_s = ms / 1e3 / args.steps
+    value = world * kvb / per_call_s / 1e9
+    peak, peak_kind = measured_peak()
+    achieved = kvb / per_call_s / 1e9
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "us_per_call": round(per_call_s * 1e6, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+                   "max_len": w.max_len, "block_size": w.block_size, "num_splits": call.S,
+                   "effective_splits": call.s_eff, "kv_bytes_per_call": kvb,
+                   "l2": f"inputs rotate over {copies} cache copies "
+                         f"({copies * (w.k.nbytes + w.v.nbytes) / 1e6:.0f} MB, L2 {l2 / 1e6:.0f} MB)",
+                   "parallelism": f"replicas{world}" if world > 1 else "single"},
+        "roofline": {"bound": "hbm", "kernel": "fd_decode (split + combine)",
+                     "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                     "frac_of_spec_8tbs": round(achieved / SPEC_HBM_GBS, 4),
+                     "traffic": ncu_traffic(w.name)},
+        "gpu_launches": args.steps * call.launches_per_call,
+        "clocks": clocks,
+    }
+
+    if not args.no_e2e:
+        result["e2e"] = e2e(torch, fd, call, w, device, min(args.steps, 30), 3, barrier, world)
+
+    if not args.no_sweep and args.workload == "codellama34b" and rank == 0 and world == 1:
+        result["sweep"] = sweep(torch, fd, device)
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def e2e(torch, fd, call, w, device, steps, warmup, barrier, world):
+    """The same call from pinned host buffers: H2D of q, K, V, fd_decode,
+    D2H of out and lse, all inside the timed region on one stream."""
+    import numpy as np
+    hq = torch.from_numpy(np.ascontiguousarray(w.q).view(np.int16)).view(torch.bfloat16).pin_memory()
+    hk = torch.from_numpy(np.ascontiguousarray(w.k).view(np.int16)).view(torch.bfloat16).pin_memory()
+    hv = torch.from_numpy(np.ascontiguousarray(w.v).view(np.int16)).view(torch.bfloat16).pin_memory()
+    dq, dk, dv = torch.empty_like(hq, device=device), torch.empty_like(hk, device=device), \
+        torch.empty_like(hv, device=device)
+    ho = torch.empty(call.out.shape, dtype=torch.bfloat16).pin_memory()
+    hl = torch.empty(call.lse.shape, dtype=torch.float32).pin_memory()
+
+    def step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        call(dk, dv, dq)
+        ho.copy_(call.out, non_blocking=True)
+        hl.copy_(call.lse, non_blocking=True)
+
+    ms = timed(torch, step, steps, warmup, barrier)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    per = ms / 1e3 / steps
+    h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2
+    d2h = ho.numel() * 2 + hl.numel() * 4
+    return {"value": round(world * w.kv_bytes() / per / 1e9, 2), "unit": "GB/s",
+            "us_per_call": round(per * 1e6, 1), "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+def sweep(torch, fd, device):
+    from split_kv_decode_attn_b200 import workloads as wl
+    peak, _ = measured_peak()
+    rows = []
+    for L in wl.CONFIG2_LENGTHS:
+        w = wl.config(2, L=L)
+        copies, _ = copies_for(torch, w.k.nbytes + w.v.nbytes, device)
+        call = Call(torch, fd, w, device, None, copies)
+        steps = max(200, min(20000, int(0.3e9 / max(w.kv_bytes(), 1) * 100)))
+        ms = timed(torch, call, steps, 50)
+        per = ms / 1e3 / steps
+        gbs = w.kv_bytes() / per / 1e9
+        rows.append({"L": L, "num_splits": call.S, "effective_splits": call.s_eff,
+                     "us_per_call": round(per * 1e6, 3), "GB/s": round(gbs, 1),
+                     "frac_measured": round(gbs / peak, 4), "frac_spec": round(gbs / SPEC_HBM_GBS, 4),
+                     "copies": copies, "steps": steps})
+        del call
+        torch.cuda.empty_cache()
+    return rows
+
+
+# ------------------------------------------------------- reference arm
+
+def run_reference(args):
+    """The fp64 CPU oracle timed as the reference arm: each step is one
+    bounded sample of the workload (all G query heads of one (sequence, KV
+    head) group over a window of the history), sized so the whole run fits
+    in about two minutes.  Rank 0 alone runs it."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    w = make_workload(args.workload, args.L, 0)
+    cores = os.cpu_count() or 1
+    G = w.G
+    groups = [(b, h) for b in range(w.B) for h in range(w.Hkv) if w.lengths()[b] > 0]
+    nsteps = args.steps + args.warmup
+    budget_per_step = 120.0 / max(nsteps, 1)
+
+    def sample(i, n_tok):
+        b, h = groups[i % len(groups)]
+        k, v = w.logical_kv(b, h)
+        n = min(n_tok, len(k))
+        off = (i * 7919) % max(len(k) - n + 1, 1)
+        oracle.attend(w.q[b, h * G:(h + 1) * G], np.ascontiguousarray(k[off:off + n]),
+                      np.ascontiguousarray(v[off:off + n]), w.scale)
+        return n * w.D * 4
+
+    # calibrate the window so that a step takes about the per-step budget
+    n_tok = 1024
+    t0 = time.perf_counter()
+    sample(0, n_tok)
+    dt = max(time.perf_counter() - t0, 1e-6)
+    n_tok = int(max(64, min(int(w.lengths().max()), n_tok * budget_per_step / dt)))
+    for i in range(args.warmup):
+        sample(i, n_tok)
+    t0 = time.perf_counter()
+    nbytes = 0
+    for i in range(args.steps):
+        nbytes += sample(i, n_tok)
+    dt = time.perf_counter() - t0
+    value = nbytes / dt / 1e9
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+                   "max_len": w.max_len},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: the {G} query heads of one (sequence, KV head) "
+                                   f"group over a {n_tok}-token window of its history, one thread"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_fd(args)
+
+
+if __name__ == "__main__":
+    main()
