@@ -156,6 +156,42 @@ FD_API fd_status fd_decode(const fd_problem* p, const void* q, const void* k_cac
                     void* out, float* lse, void* workspace,
                     size_t workspace_bytes, fd_stream_t stream);
 
+/* Largest workspace, in bytes, that fd_decode_static_workspace can use. */
+#define FD_STATIC_WORKSPACE_BYTES (8u << 20)
+
+/* fd_decode for callers that cannot allocate device memory.
+ * The paper has no counterpart to this entry point; it is an addition of this
+ * library. Some callers cannot call cudaMalloc at all. Examples: a plain C
+ * host program that links only this library and has no device allocator of
+ * its own; code inside a framework whose memory pool owns all device memory
+ * and forbids raw allocations; a decode loop that must not call cudaMalloc
+ * mid-step, because it can block on the device and can fail when memory runs
+ * short.
+ * Such callers still pass q, the caches, seqlens, block_table, out and lse,
+ * exactly as for fd_decode. The workspace comes from a file-scope static
+ * __device__ array of FD_STATIC_WORKSPACE_BYTES bytes, which every GPU that
+ * loads this library holds until the process exits. This entry point calls
+ * no cudaMalloc, cudaFree or other allocating routine.
+ *  - Set-up: the first call on a device looks up the array's device address
+ *    with the device current (cudaGetSymbolAddress) and caches it. Make that
+ *    first call before any stream capture on that device.
+ *  - Size limit: when the effective split count needs more than
+ *    FD_STATIC_WORKSPACE_BYTES (see fd_workspace_bytes), the call returns
+ *    FD_ERR_WORKSPACE and launches nothing. Pass a smaller num_splits, or use
+ *    fd_decode with your own workspace.
+ *  - Sharing: every call on a device uses the same array, which keeps the
+ *    last call's contents. Nothing in it has to start at zero, because each
+ *    call writes every partial result before reading it. Calls that overlap
+ *    on the GPU, such as calls on two streams, race on the array and give
+ *    wrong results: serialise them.
+ * Returns the same codes as fd_decode. */
+FD_API fd_status fd_decode_static_workspace(const fd_problem* p, const void* q,
+                                            const void* k_cache, const void* v_cache,
+                                            const int32_t* seqlens,
+                                            const int32_t* block_table, float scale,
+                                            int num_splits, void* out, float* lse,
+                                            fd_stream_t stream);
+
 /* Waits for `stream`, then reads and clears the current device's error word.
  * A kernel sets that word when one of its bounded waits runs out. Returns
  * FD_OK, FD_ERR_DEVICE_TIMEOUT, or FD_ERR_CUDA. */

@@ -28,7 +28,10 @@ FD_ERR_DEVICE_TIMEOUT = -5
 
 # Entry points declared in include/fd.h.
 EXPORTS = ("fd_plan", "fd_plan_sm", "fd_split_chunk", "fd_workspace_bytes", "fd_decode",
-           "fd_check_device_error", "fd_status_string")
+           "fd_decode_static_workspace", "fd_check_device_error", "fd_status_string")
+
+# Mirrors FD_STATIC_WORKSPACE_BYTES in include/fd.h.
+FD_STATIC_WORKSPACE_BYTES = 8 << 20
 
 
 class FdError(RuntimeError):
@@ -67,6 +70,9 @@ def load_library(path: str = LIB_PATH):
         lib.fd_decode.argtypes = [ctypes.POINTER(fd_problem), vp, vp, vp, vp, vp, F, I, vp, vp,
                                   vp, sz, vp]
         lib.fd_decode.restype = I
+        lib.fd_decode_static_workspace.argtypes = [ctypes.POINTER(fd_problem), vp, vp, vp, vp,
+                                                   vp, F, I, vp, vp, vp]
+        lib.fd_decode_static_workspace.restype = I
         lib.fd_check_device_error.argtypes = [vp]
         lib.fd_check_device_error.restype = I
         lib.fd_status_string.argtypes = [I]
@@ -123,6 +129,17 @@ def fd_decode(problem: fd_problem, q, k_cache, v_cache, seqlens, block_table, sc
         ctypes.byref(problem), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens),
         _ptr(block_table), ctypes.c_float(scale), int(num_splits), _ptr(out), _ptr(lse),
         _ptr(workspace), int(workspace_bytes), _stream(stream)))
+
+
+def fd_decode_static_workspace(problem: fd_problem, q, k_cache, v_cache, seqlens, block_table,
+                               scale: float, num_splits: int, out, lse, stream=None) -> int:
+    """Call the C fd_decode_static_workspace: fd_decode for callers that cannot
+    allocate device memory; its scratch is the library's static device array
+    of FD_STATIC_WORKSPACE_BYTES.  Returns the status code."""
+    return int(load_library().fd_decode_static_workspace(
+        ctypes.byref(problem), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens),
+        _ptr(block_table), ctypes.c_float(scale), int(num_splits), _ptr(out), _ptr(lse),
+        _stream(stream)))
 
 
 def fd_check_device_error(stream=None) -> int:

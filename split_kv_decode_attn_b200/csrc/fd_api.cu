@@ -397,6 +397,36 @@ fd_status fd_decode(const fd_problem* p, const void* q, const void* k_cache,
   return FD_OK;
 }
 
+// Scratch of fd_decode_static_workspace: a file-scope device array, so that
+// callers who cannot allocate device memory still get a workspace.
+static __device__ __align__(256) unsigned char g_static_workspace[FD_STATIC_WORKSPACE_BYTES];
+
+fd_status fd_decode_static_workspace(const fd_problem* p, const void* q, const void* k_cache,
+                                     const void* v_cache, const int32_t* seqlens,
+                                     const int32_t* block_table, float scale, int num_splits,
+                                     void* out, float* lse, fd_stream_t stream) {
+  // Host-side checks first: an oversized request launches nothing.
+  if (!p || num_splits < 1 || num_splits > kMaxSplits) return FD_ERR_INVALID_ARGUMENT;
+  const fd_status st = check_shape(p->B, p->Hq, p->Hkv, p->D, p->max_len, p->block_size);
+  if (st != FD_OK) return st;
+  const int n_splits = effective_splits(p->max_len, chunk_for(p->max_len, num_splits));
+  const size_t need = n_splits > 1 ? fd_workspace_bytes(p->B, p->Hq, p->D, n_splits) : 0;
+  if (need > FD_STATIC_WORKSPACE_BYTES) return FD_ERR_WORKSPACE;
+
+  // Set-up, once per device, with that device current: the host-side name of
+  // the array is not a device address; ask the runtime for the real one.
+  static std::atomic<void*> ws_ptr[kMaxDevices];
+  int dev = 0;
+  if (current_device(&dev) != FD_OK) return FD_ERR_CUDA;
+  void* ws = ws_ptr[dev].load();
+  if (!ws) {
+    if (cudaGetSymbolAddress(&ws, g_static_workspace) != cudaSuccess || !ws) return FD_ERR_CUDA;
+    ws_ptr[dev].store(ws);
+  }
+  return fd_decode(p, q, k_cache, v_cache, seqlens, block_table, scale, num_splits, out, lse, ws,
+                   FD_STATIC_WORKSPACE_BYTES, stream);
+}
+
 fd_status fd_check_device_error(fd_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return FD_ERR_CUDA;
