@@ -23,17 +23,23 @@ constexpr int kMaxDevices = 64;
 // ---------------------------------------------------------------- planner
 
 // Cost model of one call, in microseconds, used to pick the split count.
-// Constants are measured on B200 (see the planner notes in the design doc):
-//   kHbmGBs     sustained K/V streaming rate of the whole device
-//   kCtaGBs     streaming rate one CTA reaches on its own (pipeline depth /
-//               memory latency)
-//   kCtaFixedUs per-CTA fixed cost: launch, first-tile latency, epilogue
-//   kCombineUs  second kernel of a split call, before its bytes
+// The constants were fitted to split-count sweeps measured on B200 over the
+// five workload shapes (the planner's pick is the fastest measured split
+// count, or within a few percent of it, on every uniform-length workload):
+//   kHbmGBs      streaming rate of the whole device
+//   kCtaGBs      rate of one CTA alone on an SM (contiguous cache)
+//   kCtaPagedGBs rate of one CTA alone on an SM when pages hold fewer than
+//                64 tokens (one TMA box per page)
+//   kSmPairGBs   rate of an SM running two CTAs, both together
+//   kCtaFixedUs  per-CTA fixed cost (first-tile latency, epilogue)
+//   kCombineUs   the combine kernel of a call with several splits
 struct PlanModel {
   static constexpr double kHbmGBs = 6500.0;
-  static constexpr double kCtaGBs = 45.0;
-  static constexpr double kCtaFixedUs = 1.5;
-  static constexpr double kCombineUs = 2.0;
+  static constexpr double kCtaGBs = 50.0;
+  static constexpr double kCtaPagedGBs = 30.0;
+  static constexpr double kSmPairGBs = 54.0;
+  static constexpr double kCtaFixedUs = 0.5;
+  static constexpr double kCombineUs = 1.0;
 };
 
 int tile_round_up(long long x) {
@@ -51,25 +57,28 @@ int effective_splits(int max_len, int chunk) {
   return static_cast<int>((static_cast<long long>(max_len) + chunk - 1) / chunk);
 }
 
-double model_time_us(int num_sms, int B, int Hq, int Hkv, int D, int max_len, int S) {
+// Time of one wave of k equal CTAs of cta_bytes each.  CTAs are spread over
+// the SMs first one per SM, then two per SM.
+double wave_time_us(double cta_bytes, double k, int num_sms, double solo_gbs) {
+  const double share = PlanModel::kHbmGBs / k;
+  const double limit = k <= num_sms ? solo_gbs : PlanModel::kSmPairGBs / 2.0;
+  return cta_bytes / (std::min(share, limit) * 1e3) + PlanModel::kCtaFixedUs;
+}
+
+double model_time_us(int num_sms, int B, int Hkv, int D, int max_len, int block_size, int S) {
   const int chunk = chunk_for(max_len, S);
   const int s_eff = effective_splits(max_len, chunk);
   const double units = static_cast<double>(B) * Hkv * s_eff;
   const double slots = static_cast<double>(num_sms) * fd::kCtasPerSm;
-  const double chunk_tok = std::min<double>(chunk, max_len);
-  const double cta_bytes = chunk_tok * D * 4.0;
+  const double cta_bytes = std::min<double>(chunk, max_len) * D * 4.0;
+  const double solo = (block_size > 0 && block_size < fd::kTile) ? PlanModel::kCtaPagedGBs
+                                                                 : PlanModel::kCtaGBs;
   const double full_waves = std::floor(units / slots);
   const double rem = units - full_waves * slots;
-  const double hbm = PlanModel::kHbmGBs * 1e3;   // bytes per microsecond
-  const double cta = PlanModel::kCtaGBs * 1e3;
   double t = 0.0;
-  if (full_waves > 0)
-    t += full_waves * (std::max(cta_bytes * slots / hbm, cta_bytes / cta) + PlanModel::kCtaFixedUs);
-  if (rem > 0) t += std::max(cta_bytes * rem / hbm, cta_bytes / cta) + PlanModel::kCtaFixedUs;
-  if (s_eff > 1) {
-    const double ws = static_cast<double>(B) * Hq * s_eff * (D + 1) * 4.0;
-    t += PlanModel::kCombineUs + 2.0 * ws / hbm;
-  }
+  if (full_waves > 0) t += full_waves * wave_time_us(cta_bytes, slots, num_sms, solo);
+  if (rem > 0) t += wave_time_us(cta_bytes, rem, num_sms, solo);
+  if (s_eff > 1) t += PlanModel::kCombineUs;
   return t;
 }
 
@@ -204,19 +213,18 @@ fd_status launch_split(const CUtensorMap& tk, const CUtensorMap& tv, const fd::S
 }
 
 template <int D>
-fd_status launch_combine(const fd::CombineArgs& c, cudaStream_t stream) {
+fd_status launch_combine(const fd::SplitArgs& a, int B, cudaStream_t stream) {
   cudaLaunchConfig_t cfg{};
-  const int rows = c.B * c.Hq;
+  const int rows = B * a.Hq;
   cfg.gridDim = dim3(static_cast<unsigned>((rows + 3) / 4));
   cfg.blockDim = dim3(128);
-  cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, fd::fd_combine_kernel<D>, c) != cudaSuccess) return FD_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, fd::fd_combine_kernel<D>, a, B) != cudaSuccess) return FD_ERR_CUDA;
   return FD_OK;
 }
 
@@ -264,13 +272,13 @@ int fd_plan_sm(int num_sms, int B, int Hq, int Hkv, int D, int max_len, int bloc
   if (static_cast<long long>(B) * Hkv >= static_cast<long long>(num_sms) * fd::kCtasPerSm) return 1;
   const int s_max = static_cast<int>(std::min<long long>(tiles, kMaxSplits));
   int best = 1;
-  double best_t = model_time_us(num_sms, B, Hq, Hkv, D, max_len, 1);
+  double best_t = model_time_us(num_sms, B, Hkv, D, max_len, block_size, 1);
   int last_eff = 1;
   for (int S = 2; S <= s_max; ++S) {
     const int eff = effective_splits(max_len, chunk_for(max_len, S));
     if (eff == last_eff) continue;  // same chunking as a smaller S
     last_eff = eff;
-    const double t = model_time_us(num_sms, B, Hq, Hkv, D, max_len, S);
+    const double t = model_time_us(num_sms, B, Hkv, D, max_len, block_size, S);
     if (t < best_t * 0.98) {  // prefer fewer splits unless clearly faster
       best_t = t;
       best = S;
@@ -324,9 +332,10 @@ fd_status fd_decode(const fd_problem* p, const void* q, const void* k_cache,
   if (n_splits > 1) {
     const size_t need = fd_workspace_bytes(B, Hq, D, n_splits);
     if (!workspace || workspace_bytes < need) return FD_ERR_WORKSPACE;
-    part_o = static_cast<float*>(workspace);
-    part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                        round256(static_cast<size_t>(B) * Hq * n_splits * D * 4));
+    const size_t rows = static_cast<size_t>(B) * Hq * n_splits;
+    char* w = static_cast<char*>(workspace);
+    part_o = reinterpret_cast<float*>(w);
+    part_lse = reinterpret_cast<float*>(w + round256(rows * D * 4));
   }
 
   int dev = 0;
@@ -378,23 +387,8 @@ fd_status fd_decode(const fd_problem* p, const void* q, const void* k_cache,
     r = paged ? dispatch_split<64, true>(G, tk, tv, a, n_splits, Hkv, B, s)
               : dispatch_split<64, false>(G, tk, tv, a, n_splits, Hkv, B, s);
   if (r != FD_OK) return r;
-
-  if (n_splits > 1) {
-    fd::CombineArgs c{};
-    c.part_o = part_o;
-    c.part_lse = part_lse;
-    c.seqlens = seqlens;
-    c.out = static_cast<__nv_bfloat16*>(out);
-    c.lse = lse;
-    c.B = B;
-    c.Hq = Hq;
-    c.max_len = p->max_len;
-    c.chunk = chunk;
-    c.n_splits = n_splits;
-    r = D == 128 ? launch_combine<128>(c, s) : launch_combine<64>(c, s);
-    if (r != FD_OK) return r;
-  }
-  return FD_OK;
+  if (n_splits > 1) r = D == 128 ? launch_combine<128>(a, B, s) : launch_combine<64>(a, B, s);
+  return r;
 }
 
 // Scratch of fd_decode_static_workspace: a file-scope device array, so that

@@ -12,9 +12,12 @@
 // described in the last abstract of scifaro.com's "Related papers:
 // INT-FlashAttention" list.
 //
-// Combine kernel: merges the partials of every (sequence, query head) with
-// the log-sum-exp weights m = max_s lse_s, O = sum_s e^(lse_s - m) O_s /
-// sum_s e^(lse_s - m), lse = m + ln sum_s e^(lse_s - m).
+// Combine kernel: one warp per (sequence, query head) merges that row's
+// partials with the log-sum-exp weights m = max_s lse_s,
+// O = sum_s e^(lse_s - m) O_s / sum_s e^(lse_s - m), lse = m + ln sum_s
+// e^(lse_s - m).  It is chained to the split kernel by programmatic
+// dependent launch.  A sequence whose history fits one split gets its result
+// straight from the split kernel.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -59,15 +62,6 @@ struct SplitArgs {
   float scale_log2;             // scale * log2(e)
 };
 
-struct CombineArgs {
-  const float* part_o;
-  const float* part_lse;
-  const int32_t* seqlens;
-  __nv_bfloat16* out;
-  float* lse;
-  int B, Hq, max_len, chunk, n_splits;
-};
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -86,6 +80,69 @@ __device__ __forceinline__ void raise_device_error(unsigned int code) {
   atomicOr(&g_error_word, code);
 }
 
+// Merge the n_parts partials of one (sequence, query head) row; one warp,
+// lanes cover D.  Partials written by other CTAs are read through L2
+// (ld.global.cg).  Splits are summed in index order, so the result is
+// deterministic.
+template <int D>
+__device__ __forceinline__ void combine_row(const float* po, const float* pl, int n_parts,
+                                            __nv_bfloat16* orow, float* lse_out, int lane) {
+  constexpr int VPL = D / 32;  // 4 or 2 values per lane
+  constexpr float kLog2e = 1.4426950408889634074f;
+  float mx = -INFINITY;
+  for (int s = lane; s < n_parts; s += 32) mx = fmaxf(mx, __ldcg(pl + s));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  float acc[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
+  float W = 0.f;
+  const float* col = po + lane * VPL;
+  int s = 0;
+  for (; s + 8 <= n_parts; s += 8) {
+    float l8[8], o8[8][VPL];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      l8[j] = __ldcg(pl + s + j);
+      if constexpr (VPL == 4) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(col + (s + j) * D));
+        o8[j][0] = v.x; o8[j][1] = v.y; o8[j][2] = v.z; o8[j][3] = v.w;
+      } else {
+        const float2 v = __ldcg(reinterpret_cast<const float2*>(col + (s + j) * D));
+        o8[j][0] = v.x; o8[j][1] = v.y;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float w = ex2((l8[j] - mx) * kLog2e);
+      W += w;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) acc[i] += w * o8[j][i];
+    }
+  }
+  for (; s < n_parts; ++s) {
+    const float w = ex2((__ldcg(pl + s) - mx) * kLog2e);
+    W += w;
+    if constexpr (VPL == 4) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(col + s * D));
+      acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
+    } else {
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(col + s * D));
+      acc[0] += w * v.x; acc[1] += w * v.y;
+    }
+  }
+  const float inv = 1.f / W;
+  if constexpr (VPL == 4) {
+    uint2 pk;
+    pk.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    pk.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<uint2*>(orow + lane * VPL) = pk;
+  } else {
+    *reinterpret_cast<uint32_t*>(orow + lane * VPL) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  }
+  if (lse_out && lane == 0) *lse_out = mx + logf(W);
+}
+
 template <int D, int STAGES>
 struct SplitSmem {
   static constexpr int kHalves = D / 64;               // 128-byte swizzle rows
@@ -93,7 +150,7 @@ struct SplitSmem {
   static constexpr int kTileBytes = kHalves * kHalfBytes;
   static constexpr int kStageBytes = 2 * kTileBytes;   // K tile + V tile
   static constexpr int kBarOffset = STAGES * kStageBytes;
-  static constexpr int kBytes = kBarOffset + 2 * STAGES * 8 + 16;
+  static constexpr int kBytes = kBarOffset + 2 * STAGES * 8 + 16;  // + error flag
   static constexpr int kDynamicBytes = kBytes + 1024;  // room to align to 1 KB
 };
 
@@ -145,9 +202,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   const int h0 = kvh * a.G;
 
   if (start >= end) {
-    // Empty split.  With several splits the combine kernel skips it; with one
-    // split the sequence is empty: out = 0, lse = -inf.
-    if (a.n_splits == 1) {
+    // Empty split.  Split 0 is empty only for an empty sequence, whose
+    // result is out = 0, lse = -inf; other empty splits take no part.
+    if (split == 0) {
       for (int i = threadIdx.x; i < a.G * D; i += kThreads)
         a.out[(static_cast<size_t>(b) * a.Hq + h0) * D + i] = __float2bfloat16_rn(0.f);
       if (a.lse && threadIdx.x < a.G) a.lse[static_cast<size_t>(b) * a.Hq + h0 + threadIdx.x] = -INFINITY;
@@ -446,6 +503,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   }
   named_barrier_sync(1, kConsumerWarps * 32);
 
+  // Splits of this sequence that hold tokens; with one, write the result.
+  const int n_parts = min((n + a.chunk - 1) / a.chunk, a.n_splits);
+  const bool direct = n_parts == 1;
   const int t = threadIdx.x;
   for (int idx = t; idx < a.G * D; idx += kConsumerWarps * 32) {
     const int g = idx / D, d = idx - (idx / D) * D;
@@ -465,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     O = O / Lsum;
     const float lse_val = (M + log2f(Lsum)) * 0.69314718055994530942f;
     const size_t row = static_cast<size_t>(b) * a.Hq + h0 + g;
-    if (a.n_splits == 1) {
+    if (direct) {
       a.out[row * D + d] = __float2bfloat16_rn(O);
       if (d == 0 && a.lse) a.lse[row] = lse_val;
     } else {
@@ -473,64 +533,24 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       if (d == 0) a.part_lse[row * a.n_splits + split] = lse_val;
     }
   }
+  if (direct) return;
+
 }
 
-// One warp per (sequence, query head); lanes cover D with vector loads.
 template <int D>
-__global__ void __launch_bounds__(128) fd_combine_kernel(const CombineArgs a) {
-  constexpr int VPL = D / 32;  // values per lane (4 or 2)
-  grid_dependency_wait();      // partials come from the split kernel
+__global__ void __launch_bounds__(128) fd_combine_kernel(const SplitArgs a, int B) {
+  grid_dependency_wait();     // partials come from the split kernel
+  grid_dependents_launch();   // the next call's split kernel may start its prologue
   const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (row >= a.B * a.Hq) return;
+  if (row >= B * a.Hq) return;
   const int b = row / a.Hq;
   const int n = seq_length(a.seqlens, b, a.max_len);
-  int ns = (n + a.chunk - 1) / a.chunk;
-  ns = ns < a.n_splits ? ns : a.n_splits;
-  __nv_bfloat16* orow = a.out + static_cast<size_t>(row) * D + lane * VPL;
-  if (ns == 0) {
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) orow[i] = __float2bfloat16_rn(0.f);
-    if (a.lse && lane == 0) a.lse[row] = -INFINITY;
-    return;
-  }
-  const float* pl = a.part_lse + static_cast<size_t>(row) * a.n_splits;
-  const float* po = a.part_o + static_cast<size_t>(row) * a.n_splits * D + lane * VPL;
-  float mx = -INFINITY;
-  for (int s = lane; s < ns; s += 32) mx = fmaxf(mx, pl[s]);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  constexpr float kLog2e = 1.4426950408889634074f;
-  float accv[VPL];
-#pragma unroll
-  for (int i = 0; i < VPL; ++i) accv[i] = 0.f;
-  float W = 0.f;
-#pragma unroll 4
-  for (int s = 0; s < ns; ++s) {
-    const float w = ex2((pl[s] - mx) * kLog2e);
-    W += w;
-    if constexpr (VPL == 4) {
-      const float4 o = *reinterpret_cast<const float4*>(po + static_cast<size_t>(s) * D);
-      accv[0] += w * o.x;
-      accv[1] += w * o.y;
-      accv[2] += w * o.z;
-      accv[3] += w * o.w;
-    } else {
-      const float2 o = *reinterpret_cast<const float2*>(po + static_cast<size_t>(s) * D);
-      accv[0] += w * o.x;
-      accv[1] += w * o.y;
-    }
-  }
-  const float inv = 1.f / W;
-  if constexpr (VPL == 4) {
-    uint2 pk;
-    pk.x = pack_bf16x2(accv[0] * inv, accv[1] * inv);
-    pk.y = pack_bf16x2(accv[2] * inv, accv[3] * inv);
-    *reinterpret_cast<uint2*>(orow) = pk;
-  } else {
-    *reinterpret_cast<uint32_t*>(orow) = pack_bf16x2(accv[0] * inv, accv[1] * inv);
-  }
-  if (a.lse && lane == 0) a.lse[row] = mx + logf(W);
+  const int n_parts = min((n + a.chunk - 1) / a.chunk, a.n_splits);
+  if (n_parts <= 1) return;
+  combine_row<D>(a.part_o + static_cast<size_t>(row) * a.n_splits * D,
+                 a.part_lse + static_cast<size_t>(row) * a.n_splits, n_parts,
+                 a.out + static_cast<size_t>(row) * D, a.lse ? a.lse + row : nullptr, lane);
 }
 
 }  // namespace fd

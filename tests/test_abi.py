@@ -57,7 +57,8 @@ def test_workspace_bytes():
     assert fd.fd_workspace_bytes(1, 64, 128, 1) == 0
     B, Hq, D, S = 1, 64, 128, 37
     rows = B * Hq * S
-    expect = (rows * D * 4 + 255) // 256 * 256 + (rows * 4 + 255) // 256 * 256
+    r256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    expect = r256(rows * D * 4) + r256(rows * 4)
     assert fd.fd_workspace_bytes(B, Hq, D, S) == expect
     assert fd.fd_workspace_bytes(0, 64, 128, 2) == 0
     assert fd.fd_workspace_bytes(1, 64, 128, 0) == 0
@@ -83,8 +84,22 @@ def test_plan_long_history_fills_the_device():
         chunk = fd.fd_split_chunk(L, S)
         s_eff = -(-L // chunk)
         ctas = 8 * s_eff
-        assert ctas >= 0.9 * B200_SMS, (L, S, ctas)
+        assert ctas >= 0.75 * B200_SMS, (L, S, ctas)
         assert ctas <= 4 * 2 * B200_SMS, (L, S, ctas)
+
+
+# Split counts that were fastest, or within 4 %, in sweeps measured on B200
+# (the planner's constants were fitted to those sweeps).
+@pytest.mark.parametrize("shape,good", [
+    ((1, 64, 8, 128, 8192, 0), {12, 16, 18}),
+    ((1, 64, 8, 128, 16384, 0), {16, 18, 20}),
+    ((1, 64, 8, 128, 32768, 0), {16, 18, 24}),
+    ((1, 64, 8, 128, 65536, 0), {16, 18, 24}),
+    ((8, 32, 8, 128, 131072, 16), {4, 18}),
+    ((1, 32, 8, 128, 262144, 0), {16, 18, 24, 32}),
+])
+def test_plan_matches_measured_sweeps(shape, good):
+    assert fd.fd_plan_sm(B200_SMS, *shape) in good
 
 
 def test_plan_splits_grow_with_length_and_are_deterministic():
