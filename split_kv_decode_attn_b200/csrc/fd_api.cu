@@ -184,7 +184,7 @@ template <int D, int NB, int MODE, bool PAGED>
 fd_status launch_split(const CUtensorMap& tk, const CUtensorMap& tv, const fd::SplitArgs& a,
                        int n_splits, int Hkv, int B, cudaStream_t stream) {
   constexpr int STAGES = D == 128 ? 3 : 6;
-  using L = fd::SplitSmem<D, STAGES>;
+  using L = fd::SplitSmem<D, NB, STAGES>;
   auto kern = fd::fd_split_kernel<D, NB, MODE, PAGED, STAGES>;
   // The shared-memory opt-in is per device; remember which devices have it.
   static std::atomic<unsigned long long> attr_done{0};
@@ -228,13 +228,22 @@ fd_status launch_combine(const fd::SplitArgs& a, int B, cudaStream_t stream) {
   return FD_OK;
 }
 
+// Launches the split kernel and, with several splits, the combine kernel.
+template <int D, int NB, int MODE, bool PAGED>
+fd_status launch_call(const CUtensorMap& tk, const CUtensorMap& tv, const fd::SplitArgs& a,
+                      int n_splits, int Hkv, int B, cudaStream_t s) {
+  fd_status r = launch_split<D, NB, MODE, PAGED>(tk, tv, a, n_splits, Hkv, B, s);
+  if (r == FD_OK && n_splits > 1) r = launch_combine<D>(a, B, s);
+  return r;
+}
+
 template <int D, bool PAGED>
 fd_status dispatch_split(int G, const CUtensorMap& tk, const CUtensorMap& tv,
                          const fd::SplitArgs& a, int n_splits, int Hkv, int B,
                          cudaStream_t s) {
-  if (G <= 4) return launch_split<D, 1, fd::kDup, PAGED>(tk, tv, a, n_splits, Hkv, B, s);
-  if (G == 8) return launch_split<D, 1, fd::kHiLo, PAGED>(tk, tv, a, n_splits, Hkv, B, s);
-  return launch_split<D, 2, fd::kHiLo, PAGED>(tk, tv, a, n_splits, Hkv, B, s);
+  if (G <= 4) return launch_call<D, 1, fd::kDup, PAGED>(tk, tv, a, n_splits, Hkv, B, s);
+  if (G == 8) return launch_call<D, 1, fd::kHiLo, PAGED>(tk, tv, a, n_splits, Hkv, B, s);
+  return launch_call<D, 2, fd::kHiLo, PAGED>(tk, tv, a, n_splits, Hkv, B, s);
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -386,8 +395,6 @@ fd_status fd_decode(const fd_problem* p, const void* q, const void* k_cache,
   else
     r = paged ? dispatch_split<64, true>(G, tk, tv, a, n_splits, Hkv, B, s)
               : dispatch_split<64, false>(G, tk, tv, a, n_splits, Hkv, B, s);
-  if (r != FD_OK) return r;
-  if (n_splits > 1) r = D == 128 ? launch_combine<128>(a, B, s) : launch_combine<64>(a, B, s);
   return r;
 }
 

@@ -82,13 +82,33 @@ __device__ __forceinline__ void raise_device_error(unsigned int code) {
 
 // Merge the n_parts partials of one (sequence, query head) row; one warp,
 // lanes cover D.  Partials written by other CTAs are read through L2
-// (ld.global.cg).  Splits are summed in index order, so the result is
-// deterministic.
+// (ld.global.cg).  The first 16 split rows are requested together with the
+// lse values, so a row with up to 16 splits costs one round trip.  Splits
+// are summed in index order, so the result is deterministic.
 template <int D>
 __device__ __forceinline__ void combine_row(const float* po, const float* pl, int n_parts,
                                             __nv_bfloat16* orow, float* lse_out, int lane) {
   constexpr int VPL = D / 32;  // 4 or 2 values per lane
+  constexpr int BATCH = 16;
   constexpr float kLog2e = 1.4426950408889634074f;
+  const float* col = po + lane * VPL;
+  float lb[BATCH], ob[BATCH][VPL];
+  auto load_batch = [&](int s0) {
+#pragma unroll
+    for (int j = 0; j < BATCH; ++j) {
+      if (s0 + j < n_parts) {
+        lb[j] = __ldcg(pl + s0 + j);
+        if constexpr (VPL == 4) {
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(col + (s0 + j) * D));
+          ob[j][0] = v.x; ob[j][1] = v.y; ob[j][2] = v.z; ob[j][3] = v.w;
+        } else {
+          const float2 v = __ldcg(reinterpret_cast<const float2*>(col + (s0 + j) * D));
+          ob[j][0] = v.x; ob[j][1] = v.y;
+        }
+      }
+    }
+  };
+  load_batch(0);
   float mx = -INFINITY;
   for (int s = lane; s < n_parts; s += 32) mx = fmaxf(mx, __ldcg(pl + s));
 #pragma unroll
@@ -97,38 +117,16 @@ __device__ __forceinline__ void combine_row(const float* po, const float* pl, in
 #pragma unroll
   for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
   float W = 0.f;
-  const float* col = po + lane * VPL;
-  int s = 0;
-  for (; s + 8 <= n_parts; s += 8) {
-    float l8[8], o8[8][VPL];
+  for (int s0 = 0; s0 < n_parts; s0 += BATCH) {
+    if (s0 > 0) load_batch(s0);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      l8[j] = __ldcg(pl + s + j);
-      if constexpr (VPL == 4) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(col + (s + j) * D));
-        o8[j][0] = v.x; o8[j][1] = v.y; o8[j][2] = v.z; o8[j][3] = v.w;
-      } else {
-        const float2 v = __ldcg(reinterpret_cast<const float2*>(col + (s + j) * D));
-        o8[j][0] = v.x; o8[j][1] = v.y;
+    for (int j = 0; j < BATCH; ++j) {
+      if (s0 + j < n_parts) {
+        const float w = ex2((lb[j] - mx) * kLog2e);
+        W += w;
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) acc[i] += w * ob[j][i];
       }
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float w = ex2((l8[j] - mx) * kLog2e);
-      W += w;
-#pragma unroll
-      for (int i = 0; i < VPL; ++i) acc[i] += w * o8[j][i];
-    }
-  }
-  for (; s < n_parts; ++s) {
-    const float w = ex2((__ldcg(pl + s) - mx) * kLog2e);
-    W += w;
-    if constexpr (VPL == 4) {
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(col + s * D));
-      acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
-    } else {
-      const float2 v = __ldcg(reinterpret_cast<const float2*>(col + s * D));
-      acc[0] += w * v.x; acc[1] += w * v.y;
     }
   }
   const float inv = 1.f / W;
@@ -143,7 +141,7 @@ __device__ __forceinline__ void combine_row(const float* po, const float* pl, in
   if (lse_out && lane == 0) *lse_out = mx + logf(W);
 }
 
-template <int D, int STAGES>
+template <int D, int NB, int STAGES>
 struct SplitSmem {
   static constexpr int kHalves = D / 64;               // 128-byte swizzle rows
   static constexpr int kHalfBytes = kTile * 128;       // one 64-column half tile
@@ -152,152 +150,32 @@ struct SplitSmem {
   static constexpr int kBarOffset = STAGES * kStageBytes;
   static constexpr int kBytes = kBarOffset + 2 * STAGES * 8 + 16;  // + error flag
   static constexpr int kDynamicBytes = kBytes + 1024;  // room to align to 1 KB
+  // Epilogue scratch, laid over the drained pipeline buffers (floats):
+  static constexpr int kNcol = NB * 8;
+  static constexpr int kRedAcc = 0;                                   // [warp][col][D]
+  static constexpr int kRedM = kRedAcc + kConsumerWarps * kNcol * D;  // [warp][col]
+  static constexpr int kRedL = kRedM + kConsumerWarps * kNcol;        // [warp][col]
+  static constexpr int kRedW = kRedL + kConsumerWarps * kNcol;        // [warp][col]
+  static constexpr int kSplitLse = kRedW + kConsumerWarps * kNcol;    // [col]: this split's lse
+  static constexpr int kScratchFloats = kSplitLse + kNcol;
+  static_assert(kScratchFloats * 4 <= kBarOffset, "epilogue scratch must fit the pipeline buffers");
 };
 
-template <int D, int NB, int MODE, bool PAGED, int STAGES>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
-    fd_split_kernel(const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const SplitArgs a) {
-  using L = SplitSmem<D, STAGES>;
+// Consumer warps of the split kernel: scores, online softmax and P.V over the
+// split's tiles, then the merge of the four warps' softmax states into this
+// split's result, which goes to `out` (the sequence has one split) or to the
+// global partials (several splits).
+template <int D, int NB, int MODE, int STAGES>
+__device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* smem,
+                                                uint32_t smem_base, uint32_t bar_full,
+                                                uint32_t bar_empty, volatile int* cta_error,
+                                                int warp, int lane, int b, int h0, int split,
+                                                int start, int end, int n_tiles, int n_parts) {
+  using L = SplitSmem<D, NB, STAGES>;
   constexpr int KSTEPS = D / 16;   // k-steps of the score MMA (over D)
   constexpr int DBLK = D / 16;     // m-blocks of the P.V MMA (over D)
   constexpr int NCOL = NB * 8;     // MMA columns (query heads, maybe doubled)
-  static_assert(MODE != kDup || NB == 1, "duplicated columns need one column block");
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const uint32_t smem_base = smem_u32(smem);
-  const uint32_t bar_full = smem_base + L::kBarOffset;
-  const uint32_t bar_empty = bar_full + STAGES * 8;
-  volatile int* cta_error = reinterpret_cast<volatile int*>(smem + L::kBarOffset + 2 * STAGES * 8);
-
-  const int split = blockIdx.x;
-  const int kvh = blockIdx.y;
-  const int b = blockIdx.z;
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_empty + 8 * s, kConsumerWarps);
-    }
-    *cta_error = 0;
-    fence_mbar_init();
-  }
-  if (warp == kConsumerWarps && lane == 0) {
-    prefetch_tensormap(&tmK);
-    prefetch_tensormap(&tmV);
-  }
-  __syncthreads();
-
-  // Inputs may be produced by the previous kernel on the stream.
-  grid_dependency_wait();
-  grid_dependents_launch();
-
-  const int n = seq_length(a.seqlens, b, a.max_len);
-  const int start = split * a.chunk;
-  const int end = min(start + a.chunk, n);
-  const int h0 = kvh * a.G;
-
-  if (start >= end) {
-    // Empty split.  Split 0 is empty only for an empty sequence, whose
-    // result is out = 0, lse = -inf; other empty splits take no part.
-    if (split == 0) {
-      for (int i = threadIdx.x; i < a.G * D; i += kThreads)
-        a.out[(static_cast<size_t>(b) * a.Hq + h0) * D + i] = __float2bfloat16_rn(0.f);
-      if (a.lse && threadIdx.x < a.G) a.lse[static_cast<size_t>(b) * a.Hq + h0 + threadIdx.x] = -INFINITY;
-    }
-    return;
-  }
-  const int n_tiles = (end - start + kTile - 1) / kTile;
-
-  if (warp == kConsumerWarps) {
-    // ------------------------------------------------------------- producer
-    const uint64_t policy = policy_evict_first();
-    int issued = 0;
-    bool ok = true;
-    if constexpr (!PAGED) {
-      const int plane = b * a.Hkv + kvh;
-      for (int it = 0; it < n_tiles; ++it) {
-        const int s = it % STAGES, k = it / STAGES;
-        if (k > 0 && !mbar_wait(bar_empty + 8 * s, (k - 1) & 1, kWaitLimitNs)) { ok = false; break; }
-        if (lane == 0) {
-          const int t0 = start + it * kTile;
-          const uint32_t dk = smem_base + s * L::kStageBytes;
-          const uint32_t dv = dk + L::kTileBytes;
-          mbar_arrive_expect_tx(bar_full + 8 * s, L::kStageBytes);
-#pragma unroll
-          for (int hf = 0; hf < L::kHalves; ++hf) {
-            tma_load_3d(dk + hf * L::kHalfBytes, &tmK, bar_full + 8 * s, hf * 64, t0, plane, policy);
-            tma_load_3d(dv + hf * L::kHalfBytes, &tmV, bar_full + 8 * s, hf * 64, t0, plane, policy);
-          }
-        }
-        ++issued;
-        __syncwarp();
-      }
-    } else {
-      const int bs = a.block_size, lbs = a.log2_block_size;
-      const int rows = bs < kTile ? bs : kTile;            // rows per TMA box
-      const int pages_per_tile = bs < kTile ? kTile / bs : 1;
-      const int n_pages = (n + bs - 1) >> lbs;
-      const int32_t* bt = a.block_table + static_cast<size_t>(b) * a.max_blocks_per_seq;
-      // A window of 32 page ids, one per lane, plus the next window in flight.
-      int win = start >> lbs;
-      int cur = (win + lane < n_pages) ? __ldg(bt + win + lane) : 0;
-      int nxt = (win + 32 + lane < n_pages) ? __ldg(bt + win + 32 + lane) : 0;
-      for (int it = 0; it < n_tiles; ++it) {
-        const int s = it % STAGES, k = it / STAGES;
-        if (k > 0 && !mbar_wait(bar_empty + 8 * s, (k - 1) & 1, kWaitLimitNs)) { ok = false; break; }
-        const int t0 = start + it * kTile;
-        const int pg = t0 >> lbs;
-        if (pg >= win + 32) {
-          win += 32;
-          cur = nxt;
-          nxt = (win + 32 + lane < n_pages) ? __ldg(bt + win + 32 + lane) : 0;
-        }
-        const int row0 = bs > kTile ? (t0 & (bs - 1)) : 0;
-        const int valid_pages = min(pages_per_tile, n_pages - pg);
-        const uint32_t dk = smem_base + s * L::kStageBytes;
-        const uint32_t dv = dk + L::kTileBytes;
-        int pid[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) pid[j] = __shfl_sync(0xffffffffu, cur, (pg - win + j) & 31);
-        if (lane == 0) {
-          mbar_arrive_expect_tx(bar_full + 8 * s,
-                                valid_pages * rows * 128 * L::kHalves * 2);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (j < valid_pages) {
-              const int plane = pid[j] * a.Hkv + kvh;
-#pragma unroll
-              for (int hf = 0; hf < L::kHalves; ++hf) {
-                const uint32_t off = hf * L::kHalfBytes + j * rows * 128;
-                tma_load_3d(dk + off, &tmK, bar_full + 8 * s, hf * 64, row0, plane, policy);
-                tma_load_3d(dv + off, &tmV, bar_full + 8 * s, hf * 64, row0, plane, policy);
-              }
-            }
-          }
-        }
-        ++issued;
-        __syncwarp();
-      }
-    }
-    if (!ok && lane == 0) {
-      raise_device_error(1u);
-      *cta_error = 1;
-    }
-    // No copy may still be landing in shared memory when the CTA retires.
-    if (lane == 0) {
-      for (int it = issued > STAGES ? issued - STAGES : 0; it < issued; ++it)
-        if (!mbar_wait(bar_full + 8 * (it % STAGES), (it / STAGES) & 1, kWaitLimitNs))
-          raise_device_error(2u);
-    }
-    return;
-  }
-
-  // --------------------------------------------------------------- consumers
   // B fragments of Q^T (k = head dim, n = query head), loaded once.
   uint32_t qf[NB][KSTEPS][2];
   {
@@ -340,7 +218,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
   for (int it = 0; it < n_tiles; ++it) {
     const int s = it % STAGES, k = it / STAGES;
-    if (!mbar_wait(bar_full + 8 * s, k & 1, kWaitLimitNs)) {
+    const bool ok = mbar_wait(bar_full + 8 * s, k & 1, kWaitLimitNs);
+    if (!__all_sync(0xffffffffu, ok)) {
       failed = true;
       break;
     }
@@ -472,19 +351,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         l_run[nb][j] += __shfl_xor_sync(0xffffffffu, l_run[nb][j], off);
 
   // Every consumer warp is past its last shared-memory read of the pipeline.
-  named_barrier_sync(1, kConsumerWarps * 32);
-  if (*cta_error) return;
 
-  // Merge the four warps' partial softmax states through shared memory
-  // (the pipeline buffers are free: every issued tile has landed and been read).
-  float* red_acc = reinterpret_cast<float*>(smem);                 // [warp][NCOL][D]
-  float* red_m = red_acc + kConsumerWarps * NCOL * D;               // [warp][NCOL]
-  float* red_l = red_m + kConsumerWarps * NCOL;                     // [warp][NCOL]
-  {
+  // Every consumer warp is past its last shared-memory read of the pipeline,
+  // so the drained buffers hold the epilogue scratch.
+  named_barrier_sync(1, kConsumerWarps * 32);
+  const int t = threadIdx.x;
+  float* f = reinterpret_cast<float*>(smem);
+  const bool live = !*cta_error;
+  if (live) {
     const int j0 = 2 * (lane & 3);
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
-      float* base = red_acc + (warp * NCOL + nb * 8 + j0) * D;
+      float* base = f + L::kRedAcc + (warp * NCOL + nb * 8 + j0) * D;
 #pragma unroll
       for (int db = 0; db < DBLK; ++db) {
         const int d = db * 16 + (lane >> 2);
@@ -494,47 +372,214 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         base[D + d + 8] = acc[nb][db][3];
       }
       if (lane < 4) {
-        red_m[warp * NCOL + nb * 8 + j0] = m_run[nb][0];
-        red_m[warp * NCOL + nb * 8 + j0 + 1] = m_run[nb][1];
-        red_l[warp * NCOL + nb * 8 + j0] = l_run[nb][0];
-        red_l[warp * NCOL + nb * 8 + j0 + 1] = l_run[nb][1];
+        f[L::kRedM + warp * NCOL + nb * 8 + j0] = m_run[nb][0];
+        f[L::kRedM + warp * NCOL + nb * 8 + j0 + 1] = m_run[nb][1];
+        f[L::kRedL + warp * NCOL + nb * 8 + j0] = l_run[nb][0];
+        f[L::kRedL + warp * NCOL + nb * 8 + j0 + 1] = l_run[nb][1];
       }
     }
   }
   named_barrier_sync(1, kConsumerWarps * 32);
-
-  // Splits of this sequence that hold tokens; with one, write the result.
-  const int n_parts = min((n + a.chunk - 1) / a.chunk, a.n_splits);
-  const bool direct = n_parts == 1;
-  const int t = threadIdx.x;
-  for (int idx = t; idx < a.G * D; idx += kConsumerWarps * 32) {
-    const int g = idx / D, d = idx - (idx / D) * D;
-    const int col = g;  // head g lives in column g (kDup adds column g + 4)
+  // Per head: the weight of each warp's state and this split's lse.
+  if (live && t < a.G) {
+    float mw[kConsumerWarps];
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red_m[w * NCOL + col]);
-    float Lsum = 0.f, O = 0.f;
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      mw[w] = f[L::kRedM + w * NCOL + t];
+      M = fmaxf(M, mw[w]);
+    }
+    if (M == -INFINITY) {  // no token in this split
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) f[L::kRedW + w * NCOL + t] = 0.f;
+      f[L::kSplitLse + t] = -INFINITY;
+    } else {
+      float e[kConsumerWarps];
+      float Ls = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        e[w] = ex2(mw[w] - M);
+        Ls += e[w] * f[L::kRedL + w * NCOL + t];
+      }
+      const float inv = 1.f / Ls;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) f[L::kRedW + w * NCOL + t] = e[w] * inv;
+      f[L::kSplitLse + t] = (M + log2f(Ls)) * 0.69314718055994530942f;
+    }
+  }
+  named_barrier_sync(1, kConsumerWarps * 32);
+  if (!live) return;
+
+  const bool direct = n_parts == 1;
+  for (int idx = t; idx < a.G * D; idx += kConsumerWarps * 32) {
+    const int g = idx / D, d = idx - (idx / D) * D;
+    float O = 0.f;
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) {
-      const float wt = ex2(red_m[w * NCOL + col] - M);
-      Lsum += wt * red_l[w * NCOL + col];
-      float v = red_acc[(w * NCOL + col) * D + d];
-      if constexpr (MODE == kDup) v += red_acc[(w * NCOL + col + 4) * D + d];
-      O += wt * v;
+      float v = f[L::kRedAcc + (w * NCOL + g) * D + d];
+      if constexpr (MODE == kDup) v += f[L::kRedAcc + (w * NCOL + g + 4) * D + d];
+      O += f[L::kRedW + w * NCOL + g] * v;
     }
-    O = O / Lsum;
-    const float lse_val = (M + log2f(Lsum)) * 0.69314718055994530942f;
     const size_t row = static_cast<size_t>(b) * a.Hq + h0 + g;
     if (direct) {
       a.out[row * D + d] = __float2bfloat16_rn(O);
-      if (d == 0 && a.lse) a.lse[row] = lse_val;
+      if (d == 0 && a.lse) a.lse[row] = f[L::kSplitLse + g];
     } else {
       a.part_o[(row * a.n_splits + split) * D + d] = O;
-      if (d == 0) a.part_lse[row * a.n_splits + split] = lse_val;
+      if (d == 0) a.part_lse[row * a.n_splits + split] = f[L::kSplitLse + g];
     }
   }
-  if (direct) return;
+}
 
+// Split kernel: one CTA per (split, KV head, sequence).
+template <int D, int NB, int MODE, bool PAGED, int STAGES>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    fd_split_kernel(const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const SplitArgs a) {
+  using L = SplitSmem<D, NB, STAGES>;
+  static_assert(MODE != kDup || NB == 1, "duplicated columns need one column block");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t smem_base = smem_u32(smem);
+  const uint32_t bar_full = smem_base + L::kBarOffset;
+  const uint32_t bar_empty = bar_full + STAGES * 8;
+  volatile int* cta_error = reinterpret_cast<volatile int*>(smem + L::kBarOffset + 2 * STAGES * 8);
+
+  const int split = blockIdx.x;
+  const int kvh = blockIdx.y;
+  const int b = blockIdx.z;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, kConsumerWarps);
+    }
+    *cta_error = 0;
+    fence_mbar_init();
+  }
+  if (warp == kConsumerWarps && lane == 0) {
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmV);
+  }
+  __syncthreads();
+
+  // Inputs may be produced by the previous kernel on the stream.
+  grid_dependency_wait();
+  grid_dependents_launch();
+
+  const int n = seq_length(a.seqlens, b, a.max_len);
+  const int start = split * a.chunk;
+  const int end = min(start + a.chunk, n);
+  const int h0 = kvh * a.G;
+  const int n_tiles = start < end ? (end - start + kTile - 1) / kTile : 0;
+  // Splits of this sequence that hold tokens.
+  const int n_parts = min((n + a.chunk - 1) / a.chunk, a.n_splits);
+
+  if (n_tiles == 0) {
+    // Empty split.  Split 0 is empty only for an empty sequence, whose
+    // result is out = 0, lse = -inf; other empty splits take no part.
+    if (split == 0) {
+      for (int i = threadIdx.x; i < a.G * D; i += kThreads)
+        a.out[(static_cast<size_t>(b) * a.Hq + h0) * D + i] = __float2bfloat16_rn(0.f);
+      if (a.lse && threadIdx.x < a.G) a.lse[static_cast<size_t>(b) * a.Hq + h0 + threadIdx.x] = -INFINITY;
+    }
+    return;
+  }
+
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------- producer
+    // Every lane waits (the decision is made warp-uniform); lane 0 issues.
+    const uint64_t policy = policy_evict_first();
+    int issued = 0;
+    bool ok = true;
+    if constexpr (!PAGED) {
+      const int plane = b * a.Hkv + kvh;
+      for (int it = 0; it < n_tiles; ++it) {
+        const int s = it % STAGES, k = it / STAGES;
+        if (k > 0) ok = mbar_wait(bar_empty + 8 * s, (k - 1) & 1, kWaitLimitNs);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        if (lane == 0) {
+          const int t0 = start + it * kTile;
+          const uint32_t dk = smem_base + s * L::kStageBytes;
+          const uint32_t dv = dk + L::kTileBytes;
+          mbar_arrive_expect_tx(bar_full + 8 * s, L::kStageBytes);
+#pragma unroll
+          for (int hf = 0; hf < L::kHalves; ++hf) {
+            tma_load_3d(dk + hf * L::kHalfBytes, &tmK, bar_full + 8 * s, hf * 64, t0, plane, policy);
+            tma_load_3d(dv + hf * L::kHalfBytes, &tmV, bar_full + 8 * s, hf * 64, t0, plane, policy);
+          }
+        }
+        ++issued;
+        __syncwarp();
+      }
+    } else {
+      const int bs = a.block_size, lbs = a.log2_block_size;
+      const int rows = bs < kTile ? bs : kTile;            // rows per TMA box
+      const int pages_per_tile = bs < kTile ? kTile / bs : 1;
+      const int n_pages = (n + bs - 1) >> lbs;
+      const int32_t* bt = a.block_table + static_cast<size_t>(b) * a.max_blocks_per_seq;
+      // A window of 32 page ids, one per lane, plus the next window in flight.
+      int win = start >> lbs;
+      int cur = (win + lane < n_pages) ? __ldg(bt + win + lane) : 0;
+      int nxt = (win + 32 + lane < n_pages) ? __ldg(bt + win + 32 + lane) : 0;
+      for (int it = 0; it < n_tiles; ++it) {
+        const int s = it % STAGES, k = it / STAGES;
+        if (k > 0) ok = mbar_wait(bar_empty + 8 * s, (k - 1) & 1, kWaitLimitNs);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        const int t0 = start + it * kTile;
+        const int pg = t0 >> lbs;
+        if (pg >= win + 32) {
+          win += 32;
+          cur = nxt;
+          nxt = (win + 32 + lane < n_pages) ? __ldg(bt + win + 32 + lane) : 0;
+        }
+        const int row0 = bs > kTile ? (t0 & (bs - 1)) : 0;
+        const int valid_pages = min(pages_per_tile, n_pages - pg);
+        const uint32_t dk = smem_base + s * L::kStageBytes;
+        const uint32_t dv = dk + L::kTileBytes;
+        int pid[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) pid[j] = __shfl_sync(0xffffffffu, cur, (pg - win + j) & 31);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar_full + 8 * s,
+                                valid_pages * rows * 128 * L::kHalves * 2);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (j < valid_pages) {
+              const int plane = pid[j] * a.Hkv + kvh;
+#pragma unroll
+              for (int hf = 0; hf < L::kHalves; ++hf) {
+                const uint32_t off = hf * L::kHalfBytes + j * rows * 128;
+                tma_load_3d(dk + off, &tmK, bar_full + 8 * s, hf * 64, row0, plane, policy);
+                tma_load_3d(dv + off, &tmV, bar_full + 8 * s, hf * 64, row0, plane, policy);
+              }
+            }
+          }
+        }
+        ++issued;
+        __syncwarp();
+      }
+    }
+    if (!ok && lane == 0) {
+      raise_device_error(1u);
+      *cta_error = 1;
+    }
+    // No copy may still be landing in shared memory when the CTA retires.
+    if (lane == 0) {
+      for (int it = issued > STAGES ? issued - STAGES : 0; it < issued; ++it)
+        if (!mbar_wait(bar_full + 8 * (it % STAGES), (it / STAGES) & 1, kWaitLimitNs))
+          raise_device_error(2u);
+    }
+  } else {
+    // ------------------------------------------------------------- consumers
+    split_consumers<D, NB, MODE, STAGES>(a, smem, smem_base, bar_full, bar_empty, cta_error,
+                                         warp, lane, b, h0, split, start, end, n_tiles,
+                                         n_parts);
+  }
 }
 
 template <int D>
