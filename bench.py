@@ -425,10 +425,11 @@ def sweep(torch, fd, device):
 # ------------------------------------------------------- reference arm
 
 def run_reference(args):
-    """The fp64 CPU oracle timed as the reference arm: each step is one
-    bounded sample of the workload (all G query heads of one (sequence, KV
-    head) group over a window of the history), sized so the whole run fits
-    in about two minutes.  Rank 0 alone runs it."""
+    """The fp64 CPU oracle timed as the reference arm, on this host's cores.
+    Each step is one bounded sample of the workload: every query head of one
+    sequence (threads over heads) over a window of its history.  The window
+    is calibrated so that the whole --steps/--warmup run takes about two
+    minutes.  Rank 0 alone runs it."""
     rank, world, _ = dist_env()
     if rank != 0:
         return
@@ -436,26 +437,30 @@ def run_reference(args):
     import oracle
     w = make_workload(args.workload, args.L, 0)
     cores = os.cpu_count() or 1
-    G = w.G
-    groups = [(b, h) for b in range(w.B) for h in range(w.Hkv) if w.lengths()[b] > 0]
-    nsteps = args.steps + args.warmup
-    budget_per_step = 120.0 / max(nsteps, 1)
+    threads = min(cores, w.Hq)
+    lengths = w.lengths()
+    seqs = [b for b in range(w.B) if lengths[b] > 0]
+    budget_per_step = 120.0 / max(args.steps + args.warmup, 1)
 
     def sample(i, n_tok):
-        b, h = groups[i % len(groups)]
-        k, v = w.logical_kv(b, h)
-        n = min(n_tok, len(k))
-        off = (i * 7919) % max(len(k) - n + 1, 1)
-        oracle.attend(w.q[b, h * G:(h + 1) * G], np.ascontiguousarray(k[off:off + n]),
-                      np.ascontiguousarray(v[off:off + n]), w.scale)
-        return n * w.D * 4
+        b = seqs[i % len(seqs)]
+        n = min(n_tok, int(lengths[b]))
+        off = (i * 7919) % max(int(lengths[b]) - n + 1, 1)
+        if w.paged:
+            kv = [w.logical_kv(b, h) for h in range(w.Hkv)]
+            k = np.stack([x[0][off:off + n] for x in kv])[None]
+            v = np.stack([x[1][off:off + n] for x in kv])[None]
+        else:
+            k, v = w.k[b:b + 1, :, off:off + n], w.v[b:b + 1, :, off:off + n]
+        oracle.decode(w.q[b:b + 1], np.ascontiguousarray(k), np.ascontiguousarray(v), w.scale,
+                      nthreads=threads)
+        return n * w.Hkv * w.D * 4
 
-    # calibrate the window so that a step takes about the per-step budget
     n_tok = 1024
     t0 = time.perf_counter()
     sample(0, n_tok)
     dt = max(time.perf_counter() - t0, 1e-6)
-    n_tok = int(max(64, min(int(w.lengths().max()), n_tok * budget_per_step / dt)))
+    n_tok = int(max(16, min(int(lengths.max()), n_tok * budget_per_step / dt)))
     for i in range(args.warmup):
         sample(i, n_tok)
     t0 = time.perf_counter()
@@ -471,9 +476,9 @@ def run_reference(args):
         "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
                    "max_len": w.max_len},
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": f"each step: the {G} query heads of one (sequence, KV head) "
-                                   f"group over a {n_tok}-token window of its history, one thread"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": f"each step: all {w.Hq} query heads of one sequence over a "
+                                   f"{n_tok}-token window of its history, {threads} threads"},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }), flush=True)
