@@ -196,7 +196,13 @@ class Call:
         self.table = None if w.block_table is None else torch.from_numpy(w.block_table).to(device)
         self.prob = fd.make_problem(w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size, w.num_blocks,
                                     w.max_blocks_per_seq)
-        self.S = num_splits or fd.fd_plan(w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size)
+        if num_splits:
+            self.S = num_splits
+        elif w.seqlens is not None:  # lengths known on the host: length-aware planner
+            self.S = fd.fd_plan_seqlens(0, w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size,
+                                        w.seqlens)
+        else:
+            self.S = fd.fd_plan(w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size)
         assert self.S >= 1, fd.fd_status_string(self.S)
         chunk = fd.fd_split_chunk(w.max_len, self.S)
         self.s_eff = max(1, -(-w.max_len // chunk)) if w.max_len else 1
@@ -217,6 +223,22 @@ class Call:
                                self.ws, self.wbytes, self.stream)
         if st != 0:
             raise RuntimeError(f"fd_decode: {self.fd.fd_status_string(st)}")
+
+
+def max_over_ranks(torch, ms, world, device=None):
+    """The slowest rank's time: the job is done when every rank is done."""
+    if world <= 1:
+        return float(ms)
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_rank_step, ms_total, steps, world):
+    """Whole-job GB/s: every rank's algorithmic bytes over the slowest rank's time."""
+    per_step_s = ms_total / 1e3 / steps
+    return world * bytes_per_rank_step / per_step_s / 1e9
 
 
 def timed(torch, fn, steps, warmup, barrier=None):
@@ -320,13 +342,9 @@ def run_fd(args):
     clocks = sampler.stop()
     assert fd.fd_check_device_error() == 0
 
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(torch, ms, world, device)
     per_call_s = ms / 1e3 / args.steps
-    value = world * kvb / per_call_s / 1e9
+    value = job_throughput(kvb, ms, args.steps, world)
     peak, peak_kind = measured_peak()
     achieved = kvb / per_call_s / 1e9
 
@@ -387,16 +405,11 @@ def e2e(torch, fd, call, w, device, steps, warmup, barrier, world):
         ho.copy_(call.out, non_blocking=True)
         hl.copy_(call.lse, non_blocking=True)
 
-    ms = timed(torch, step, steps, warmup, barrier)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(torch, timed(torch, step, steps, warmup, barrier), world, device)
     per = ms / 1e3 / steps
     h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2
     d2h = ho.numel() * 2 + hl.numel() * 4
-    return {"value": round(world * w.kv_bytes() / per / 1e9, 2), "unit": "GB/s",
+    return {"value": round(job_throughput(w.kv_bytes(), ms, steps, world), 2), "unit": "GB/s",
             "us_per_call": round(per * 1e6, 1), "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps}
 

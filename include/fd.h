@@ -104,6 +104,20 @@ FD_API int fd_plan(int B, int Hq, int Hkv, int D, int max_len, int block_size);
 FD_API int fd_plan_sm(int num_sms, int B, int Hq, int Hkv, int D, int max_len,
                int block_size);
 
+/* Split-count planner that also sees the sequence lengths of the batch.
+ * Same rule as fd_plan, with one difference. When the lengths differ,
+ * splitting also evens out the work per CTA: one long sequence would
+ * otherwise decide the end of the call. This planner therefore models the
+ * actual per-sequence lengths instead of assuming max_len for every sequence.
+ *   num_sms   SM count to plan for; <= 0 means the current device's
+ *   seqlens   HOST array [B] of valid tokens per sequence, clamped to
+ *             [0, max_len] as in fd_decode
+ * Returns S >= 1, or a negative fd_status (a NULL seqlens is
+ * FD_ERR_INVALID_ARGUMENT). Host only and deterministic. It costs O(B)
+ * per candidate split count. */
+FD_API int fd_plan_seqlens(int num_sms, int B, int Hq, int Hkv, int D, int max_len,
+                           int block_size, const int32_t* seqlens);
+
 /* Tokens per split for a given split count. This is ceil(max_len /
  * num_splits) rounded up to the 64-token tile. Split s covers tokens
  * [s*chunk, (s+1)*chunk) of every sequence, and splits past a sequence's end
@@ -196,6 +210,15 @@ FD_API fd_status fd_decode_static_workspace(const fd_problem* p, const void* q,
  * A kernel sets that word when one of its bounded waits runs out. Returns
  * FD_OK, FD_ERR_DEVICE_TIMEOUT, or FD_ERR_CUDA. */
 FD_API fd_status fd_check_device_error(fd_stream_t stream);
+
+/* Diagnostic of the failure path. Launches one warp that waits, with the
+ * same bounded wait the kernels use, on an mbarrier that nothing ever
+ * completes. After limit_us microseconds the wait gives up, and the kernel
+ * sets the device error word the way a stalled split kernel would. The next
+ * fd_check_device_error(stream) then returns FD_ERR_DEVICE_TIMEOUT and
+ * clears the word. Nothing faults or hangs, and the context stays usable.
+ * limit_us must be in [1, 5,000,000]. Returns FD_OK once launched. */
+FD_API fd_status fd_selftest_device_timeout(unsigned int limit_us, fd_stream_t stream);
 
 /* Static, human-readable name of a status code. */
 FD_API const char* fd_status_string(fd_status status);

@@ -27,8 +27,9 @@ FD_ERR_CUDA = -4
 FD_ERR_DEVICE_TIMEOUT = -5
 
 # Entry points declared in include/fd.h.
-EXPORTS = ("fd_plan", "fd_plan_sm", "fd_split_chunk", "fd_workspace_bytes", "fd_decode",
-           "fd_decode_static_workspace", "fd_check_device_error", "fd_status_string")
+EXPORTS = ("fd_plan", "fd_plan_sm", "fd_plan_seqlens", "fd_split_chunk", "fd_workspace_bytes", "fd_decode",
+           "fd_decode_static_workspace", "fd_check_device_error", "fd_selftest_device_timeout",
+           "fd_status_string")
 
 # Mirrors FD_STATIC_WORKSPACE_BYTES in include/fd.h.
 FD_STATIC_WORKSPACE_BYTES = 8 << 20
@@ -63,6 +64,8 @@ def load_library(path: str = LIB_PATH):
         lib.fd_plan.restype = I
         lib.fd_plan_sm.argtypes = [I] * 7
         lib.fd_plan_sm.restype = I
+        lib.fd_plan_seqlens.argtypes = [I] * 7 + [vp]
+        lib.fd_plan_seqlens.restype = I
         lib.fd_split_chunk.argtypes = [I, I]
         lib.fd_split_chunk.restype = I
         lib.fd_workspace_bytes.argtypes = [I, I, I, I]
@@ -73,6 +76,8 @@ def load_library(path: str = LIB_PATH):
         lib.fd_decode_static_workspace.argtypes = [ctypes.POINTER(fd_problem), vp, vp, vp, vp,
                                                    vp, F, I, vp, vp, vp]
         lib.fd_decode_static_workspace.restype = I
+        lib.fd_selftest_device_timeout.argtypes = [ctypes.c_uint, vp]
+        lib.fd_selftest_device_timeout.restype = I
         lib.fd_check_device_error.argtypes = [vp]
         lib.fd_check_device_error.restype = I
         lib.fd_status_string.argtypes = [I]
@@ -114,6 +119,16 @@ def fd_plan_sm(num_sms: int, B: int, Hq: int, Hkv: int, D: int, max_len: int,
     return int(load_library().fd_plan_sm(num_sms, B, Hq, Hkv, D, max_len, block_size))
 
 
+def fd_plan_seqlens(num_sms: int, B: int, Hq: int, Hkv: int, D: int, max_len: int,
+                    block_size: int, seqlens) -> int:
+    """Length-aware planner; `seqlens` is a host sequence of B ints (0 or a
+    negative num_sms plans for the current device)."""
+    import numpy as np
+    sl = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32))
+    return int(load_library().fd_plan_seqlens(num_sms, B, Hq, Hkv, D, max_len, block_size,
+                                              sl.ctypes.data))
+
+
 def fd_split_chunk(max_len: int, num_splits: int) -> int:
     return int(load_library().fd_split_chunk(max_len, num_splits))
 
@@ -144,6 +159,10 @@ def fd_decode_static_workspace(problem: fd_problem, q, k_cache, v_cache, seqlens
 
 def fd_check_device_error(stream=None) -> int:
     return int(load_library().fd_check_device_error(_stream(stream)))
+
+
+def fd_selftest_device_timeout(limit_us: int, stream=None) -> int:
+    return int(load_library().fd_selftest_device_timeout(int(limit_us), _stream(stream)))
 
 
 # ---- convenience wrapper -----------------------------------------------------

@@ -65,21 +65,53 @@ double wave_time_us(double cta_bytes, double k, int num_sms, double solo_gbs) {
   return cta_bytes / (std::min(share, limit) * 1e3) + PlanModel::kCtaFixedUs;
 }
 
-double model_time_us(int num_sms, int B, int Hkv, int D, int max_len, int block_size, int S) {
-  const int chunk = chunk_for(max_len, S);
-  const int s_eff = effective_splits(max_len, chunk);
-  const double units = static_cast<double>(B) * Hkv * s_eff;
+// Time of one call whose split kernel runs n_ctas non-empty CTAs moving
+// bytes_total bytes, the largest CTA moving max_cta bytes.  The larger of two
+// estimates: waves of CTAs of the mean size, and the largest CTA on its own
+// (which decides the end when lengths differ).
+double model_time_us(int num_sms, int block_size, double n_ctas, double bytes_total,
+                     double max_cta, int s_eff) {
+  if (n_ctas <= 0) return PlanModel::kCtaFixedUs;
   const double slots = static_cast<double>(num_sms) * fd::kCtasPerSm;
-  const double cta_bytes = std::min<double>(chunk, max_len) * D * 4.0;
   const double solo = (block_size > 0 && block_size < fd::kTile) ? PlanModel::kCtaPagedGBs
                                                                  : PlanModel::kCtaGBs;
-  const double full_waves = std::floor(units / slots);
-  const double rem = units - full_waves * slots;
-  double t = 0.0;
-  if (full_waves > 0) t += full_waves * wave_time_us(cta_bytes, slots, num_sms, solo);
-  if (rem > 0) t += wave_time_us(cta_bytes, rem, num_sms, solo);
+  const double mean = bytes_total / n_ctas;
+  const double full_waves = std::floor(n_ctas / slots);
+  const double rem = n_ctas - full_waves * slots;
+  double waves = 0.0;
+  if (full_waves > 0) waves += full_waves * wave_time_us(mean, slots, num_sms, solo);
+  if (rem > 0) waves += wave_time_us(mean, rem, num_sms, solo);
+  const double longest = wave_time_us(max_cta, std::min(n_ctas, slots), num_sms, solo);
+  double t = std::max(waves, longest);
   if (s_eff > 1) t += PlanModel::kCombineUs;
   return t;
+}
+
+// The model for a batch whose sequences all hold max_len tokens.
+double model_time_uniform(int num_sms, int B, int Hkv, int D, int max_len, int block_size,
+                          int S) {
+  const int chunk = chunk_for(max_len, S);
+  const int s_eff = effective_splits(max_len, chunk);
+  const double units = static_cast<double>(B) * Hkv;
+  const double bytes = units * max_len * D * 4.0;
+  const double max_cta = std::min<double>(chunk, max_len) * D * 4.0;
+  return model_time_us(num_sms, block_size, units * s_eff, bytes, max_cta, s_eff);
+}
+
+// The model for given per-sequence lengths (clamped to [0, max_len]).
+double model_time_lengths(int num_sms, int B, int Hkv, int D, int max_len, int block_size,
+                          const int32_t* lens, int S) {
+  const int chunk = chunk_for(max_len, S);
+  const int s_eff = effective_splits(max_len, chunk);
+  double n_ctas = 0.0, tokens = 0.0, max_tok = 0.0;
+  for (int b = 0; b < B; ++b) {
+    const double n = std::min<double>(std::max<int32_t>(lens[b], 0), max_len);
+    n_ctas += std::ceil(n / chunk);
+    tokens += n;
+    max_tok = std::max(max_tok, std::min<double>(n, chunk));
+  }
+  return model_time_us(num_sms, block_size, n_ctas * Hkv, tokens * Hkv * D * 4.0,
+                       max_tok * D * 4.0, s_eff);
 }
 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
@@ -250,6 +282,29 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// The split count with the lowest modelled time; a larger count must win by
+// more than 2 % (fewer splits mean fewer partials to merge).
+template <class Model>
+int pick_splits(int max_len, Model model) {
+  const long long tiles = (static_cast<long long>(max_len) + fd::kTile - 1) / fd::kTile;
+  if (tiles <= 1) return 1;
+  const int s_max = static_cast<int>(std::min<long long>(tiles, kMaxSplits));
+  int best = 1;
+  double best_t = model(1);
+  int last_eff = 1;
+  for (int S = 2; S <= s_max; ++S) {
+    const int eff = effective_splits(max_len, chunk_for(max_len, S));
+    if (eff == last_eff) continue;  // same chunking as a smaller S
+    last_eff = eff;
+    const double t = model(S);
+    if (t < best_t * 0.98) {
+      best_t = t;
+      best = S;
+    }
+  }
+  return best;
+}
+
 }  // namespace
 
 extern "C" {
@@ -275,25 +330,25 @@ int fd_plan_sm(int num_sms, int B, int Hq, int Hkv, int D, int max_len, int bloc
   if (num_sms < 1) return FD_ERR_INVALID_ARGUMENT;
   const fd_status st = check_shape(B, Hq, Hkv, D, max_len, block_size);
   if (st != FD_OK) return st;
-  const long long tiles = (static_cast<long long>(max_len) + fd::kTile - 1) / fd::kTile;
-  if (tiles <= 1) return 1;
   // Enough (sequence, KV head) units to fill every CTA slot: no split.
   if (static_cast<long long>(B) * Hkv >= static_cast<long long>(num_sms) * fd::kCtasPerSm) return 1;
-  const int s_max = static_cast<int>(std::min<long long>(tiles, kMaxSplits));
-  int best = 1;
-  double best_t = model_time_us(num_sms, B, Hkv, D, max_len, block_size, 1);
-  int last_eff = 1;
-  for (int S = 2; S <= s_max; ++S) {
-    const int eff = effective_splits(max_len, chunk_for(max_len, S));
-    if (eff == last_eff) continue;  // same chunking as a smaller S
-    last_eff = eff;
-    const double t = model_time_us(num_sms, B, Hkv, D, max_len, block_size, S);
-    if (t < best_t * 0.98) {  // prefer fewer splits unless clearly faster
-      best_t = t;
-      best = S;
-    }
+  return pick_splits(max_len, [&](int S) {
+    return model_time_uniform(num_sms, B, Hkv, D, max_len, block_size, S);
+  });
+}
+
+int fd_plan_seqlens(int num_sms, int B, int Hq, int Hkv, int D, int max_len, int block_size,
+                    const int32_t* seqlens) {
+  const fd_status st = check_shape(B, Hq, Hkv, D, max_len, block_size);
+  if (st != FD_OK) return st;
+  if (!seqlens) return FD_ERR_INVALID_ARGUMENT;
+  if (num_sms < 1) {
+    int dev = 0;
+    if (current_device(&dev) != FD_OK || device_sms(dev, &num_sms) != FD_OK) return FD_ERR_CUDA;
   }
-  return best;
+  return pick_splits(max_len, [&](int S) {
+    return model_time_lengths(num_sms, B, Hkv, D, max_len, block_size, seqlens, S);
+  });
 }
 
 int fd_plan(int B, int Hq, int Hkv, int D, int max_len, int block_size) {
@@ -426,6 +481,15 @@ fd_status fd_decode_static_workspace(const fd_problem* p, const void* q, const v
   }
   return fd_decode(p, q, k_cache, v_cache, seqlens, block_table, scale, num_splits, out, lse, ws,
                    FD_STATIC_WORKSPACE_BYTES, stream);
+}
+
+fd_status fd_selftest_device_timeout(unsigned int limit_us, fd_stream_t stream) {
+  if (limit_us == 0 || limit_us > 5000000u) return FD_ERR_INVALID_ARGUMENT;
+  int dev = 0;
+  if (current_device(&dev) != FD_OK) return FD_ERR_CUDA;
+  fd::fd_wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<unsigned long long>(limit_us) * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? FD_OK : FD_ERR_CUDA;
 }
 
 fd_status fd_check_device_error(fd_stream_t stream) {

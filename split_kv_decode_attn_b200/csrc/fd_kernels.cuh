@@ -598,4 +598,18 @@ __global__ void __launch_bounds__(128) fd_combine_kernel(const SplitArgs a, int 
                  a.out + static_cast<size_t>(row) * D, a.lse ? a.lse + row : nullptr, lane);
 }
 
+// Diagnostic: waits, with the kernels' bounded wait, on an mbarrier that
+// nothing ever arrives on, and reports the timeout through the device error
+// word as the split kernel would.  Nothing faults and nothing hangs.
+__global__ void fd_wait_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) unsigned long long bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const bool ok = mbar_wait(smem_u32(&bar), 0, limit_ns);
+  if (!__all_sync(0xffffffffu, ok) && threadIdx.x == 0) raise_device_error(4u);
+}
+
 }  // namespace fd

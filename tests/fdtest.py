@@ -61,8 +61,14 @@ class OnDevice:
                                w.max_blocks_per_seq)
 
     def plan(self) -> int:
+        """The split count the benchmark uses: the length-aware planner when
+        the lengths are known, else fd_plan."""
         w = self.w
-        s = fd.fd_plan(w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size)
+        if w.seqlens is not None:
+            s = fd.fd_plan_seqlens(0, w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size,
+                                   w.seqlens)
+        else:
+            s = fd.fd_plan(w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size)
         assert s >= 1, fd.fd_status_string(s)
         return s
 

@@ -57,8 +57,9 @@ def test_varlen_batch_with_nan_padding():
     ref, rl = reference(w)
     e = assert_close(got, gl, ref, rl, f"varlen S={S}")
     print(f"varlen planner S={S} errors {e}")
-    got8, gl8, _ = run_gpu(d, 8)
-    assert_close(got8, gl8, ref, rl, "varlen S=8")
+    for S2 in (1, 8, 24):
+        got2, gl2, _ = run_gpu(d, S2)
+        assert_close(got2, gl2, ref, rl, f"varlen S={S2}")
 
 
 def test_paged_cache_block16():
