@@ -63,6 +63,8 @@ def parse_args():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="codellama34b")
     ap.add_argument("--L", type=int, default=None, help="cache length of the codellama34b workload")
     ap.add_argument("--splits", type=int, default=None, help="override the planner's split count")
+    ap.add_argument("--layout", choices=["HND", "NHD"], default="HND",
+                    help="cache dimension order (heads outside tokens, or tokens outside heads)")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -195,7 +197,7 @@ class Call:
         self.seqlens = None if w.seqlens is None else torch.from_numpy(w.seqlens).to(device)
         self.table = None if w.block_table is None else torch.from_numpy(w.block_table).to(device)
         self.prob = fd.make_problem(w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size, w.num_blocks,
-                                    w.max_blocks_per_seq)
+                                    w.max_blocks_per_seq, w.kv_layout)
         if num_splits:
             self.S = num_splits
         elif w.seqlens is not None:  # lengths known on the host: length-aware planner
@@ -264,18 +266,23 @@ def copies_for(torch, nbytes, device):
     return max(2, math.ceil(4 * l2 / max(nbytes, 1))), l2
 
 
-def make_workload(name, L, rank, nthreads=None):
+def make_workload(name, L, rank, nthreads=None, layout="HND"):
     from split_kv_decode_attn_b200 import workloads as wl
     idx, default_L = WORKLOADS[name]
     if idx == 2:
         w = wl.config(2, L=L or default_L, nthreads=nthreads)
     else:
         w = wl.config(idx, nthreads=nthreads)
-    if rank:
+    if rank or layout != "HND":
         # replicas: each rank decodes its own sequences (same shapes)
+        # replicas: rank r decodes its own sequences (same shapes); the token-
+        # major layout draws its cache in that storage order
         w2 = wl.make_problem(w.B, w.Hq, w.Hkv, w.D, w.max_len, wl.CONFIG_SEED_BASE + 1000 * rank + idx,
                              seqlens=w.seqlens, nan_pad=w.seqlens is not None and not w.paged,
-                             block_size=w.block_size, name=w.name, nthreads=nthreads)
+                             block_size=w.block_size, name=w.name + ("" if layout == "HND" else "-NHD"),
+                             nthreads=nthreads, layout=layout)
+        if "dominant_positions" in w.meta and layout == "HND":
+            wl.plant_dominant_keys(w2, 64, wl.CONFIG_SEED_BASE + 1000 * rank + idx)
         w = w2
     return w
 
@@ -296,7 +303,7 @@ def cpu_baseline(w, seconds):
     while True:
         b = calls % w.B
         n = int(lengths[b])
-        if w.paged:
+        if w.paged or w.layout != "HND":
             kv = [w.logical_kv(b, h) for h in range(w.Hkv)]
             k = np.stack([x[0] for x in kv])[None]
             v = np.stack([x[1] for x in kv])[None]
@@ -331,7 +338,7 @@ def run_fd(args):
     device = torch.device("cuda", torch.cuda.current_device())
     fd.load_library()
 
-    w = make_workload(args.workload, args.L, rank)
+    w = make_workload(args.workload, args.L, rank, layout=args.layout)
     kvb = w.kv_bytes()
     copies, l2 = copies_for(torch, (w.k.nbytes + w.v.nbytes), device)
     call = Call(torch, fd, w, device, args.splits, copies)
@@ -448,7 +455,7 @@ def run_reference(args):
         return
     import numpy as np
     import oracle
-    w = make_workload(args.workload, args.L, 0)
+    w = make_workload(args.workload, args.L, 0, layout=args.layout)
     cores = os.cpu_count() or 1
     threads = min(cores, w.Hq)
     lengths = w.lengths()
@@ -459,7 +466,7 @@ def run_reference(args):
         b = seqs[i % len(seqs)]
         n = min(n_tok, int(lengths[b]))
         off = (i * 7919) % max(int(lengths[b]) - n + 1, 1)
-        if w.paged:
+        if w.paged or w.layout != "HND":
             kv = [w.logical_kv(b, h) for h in range(w.Hkv)]
             k = np.stack([x[0][off:off + n] for x in kv])[None]
             v = np.stack([x[1][off:off + n] for x in kv])[None]

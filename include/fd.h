@@ -52,7 +52,7 @@ typedef enum fd_status {
   FD_OK = 0,
   /* Null pointer, non-positive size, Hq % Hkv != 0, a tensor pointer not
    * 16-byte aligned (lse: 4-byte), num_splits outside [1, 1024], scale not
-   * finite and positive, seqlen-independent shape limits exceeded. */
+   * finite and positive, unknown kv_layout, shape limits exceeded. */
   FD_ERR_INVALID_ARGUMENT = -1,
   /* Head dim D not in {64, 128}, group size Hq/Hkv not in {1, 2, 4, 8, 16},
    * block_size not a power of two in [8, 256], or the device is not sm_100. */
@@ -66,6 +66,14 @@ typedef enum fd_status {
   FD_ERR_DEVICE_TIMEOUT = -5
 } fd_status;
 
+/* Order of the cache dimensions (see fd_decode for the full shapes). */
+typedef enum fd_kv_layout {
+  /* heads outside tokens: [B, Hkv, max_len, D] or [num_blocks, Hkv, block_size, D] */
+  FD_LAYOUT_HND = 0,
+  /* tokens outside heads: [B, max_len, Hkv, D] or [num_blocks, block_size, Hkv, D] */
+  FD_LAYOUT_NHD = 1
+} fd_kv_layout;
+
 /* Shape of one decode-attention call.
  *   B           sequences in the batch (1 .. 65535)
  *   Hq, Hkv     query heads and KV heads (Hkv .. 65535, Hq % Hkv == 0)
@@ -75,7 +83,8 @@ typedef enum fd_status {
  *               (<= max_blocks_per_seq * block_size)
  *   block_size  0 for a contiguous cache; otherwise tokens per page
  *   num_blocks  paged cache: pages in the pool (ignored when contiguous)
- *   max_blocks_per_seq  paged cache: row length of block_table */
+ *   max_blocks_per_seq  paged cache: row length of block_table
+ *   kv_layout   an fd_kv_layout value (FD_LAYOUT_HND when zero-initialised) */
 typedef struct fd_problem {
   int32_t B;
   int32_t Hq;
@@ -85,6 +94,7 @@ typedef struct fd_problem {
   int32_t block_size;
   int32_t num_blocks;
   int32_t max_blocks_per_seq;
+  int32_t kv_layout;
 } fd_problem;
 
 /* Split-count planner.
@@ -136,9 +146,11 @@ FD_API size_t fd_workspace_bytes(int B, int Hq, int D, int num_splits);
  *   p            shape (see fd_problem)
  *   q            [B, Hq, D] bf16, 16-byte aligned
  *   k_cache, v_cache
- *                contiguous: [B, Hkv, max_len, D] bf16;
- *                paged:      [num_blocks, Hkv, block_size, D] bf16;
- *                16-byte aligned
+ *                FD_LAYOUT_HND contiguous: [B, Hkv, max_len, D] bf16;
+ *                FD_LAYOUT_HND paged:      [num_blocks, Hkv, block_size, D];
+ *                FD_LAYOUT_NHD contiguous: [B, max_len, Hkv, D];
+ *                FD_LAYOUT_NHD paged:      [num_blocks, block_size, Hkv, D];
+ *                row-major, 16-byte aligned
  *   seqlens      [B] int32 valid tokens per sequence, or NULL (all max_len).
  *                Values are clamped to [0, max_len]. Rows at or past a
  *                sequence's length are never summed; they may hold anything,

@@ -42,11 +42,15 @@ class FdError(RuntimeError):
                          else f"{fd_status_string(status)} ({status})")
 
 
+FD_LAYOUT_HND = 0  # cache [.., Hkv, tokens, D]
+FD_LAYOUT_NHD = 1  # cache [.., tokens, Hkv, D]
+
+
 class fd_problem(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
                 ("D", ctypes.c_int32), ("max_len", ctypes.c_int32),
                 ("block_size", ctypes.c_int32), ("num_blocks", ctypes.c_int32),
-                ("max_blocks_per_seq", ctypes.c_int32)]
+                ("max_blocks_per_seq", ctypes.c_int32), ("kv_layout", ctypes.c_int32)]
 
 
 _lib = None
@@ -167,31 +171,43 @@ def fd_selftest_device_timeout(limit_us: int, stream=None) -> int:
 
 # ---- convenience wrapper -----------------------------------------------------
 
-def make_problem(B, Hq, Hkv, D, max_len, block_size=0, num_blocks=0, max_blocks_per_seq=0):
-    return fd_problem(B, Hq, Hkv, D, max_len, block_size, num_blocks, max_blocks_per_seq)
+def make_problem(B, Hq, Hkv, D, max_len, block_size=0, num_blocks=0, max_blocks_per_seq=0,
+                 kv_layout=FD_LAYOUT_HND):
+    return fd_problem(B, Hq, Hkv, D, max_len, block_size, num_blocks, max_blocks_per_seq,
+                      kv_layout)
 
 
 def decode(q, k_cache, v_cache, seqlens=None, block_table=None, *, max_len: Optional[int] = None,
-           block_size: int = 0, scale: Optional[float] = None, num_splits: Optional[int] = None,
-           out=None, lse=None, workspace=None, stream=None):
+           kv_layout: int = FD_LAYOUT_HND, scale: Optional[float] = None,
+           num_splits: Optional[int] = None, out=None, lse=None, workspace=None, stream=None):
     """Decode attention on torch CUDA tensors.
 
-    q [B, Hq, D] bf16; contiguous caches [B, Hkv, max_len, D] bf16, or paged
-    caches [num_blocks, Hkv, block_size, D] with block_table [B, max_blocks]
-    int32; seqlens [B] int32 or None.  Returns (out [B, Hq, D] bf16,
-    lse [B, Hq] fp32).  num_splits defaults to fd_plan's choice."""
+    q [B, Hq, D] bf16.  Caches (bf16): FD_LAYOUT_HND contiguous
+    [B, Hkv, max_len, D] or paged [num_blocks, Hkv, block_size, D];
+    FD_LAYOUT_NHD contiguous [B, max_len, Hkv, D] or paged
+    [num_blocks, block_size, Hkv, D].  Paged caches come with block_table
+    [B, max_blocks] int32.  seqlens [B] int32 or None.  Returns
+    (out [B, Hq, D] bf16, lse [B, Hq] fp32).  num_splits defaults to
+    fd_plan's choice."""
     import torch
     B, Hq, D = q.shape
+    block_size = 0
     if block_table is None:
-        _, Hkv, L, _ = k_cache.shape
+        if kv_layout == FD_LAYOUT_HND:
+            _, Hkv, L, _ = k_cache.shape
+        else:
+            _, L, Hkv, _ = k_cache.shape
         max_len = L if max_len is None else max_len
-        prob = make_problem(B, Hq, Hkv, D, max_len)
+        prob = make_problem(B, Hq, Hkv, D, max_len, kv_layout=kv_layout)
     else:
-        nb, Hkv, bs, _ = k_cache.shape
+        if kv_layout == FD_LAYOUT_HND:
+            nb, Hkv, bs, _ = k_cache.shape
+        else:
+            nb, bs, Hkv, _ = k_cache.shape
         block_size = bs
         mbps = block_table.shape[1]
         max_len = mbps * bs if max_len is None else max_len
-        prob = make_problem(B, Hq, Hkv, D, max_len, bs, nb, mbps)
+        prob = make_problem(B, Hq, Hkv, D, max_len, bs, nb, mbps, kv_layout)
     if scale is None:
         scale = 1.0 / (D ** 0.5)
     if num_splits is None:

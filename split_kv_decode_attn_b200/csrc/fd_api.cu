@@ -36,7 +36,7 @@ constexpr int kMaxDevices = 64;
 struct PlanModel {
   static constexpr double kHbmGBs = 6500.0;
   static constexpr double kCtaGBs = 50.0;
-  static constexpr double kCtaPagedGBs = 30.0;
+  static constexpr double kCtaPagedGBs = 45.0;
   static constexpr double kSmPairGBs = 54.0;
   static constexpr double kCtaFixedUs = 0.5;
   static constexpr double kCombineUs = 1.0;
@@ -191,19 +191,31 @@ fd_status encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
   return g_encode ? FD_OK : FD_ERR_CUDA;
 }
 
-// 3-D view {D, rows, planes} of a bf16 cache, box {64, box_rows, 1}, 128-byte
-// swizzle, zero fill outside the tensor.
-fd_status make_cache_map(CUtensorMap* tm, const void* base, int D, long long rows,
-                         long long planes, int box_rows) {
+// 5-D view {64 columns, head, row, column half, plane} of a bf16 cache, box
+// {64, 1, box_rows, D/64, 1}: one copy brings both 64-column halves of
+// box_rows rows of one KV head, landing as [half][row][64] with the 128-byte
+// swizzle.  The strides place heads, rows and planes for each layout:
+//   HND contiguous [B, Hkv, L, D]     HND paged [pages, Hkv, bs, D]
+//   NHD contiguous [B, L, Hkv, D]     NHD paged [pages, bs, Hkv, D]
+// A plane is a sequence (contiguous) or a page (paged).  Coordinates outside
+// the view read zeros.
+fd_status make_cache_map(CUtensorMap* tm, const void* base, int D, int Hkv, long long rows,
+                         long long planes, int layout, int box_rows) {
   PFN_cuTensorMapEncodeTiled_v12000 enc;
   if (encoder(&enc) != FD_OK) return FD_ERR_CUDA;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
-                        static_cast<cuuint64_t>(planes)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
-                           static_cast<cuuint64_t>(rows) * D * 2};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+  const cuuint64_t row_bytes = static_cast<cuuint64_t>(D) * 2;
+  const cuuint64_t head_stride =
+      layout == FD_LAYOUT_HND ? static_cast<cuuint64_t>(rows) * row_bytes : row_bytes;
+  const cuuint64_t row_stride =
+      layout == FD_LAYOUT_HND ? row_bytes : static_cast<cuuint64_t>(Hkv) * row_bytes;
+  const cuuint64_t plane_stride = static_cast<cuuint64_t>(Hkv) * rows * row_bytes;
+  const int halves = D / 64;
+  cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(Hkv), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(halves), static_cast<cuuint64_t>(planes)};
+  cuuint64_t strides[4] = {head_stride, row_stride, 128, plane_stride};
+  cuuint32_t box[5] = {64, 1, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(halves), 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -381,6 +393,7 @@ fd_status fd_decode(const fd_problem* p, const void* q, const void* k_cache,
     if (static_cast<long long>(p->max_blocks_per_seq) * p->block_size < p->max_len)
       return FD_ERR_INVALID_ARGUMENT;
   }
+  if (p->kv_layout != FD_LAYOUT_HND && p->kv_layout != FD_LAYOUT_NHD) return FD_ERR_INVALID_ARGUMENT;
   if (!std::isfinite(scale) || !(scale > 0.f)) return FD_ERR_INVALID_ARGUMENT;
   if (num_splits < 1 || num_splits > kMaxSplits) return FD_ERR_INVALID_ARGUMENT;
   if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
@@ -409,19 +422,13 @@ fd_status fd_decode(const fd_problem* p, const void* q, const void* k_cache,
 
   // ---- tensor maps over the caches
   CUtensorMap tk, tv;
-  if (!paged) {
-    const long long planes = static_cast<long long>(B) * Hkv;
-    const long long rows = p->max_len > 0 ? p->max_len : 1;
-    if (make_cache_map(&tk, k_cache, D, rows, planes, fd::kTile) != FD_OK ||
-        make_cache_map(&tv, v_cache, D, rows, planes, fd::kTile) != FD_OK)
-      return FD_ERR_CUDA;
-  } else {
-    const long long planes = static_cast<long long>(p->num_blocks) * Hkv;
-    const int box_rows = std::min(p->block_size, fd::kTile);
-    if (make_cache_map(&tk, k_cache, D, p->block_size, planes, box_rows) != FD_OK ||
-        make_cache_map(&tv, v_cache, D, p->block_size, planes, box_rows) != FD_OK)
-      return FD_ERR_CUDA;
-  }
+  const int layout = p->kv_layout;
+  const long long rows = paged ? p->block_size : (p->max_len > 0 ? p->max_len : 1);
+  const long long planes = paged ? p->num_blocks : B;
+  const int box_rows = paged ? std::min(p->block_size, fd::kTile) : fd::kTile;
+  if (make_cache_map(&tk, k_cache, D, Hkv, rows, planes, layout, box_rows) != FD_OK ||
+      make_cache_map(&tv, v_cache, D, Hkv, rows, planes, layout, box_rows) != FD_OK)
+    return FD_ERR_CUDA;
 
   fd::SplitArgs a{};
   a.q = static_cast<const __nv_bfloat16*>(q);
@@ -437,6 +444,7 @@ fd_status fd_decode(const fd_problem* p, const void* q, const void* k_cache,
   a.max_len = p->max_len;
   a.block_size = paged ? p->block_size : 0;
   a.log2_block_size = paged ? ilog2(p->block_size) : 0;
+  a.log2_box_rows = ilog2(box_rows);
   a.max_blocks_per_seq = paged ? p->max_blocks_per_seq : 0;
   a.chunk = chunk;
   a.n_splits = n_splits;

@@ -56,6 +56,7 @@ struct SplitArgs {
   int Hq, Hkv, G;
   int max_len;
   int block_size, log2_block_size;
+  int log2_box_rows;            // rows per TMA box: 64, or the page size when smaller
   int max_blocks_per_seq;
   int chunk;                    // tokens per split, a multiple of kTile
   int n_splits;                 // effective split count = gridDim.x
@@ -207,10 +208,16 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
   }
 
   // Row of the 16-token slice this lane addresses for ldmatrix, and its
-  // 128-byte swizzle phase (row mod 8).
+  // 128-byte swizzle phase (row mod 8).  A tile is a stack of TMA boxes of
+  // 2^log2_box_rows rows, each laid out [column half][row][128 bytes].
   const uint32_t rowK = warp * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
   const uint32_t rowV = warp * 16 + (lane >> 4) * 8 + (lane & 7);
   const uint32_t x7 = lane & 7;
+  const uint32_t lgr = a.log2_box_rows;
+  const uint32_t half_bytes = 128u << lgr;                    // one column half of a box
+  const uint32_t box_bytes = half_bytes * (D / 64);
+  const uint32_t offK = (rowK >> lgr) * box_bytes + (rowK & ((1u << lgr) - 1)) * 128;
+  const uint32_t offV = (rowV >> lgr) * box_bytes + (rowV & ((1u << lgr) - 1)) * 128;
   const int r_lo = warp * 16 + (lane >> 2);   // token rows of the C fragment
   const int r_hi = r_lo + 8;
   const float sl2 = a.scale_log2;
@@ -239,7 +246,7 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
 #pragma unroll
     for (int ks = 0; ks < KSTEPS; ++ks) {
       const uint32_t chunk16 = ((ks & 3) << 1) + (lane >> 4);
-      const uint32_t addr = kbase + (ks >> 2) * L::kHalfBytes + rowK * 128 + ((chunk16 ^ x7) << 4);
+      const uint32_t addr = kbase + offK + (ks >> 2) * half_bytes + ((chunk16 ^ x7) << 4);
       uint32_t af[4];
       ldmatrix_x4(addr, af[0], af[1], af[2], af[3]);
 #pragma unroll
@@ -315,7 +322,7 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
 #pragma unroll
     for (int db = 0; db < DBLK; ++db) {
       const uint32_t chunk16 = ((db & 3) << 1) + ((lane >> 3) & 1);
-      const uint32_t addr = vbase + (db >> 2) * L::kHalfBytes + rowV * 128 + ((chunk16 ^ x7) << 4);
+      const uint32_t addr = vbase + offV + (db >> 2) * half_bytes + ((chunk16 ^ x7) << 4);
       uint32_t vf[4];
       ldmatrix_x4_trans(addr, vf[0], vf[1], vf[2], vf[3]);
       // Rows past the valid length may hold anything (NaN included): zero them
@@ -497,7 +504,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     int issued = 0;
     bool ok = true;
     if constexpr (!PAGED) {
-      const int plane = b * a.Hkv + kvh;
       for (int it = 0; it < n_tiles; ++it) {
         const int s = it % STAGES, k = it / STAGES;
         if (k > 0) ok = mbar_wait(bar_empty + 8 * s, (k - 1) & 1, kWaitLimitNs);
@@ -507,11 +513,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           const uint32_t dk = smem_base + s * L::kStageBytes;
           const uint32_t dv = dk + L::kTileBytes;
           mbar_arrive_expect_tx(bar_full + 8 * s, L::kStageBytes);
-#pragma unroll
-          for (int hf = 0; hf < L::kHalves; ++hf) {
-            tma_load_3d(dk + hf * L::kHalfBytes, &tmK, bar_full + 8 * s, hf * 64, t0, plane, policy);
-            tma_load_3d(dv + hf * L::kHalfBytes, &tmV, bar_full + 8 * s, hf * 64, t0, plane, policy);
-          }
+          tma_load_5d(dk, &tmK, bar_full + 8 * s, 0, kvh, t0, 0, b, policy);
+          tma_load_5d(dv, &tmV, bar_full + 8 * s, 0, kvh, t0, 0, b, policy);
         }
         ++issued;
         __syncwarp();
@@ -550,13 +553,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             if (j < valid_pages) {
-              const int plane = pid[j] * a.Hkv + kvh;
-#pragma unroll
-              for (int hf = 0; hf < L::kHalves; ++hf) {
-                const uint32_t off = hf * L::kHalfBytes + j * rows * 128;
-                tma_load_3d(dk + off, &tmK, bar_full + 8 * s, hf * 64, row0, plane, policy);
-                tma_load_3d(dv + off, &tmV, bar_full + 8 * s, hf * 64, row0, plane, policy);
-              }
+              // page j of the tile: both column halves of `rows` rows
+              const uint32_t off = j * rows * 128 * L::kHalves;
+              tma_load_5d(dk + off, &tmK, bar_full + 8 * s, 0, kvh, row0, 0, pid[j], policy);
+              tma_load_5d(dv + off, &tmV, bar_full + 8 * s, 0, kvh, row0, 0, pid[j], policy);
             }
           }
         }

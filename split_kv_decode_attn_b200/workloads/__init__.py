@@ -144,10 +144,11 @@ def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
 class Workload:
     """One decode-attention problem held on the host.
 
-    q: [B, Hq, D] bf16 bits.  Contiguous cache: k, v [B, Hkv, max_len, D].
-    Paged cache: k, v [num_blocks, Hkv, block_size, D] with
-    block_table [B, max_blocks_per_seq] int32.  seqlens: [B] int32 or None
-    (None means every sequence holds max_len tokens)."""
+    q: [B, Hq, D] bf16 bits.  Cache layout "HND": contiguous k, v
+    [B, Hkv, max_len, D], paged [num_blocks, Hkv, block_size, D].  Layout
+    "NHD": contiguous [B, max_len, Hkv, D], paged [num_blocks, block_size,
+    Hkv, D].  Paged caches come with block_table [B, max_blocks_per_seq]
+    int32.  seqlens: [B] int32 or None (every sequence holds max_len)."""
     name: str
     B: int
     Hq: int
@@ -161,7 +162,12 @@ class Workload:
     seqlens: Optional[np.ndarray] = None
     block_size: int = 0
     block_table: Optional[np.ndarray] = None
+    layout: str = "HND"
     meta: dict = field(default_factory=dict)
+
+    @property
+    def kv_layout(self) -> int:
+        return 0 if self.layout == "HND" else 1
 
     @property
     def G(self) -> int:
@@ -191,26 +197,34 @@ class Workload:
     def logical_kv(self, b: int, h: int):
         """K, V rows [n, D] (bf16 bits) of sequence b, KV head h, in token order."""
         n = int(self.lengths()[b])
+        hnd = self.layout == "HND"
         if not self.paged:
-            return self.k[b, h, :n], self.v[b, h, :n]
+            if hnd:
+                return self.k[b, h, :n], self.v[b, h, :n]
+            return self.k[b, :n, h], self.v[b, :n, h]
         bs = self.block_size
         npages = (n + bs - 1) // bs
         pages = self.block_table[b, :npages].astype(np.int64)
-        kk = self.k[pages, h].reshape(-1, self.D)[:n]
-        vv = self.v[pages, h].reshape(-1, self.D)[:n]
-        return kk, vv
+        if hnd:
+            kk, vv = self.k[pages, h], self.v[pages, h]
+        else:
+            kk, vv = self.k[pages, :, h], self.v[pages, :, h]
+        return kk.reshape(-1, self.D)[:n], vv.reshape(-1, self.D)[:n]
 
 
 def make_problem(B: int, Hq: int, Hkv: int, D: int, max_len: int, seed: int,
                  seqlens=None, nan_pad: bool = False, block_size: int = 0,
                  num_blocks: Optional[int] = None, name: str = "custom",
-                 nthreads: Optional[int] = None) -> Workload:
+                 nthreads: Optional[int] = None, layout: str = "HND") -> Workload:
     """Build a workload with i.i.d. N(0,1) bf16 q, K, V from base `seed`.
 
     Contiguous cache when block_size == 0.  Paged cache otherwise: the
     physical pool holds `num_blocks` pages (default: exactly enough for every
     sequence) and the block table is a seeded permutation of the pool,
-    reshaped [B, max_len / block_size]."""
+    reshaped [B, max_len / block_size].  `layout` orders the cache dims
+    ("HND": heads outside tokens, "NHD": tokens outside heads); K and V are
+    drawn in the storage order of that layout."""
+    assert layout in ("HND", "NHD")
     q = normal_bf16(stream_seed(seed, STREAM_Q), (B, Hq, D), nthreads=nthreads)
     if block_size:
         assert max_len % block_size == 0
@@ -219,21 +233,25 @@ def make_problem(B: int, Hq: int, Hkv: int, D: int, max_len: int, seed: int,
         assert nb >= B * per_seq
         perm = permutation(stream_seed(seed, STREAM_PERM), nb)
         table = perm[: B * per_seq].reshape(B, per_seq).copy()
-        shape = (nb, Hkv, block_size, D)
+        shape = (nb, Hkv, block_size, D) if layout == "HND" else (nb, block_size, Hkv, D)
     else:
         table = None
-        shape = (B, Hkv, max_len, D)
+        shape = (B, Hkv, max_len, D) if layout == "HND" else (B, max_len, Hkv, D)
     k = normal_bf16(stream_seed(seed, STREAM_K), shape, nthreads=nthreads)
     v = normal_bf16(stream_seed(seed, STREAM_V), shape, nthreads=nthreads)
     sl = None if seqlens is None else np.asarray(seqlens, dtype=np.int32)
     if nan_pad and sl is not None:
         assert not block_size
         for b in range(B):
-            k[b, :, int(sl[b]):, :] = BF16_NAN
-            v[b, :, int(sl[b]):, :] = BF16_NAN
+            if layout == "HND":
+                k[b, :, int(sl[b]):, :] = BF16_NAN
+                v[b, :, int(sl[b]):, :] = BF16_NAN
+            else:
+                k[b, int(sl[b]):, :, :] = BF16_NAN
+                v[b, int(sl[b]):, :, :] = BF16_NAN
     return Workload(name=name, B=B, Hq=Hq, Hkv=Hkv, D=D, max_len=max_len, q=q, k=k, v=v,
                     scale=float(np.float32(1.0 / math.sqrt(D))), seqlens=sl,
-                    block_size=block_size, block_table=table)
+                    block_size=block_size, block_table=table, layout=layout)
 
 
 def plant_dominant_keys(w: Workload, count: int, seed: int, magnitude: float = 4.0) -> np.ndarray:
@@ -241,7 +259,7 @@ def plant_dominant_keys(w: Workload, count: int, seed: int, magnitude: float = 4
     magnitude * q/|q| * sqrt(D), q being the group's first query head of that
     KV head (batch entry 0 .. B-1 alike), computed in fp64 and rounded to bf16.
     Returns the positions."""
-    assert not w.paged
+    assert not w.paged and w.layout == "HND"
     pos = distinct_positions(stream_seed(seed, STREAM_POS), count, w.max_len)
     G = w.G
     for b in range(w.B):

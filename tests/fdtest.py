@@ -58,7 +58,7 @@ class OnDevice:
     def problem(self):
         w = self.w
         return fd.make_problem(w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size, w.num_blocks,
-                               w.max_blocks_per_seq)
+                               w.max_blocks_per_seq, w.kv_layout)
 
     def plan(self) -> int:
         """The split count the benchmark uses: the length-aware planner when
@@ -102,7 +102,7 @@ def reference(w: wl.Workload, groups=None, nthreads=None):
     computed are NaN.  Paged caches are gathered to logical token order
     first (the oracle only sees logical K/V)."""
     nthreads = nthreads or os.cpu_count() or 1
-    if groups is None and not w.paged:
+    if groups is None and not w.paged and w.layout == "HND":
         return oracle.decode(w.q, w.k, w.v, w.scale, seqlens=w.seqlens, nthreads=nthreads)
     if groups is None:
         groups = [(b, h) for b in range(w.B) for h in range(w.Hkv)]

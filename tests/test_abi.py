@@ -160,6 +160,24 @@ def test_decode_rejects_bad_paging():
     assert decode(P(bs=12, nb=64, mb=64), table=0x60000) == fd.FD_ERR_UNSUPPORTED
 
 
+def test_decode_rejects_unknown_layout():
+    prob = P()
+    prob.kv_layout = 2
+    assert decode(prob) == fd.FD_ERR_INVALID_ARGUMENT
+    prob.kv_layout = -1
+    assert decode(prob) == fd.FD_ERR_INVALID_ARGUMENT
+
+
+def test_problem_struct_matches_header():
+    import ctypes
+    # nine int32 fields, in the order of fd_problem in include/fd.h
+    assert ctypes.sizeof(fd.fd_problem) == 9 * 4
+    names = [f[0] for f in fd.fd_problem._fields_]
+    text = open(os.path.join(ROOT, "include", "fd.h")).read()
+    body = text[text.index("typedef struct fd_problem {"):text.index("} fd_problem;")]
+    assert names == re.findall(r"int32_t (\w+);", body)
+
+
 def test_decode_rejects_bad_scalars():
     assert decode(P(), scale=0.0) == fd.FD_ERR_INVALID_ARGUMENT
     assert decode(P(), scale=-1.0) == fd.FD_ERR_INVALID_ARGUMENT

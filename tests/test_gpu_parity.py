@@ -129,12 +129,13 @@ def test_seqlens_are_clamped():
         assert_close(got, gl, ref, rl, f"clamp S={S}")
 
 
+@pytest.mark.parametrize("layout", ["HND", "NHD"])
 @pytest.mark.parametrize("bs", [8, 16, 32, 64, 128, 256])
-def test_paged_block_sizes_match_contiguous_bit_for_bit(bs):
+def test_paged_block_sizes_match_contiguous_bit_for_bit(bs, layout):
     B, Hq, Hkv, D, L = 3, 32, 8, 128, 1024
     lens = [1024, 517, 64]
     p = wl.make_problem(B, Hq, Hkv, D, L, seed=40 + bs, seqlens=lens, block_size=bs,
-                        num_blocks=B * L // bs + 5)
+                        num_blocks=B * L // bs + 5, layout=layout)
     # the same logical cache, contiguous
     kc = np.zeros((B, Hkv, L, D), np.uint16)
     vc = np.zeros((B, Hkv, L, D), np.uint16)
@@ -150,8 +151,28 @@ def test_paged_block_sizes_match_contiguous_bit_for_bit(bs):
     for S in (1, 5):
         gp, lp, _ = run_gpu(dp, S)
         gc_, lc, _ = run_gpu(dc, S)
-        assert_close(gp, lp, ref, rl, f"paged bs={bs} S={S}")
+        assert_close(gp, lp, ref, rl, f"paged {layout} bs={bs} S={S}")
         assert np.array_equal(gp, gc_) and np.array_equal(lp, lc)
+
+
+@pytest.mark.parametrize("D,G", [(128, 8), (128, 4), (64, 1)])
+def test_token_major_contiguous_cache(D, G):
+    """[B, max_len, Hkv, D] gives the same bits as [B, Hkv, max_len, D]."""
+    B, Hkv, L = 4, 4, 1500
+    lens = [1500, 1, 640, 0]
+    n = wl.make_problem(B, G * Hkv, Hkv, D, L, seed=60 + G, seqlens=lens, nan_pad=True,
+                        layout="NHD")
+    h = wl.Workload(name="hnd", B=B, Hq=n.Hq, Hkv=Hkv, D=D, max_len=L, q=n.q,
+                    k=np.ascontiguousarray(n.k.transpose(0, 2, 1, 3)),
+                    v=np.ascontiguousarray(n.v.transpose(0, 2, 1, 3)),
+                    scale=n.scale, seqlens=n.seqlens)
+    dn, dh = OnDevice(n), OnDevice(h)
+    ref, rl = reference(h)
+    for S in (1, 5, 32):
+        gn, ln_, _ = run_gpu(dn, S)
+        gh, lh, _ = run_gpu(dh, S)
+        assert_close(gn, ln_, ref, rl, f"NHD D={D} G={G} S={S}")
+        assert np.array_equal(gn, gh) and np.array_equal(ln_, lh)
 
 
 # ---- determinism, closed forms, buffers ----------------------------------------

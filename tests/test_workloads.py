@@ -91,3 +91,15 @@ def test_config_recipes_are_the_stated_shapes():
     sl = wl.uniform_int(wl.stream_seed(wl.CONFIG_SEED_BASE + 3, wl.STREAM_SEQLENS),
                         32, 1024, 32768)
     assert sl.min() >= 1024 and sl.max() <= 32768 and len(sl) == 32
+
+
+def test_token_major_layouts():
+    n = wl.make_problem(2, 8, 2, 64, 96, seed=3, seqlens=[96, 50], nan_pad=True, layout="NHD")
+    assert n.k.shape == (2, 96, 2, 64) and n.kv_layout == 1
+    assert np.all(n.k[1, 50:] == wl.BF16_NAN) and not np.any(n.k[0] == wl.BF16_NAN)
+    k, v = n.logical_kv(1, 1)
+    assert k.shape == (50, 64) and np.array_equal(k, n.k[1, :50, 1])
+    p = wl.make_problem(2, 8, 2, 64, 96, seed=3, block_size=16, layout="NHD")
+    assert p.k.shape == (12, 16, 2, 64)
+    k, v = p.logical_kv(0, 1)
+    assert np.array_equal(k[16:32], p.k[p.block_table[0, 1], :, 1])
