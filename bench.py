@@ -65,6 +65,8 @@ def parse_args():
     ap.add_argument("--splits", type=int, default=None, help="override the planner's split count")
     ap.add_argument("--layout", choices=["HND", "NHD"], default="HND",
                     help="cache dimension order (heads outside tokens, or tokens outside heads)")
+    ap.add_argument("--crossover", action="store_true",
+                    help="concurrency sweep: batch x cache length, planner pick vs one split")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -442,6 +444,44 @@ def sweep(torch, fd, device):
     return rows
 
 
+def crossover(args):
+    """Batch size x cache length on the CodeLlama-34B head shape (Hq=64,
+    Hkv=8, D=128, contiguous): one split, the planner's pick, and a ladder of
+    split counts.  One JSON line per (B, L) on stdout."""
+    import torch
+    import split_kv_decode_attn_b200 as fd
+    from split_kv_decode_attn_b200 import workloads as wl
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    fd.load_library()
+    peak, _ = measured_peak()
+    for B in (1, 4, 16, 64, 256):
+        for L in (512, 2048, 8192, 16384, 65536):
+            kv = B * 8 * L * 128 * 4
+            if kv > 9e9:
+                continue
+            w = wl.make_problem(B, 64, 8, 128, L, wl.CONFIG_SEED_BASE + 200 + B, name=f"B{B}-L{L}")
+            copies, _ = copies_for(torch, w.k.nbytes + w.v.nbytes, device)
+            plan = fd.fd_plan(B, 64, 8, 128, L, 0)
+            times = {}
+            for S in sorted({1, plan, 2, 4, 8, 16, 24, 32}):
+                if S > max(1, L // 64):
+                    continue
+                call = Call(torch, fd, w, device, S, copies)
+                est = timed(torch, call, 3, 2) / 3
+                steps = int(max(10, min(5000, 150.0 / max(est, 1e-3))))
+                times[S] = timed(torch, call, steps, 5) / steps * 1e3
+                del call
+            torch.cuda.empty_cache()
+            best = min(times, key=times.get)
+            print(json.dumps({"B": B, "L": L, "kv_bytes": kv, "plan": plan,
+                              "us": {str(k): round(v, 2) for k, v in times.items()},
+                              "best": best, "plan_regret": round(times[plan] / times[best] - 1, 4),
+                              "split_gain_vs_1": round(times[1] / times[plan], 3),
+                              "plan_GBs": round(kv / times[plan] / 1e3, 1),
+                              "plan_frac": round(kv / times[plan] / 1e3 / peak, 4)}), flush=True)
+
+
 # ------------------------------------------------------- reference arm
 
 def run_reference(args):
@@ -508,6 +548,8 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.crossover:
+        crossover(args)
     else:
         run_fd(args)
 

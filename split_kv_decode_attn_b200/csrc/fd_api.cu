@@ -23,23 +23,25 @@ constexpr int kMaxDevices = 64;
 // ---------------------------------------------------------------- planner
 
 // Cost model of one call, in microseconds, used to pick the split count.
-// The constants were fitted to split-count sweeps measured on B200 over the
-// five workload shapes (the planner's pick is the fastest measured split
-// count, or within a few percent of it, on every uniform-length workload):
+// The constants were fitted to split-count sweeps measured on B200: the five
+// workload shapes plus a batch x length grid (B = 1..256, L = 512..64K) on
+// the CodeLlama-34B head shape.  Over those 30 cases the planner's pick is
+// the fastest measured split count or within 5.3 % of it:
 //   kHbmGBs      streaming rate of the whole device
 //   kCtaGBs      rate of one CTA alone on an SM (contiguous cache)
-//   kCtaPagedGBs rate of one CTA alone on an SM when pages hold fewer than
-//                64 tokens (one TMA box per page)
+//   kCtaPagedGBs the same when pages hold fewer than 64 tokens (one TMA box
+//                per page instead of one per tile)
 //   kSmPairGBs   rate of an SM running two CTAs, both together
-//   kCtaFixedUs  per-CTA fixed cost (first-tile latency, epilogue)
-//   kCombineUs   the combine kernel of a call with several splits
+//   kCtaFixedUs  per-CTA fixed cost within a wave
+//   kCombineUs   extra cost of a call with several splits: the combine
+//                kernel, its dependency and the partial results
 struct PlanModel {
   static constexpr double kHbmGBs = 6500.0;
   static constexpr double kCtaGBs = 50.0;
   static constexpr double kCtaPagedGBs = 45.0;
   static constexpr double kSmPairGBs = 54.0;
-  static constexpr double kCtaFixedUs = 0.5;
-  static constexpr double kCombineUs = 1.0;
+  static constexpr double kCtaFixedUs = 0.3;
+  static constexpr double kCombineUs = 5.0;
 };
 
 int tile_round_up(long long x) {
