@@ -263,6 +263,40 @@ def timed(torch, fn, steps, warmup, barrier=None):
     return e0.elapsed_time(e1)  # ms
 
 
+def timed_graph(torch, call, copies, reps, warmup=3):
+    """Device time per call with the calls replayed from a CUDA graph (one
+    captured call per cache copy): the cost of the call itself, free of the
+    host's per-call launch work.  Returns microseconds per call."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    eager_stream = call.stream
+    try:
+        with torch.cuda.stream(s):
+            call.stream = s.cuda_stream
+            for _ in range(copies):
+                call()  # one-time set-up happens outside the capture
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            call.stream = s.cuda_stream
+            for _ in range(copies):
+                call()
+        for _ in range(warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / (reps * copies) * 1e3
+    finally:
+        call.stream = eager_stream
+
+
 def copies_for(torch, nbytes, device):
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     return max(2, math.ceil(4 * l2 / max(nbytes, 1))), l2
@@ -435,9 +469,13 @@ def sweep(torch, fd, device):
         ms = timed(torch, call, steps, 50)
         per = ms / 1e3 / steps
         gbs = w.kv_bytes() / per / 1e9
+        g_us = timed_graph(torch, call, copies, max(1, steps // copies))
+        g_gbs = w.kv_bytes() / (g_us * 1e-6) / 1e9
         rows.append({"L": L, "num_splits": call.S, "effective_splits": call.s_eff,
                      "us_per_call": round(per * 1e6, 3), "GB/s": round(gbs, 1),
                      "frac_measured": round(gbs / peak, 4), "frac_spec": round(gbs / SPEC_HBM_GBS, 4),
+                     "graph_us_per_call": round(g_us, 3), "graph_GB/s": round(g_gbs, 1),
+                     "graph_frac_measured": round(g_gbs / peak, 4),
                      "copies": copies, "steps": steps})
         del call
         torch.cuda.empty_cache()
@@ -447,7 +485,9 @@ def sweep(torch, fd, device):
 def crossover(args):
     """Batch size x cache length on the CodeLlama-34B head shape (Hq=64,
     Hkv=8, D=128, contiguous): one split, the planner's pick, and a ladder of
-    split counts.  One JSON line per (B, L) on stdout."""
+    split counts, timed on the device from CUDA-graph replays (the call's own
+    cost; eager calls below ~2K tokens are bound by the host's launch work).
+    One JSON line per (B, L) on stdout."""
     import torch
     import split_kv_decode_attn_b200 as fd
     from split_kv_decode_attn_b200 import workloads as wl
@@ -470,7 +510,7 @@ def crossover(args):
                 call = Call(torch, fd, w, device, S, copies)
                 est = timed(torch, call, 3, 2) / 3
                 steps = int(max(10, min(5000, 150.0 / max(est, 1e-3))))
-                times[S] = timed(torch, call, steps, 5) / steps * 1e3
+                times[S] = timed_graph(torch, call, copies, max(1, steps // copies))
                 del call
             torch.cuda.empty_cache()
             best = min(times, key=times.get)

@@ -92,9 +92,7 @@ def load_library(path: str = LIB_PATH):
 
 def _ptr(x) -> Optional[int]:
     """Device address of a torch tensor, an int address, or None."""
-    if x is None:
-        return None
-    if isinstance(x, int):
+    if x is None or x.__class__ is int:
         return x or None
     return x.data_ptr() or None
 
@@ -143,11 +141,13 @@ def fd_workspace_bytes(B: int, Hq: int, D: int, num_splits: int) -> int:
 
 def fd_decode(problem: fd_problem, q, k_cache, v_cache, seqlens, block_table, scale: float,
               num_splits: int, out, lse, workspace, workspace_bytes: int, stream=None) -> int:
-    """Call the C fd_decode; returns its status code."""
-    return int(load_library().fd_decode(
-        ctypes.byref(problem), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens),
-        _ptr(block_table), ctypes.c_float(scale), int(num_splits), _ptr(out), _ptr(lse),
-        _ptr(workspace), int(workspace_bytes), _stream(stream)))
+    """Call the C fd_decode; returns its status code.  Tensor arguments may be
+    torch tensors, int device addresses or None; `stream` a torch stream, an
+    int cudaStream_t or None (torch's current stream)."""
+    f = _lib.fd_decode if _lib is not None else load_library().fd_decode
+    return f(ctypes.byref(problem), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens),
+             _ptr(block_table), scale, num_splits, _ptr(out), _ptr(lse), _ptr(workspace),
+             workspace_bytes, _stream(stream))
 
 
 def fd_decode_static_workspace(problem: fd_problem, q, k_cache, v_cache, seqlens, block_table,
