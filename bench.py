@@ -65,6 +65,8 @@ def parse_args():
     ap.add_argument("--splits", type=int, default=None, help="override the planner's split count")
     ap.add_argument("--layout", choices=["HND", "NHD"], default="HND",
                     help="cache dimension order (heads outside tokens, or tokens outside heads)")
+    ap.add_argument("--shard-sequence", action="store_true",
+                    help="sequence-parallel: the ranks split one history (strong scaling)")
     ap.add_argument("--crossover", action="store_true",
                     help="concurrency sweep: batch x cache length, planner pick vs one split")
     ap.add_argument("--no-sweep", action="store_true")
@@ -482,6 +484,96 @@ def sweep(torch, fd, device):
     return rows
 
 
+def run_sharded(args):
+    """Sequence-parallel decode of the CodeLlama-34B-shaped workload: rank r
+    holds tokens [r*L/N, (r+1)*L/N) of every KV head.  A step is the local
+    partial (fd_decode_partial), the all-gather of the partial results and
+    their merge (fd_combine).  value = the whole history's K+V bytes over the
+    slowest rank's time (strong scaling)."""
+    import numpy as np
+    import torch
+    import split_kv_decode_attn_b200 as fd
+    from split_kv_decode_attn_b200 import sharded
+    from split_kv_decode_attn_b200 import workloads as wl
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+        barrier = lambda: dist.barrier(device_ids=[local])  # noqa: E731
+    else:
+        barrier = None
+        torch.cuda.set_device(0)
+    device = torch.device("cuda", torch.cuda.current_device())
+    fd.load_library()
+    L = args.L or WORKLOADS["codellama34b"][1]
+    w = wl.config(2, L=L)  # every rank draws the same history and keeps its slice
+    lo, hi = sharded.shard_bounds(L, world, rank)
+    q = dev_bf16(torch, w.q, device)
+    k0 = dev_bf16(torch, np.ascontiguousarray(w.k[:, :, lo:hi]), device)
+    v0 = dev_bf16(torch, np.ascontiguousarray(w.v[:, :, lo:hi]), device)
+    copies, _ = copies_for(torch, k0.numel() * 4, device)  # rotate slices past L2
+    ks = [k0] + [k0.clone() for _ in range(copies - 1)]
+    vs = [v0] + [v0.clone() for _ in range(copies - 1)]
+    turn = [0]
+    B, Hq, D, Hkv = w.B, w.Hq, w.D, w.Hkv
+    prob = fd.make_problem(B, Hq, Hkv, D, hi - lo)
+    S = args.splits or fd.fd_plan(B, Hq, Hkv, D, hi - lo, 0)
+    nbytes = fd.fd_workspace_bytes(B, Hq, D, S)
+    ws = torch.empty(max(nbytes, 4) // 4, dtype=torch.float32, device=device)
+    o = torch.empty((B, Hq, D), dtype=torch.float32, device=device)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=device)
+    o_all = torch.empty((world, B, Hq, D), dtype=torch.float32, device=device)
+    l_all = torch.empty((world, B, Hq), dtype=torch.float32, device=device)
+    out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=device)
+    lse_out = torch.empty((B, Hq), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device).cuda_stream
+
+    def step():
+        c = turn[0] % copies
+        turn[0] += 1
+        st = fd.fd_decode_partial(prob, q, ks[c], vs[c], None, None, w.scale, S, o, lse, ws,
+                                  nbytes, stream)
+        assert st == 0, fd.fd_status_string(st)
+        if world > 1:
+            import torch.distributed as dist
+            dist.all_gather_into_tensor(o_all, o)
+            dist.all_gather_into_tensor(l_all, lse)
+        else:
+            o_all[0].copy_(o)
+            l_all[0].copy_(lse)
+        st = fd.fd_combine(world, B, Hq, D, o_all, l_all, out, lse_out, stream)
+        assert st == 0, fd.fd_status_string(st)
+
+    ms = max_over_ranks(torch, timed(torch, step, args.steps, args.warmup, barrier), world, device)
+    assert fd.fd_check_device_error() == 0
+    kvb = w.kv_bytes()
+    per = ms / 1e3 / args.steps
+    peak, peak_kind = measured_peak()
+    result = {
+        "metric": METRIC, "value": round(kvb / per / 1e9, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "us_per_call": round(per * 1e6, 3), "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name + f"-seq{world}", "B": B, "Hq": Hq, "Hkv": Hkv, "D": D,
+                   "max_len": L, "tokens_per_rank": hi - lo, "num_splits": S,
+                   "l2": f"each rank rotates {copies} copies of its slice",
+                   "parallelism": f"seq{world}"},
+        "roofline": {"bound": "hbm", "achieved": round(kvb / world / per / 1e9, 1),
+                     "peak": peak, "unit": "GB/s", "peak_kind": peak_kind,
+                     "frac": round(kvb / world / per / 1e9 / peak, 4), "traffic": None},
+        "gpu_launches": args.steps * ((2 if S > 1 else 1) + 1),
+    }
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
 def crossover(args):
     """Batch size x cache length on the CodeLlama-34B head shape (Hq=64,
     Hkv=8, D=128, contiguous): one split, the planner's pick, and a ladder of
@@ -590,6 +682,8 @@ def main():
         run_reference(args)
     elif args.crossover:
         crossover(args)
+    elif args.shard_sequence:
+        run_sharded(args)
     else:
         run_fd(args)
 

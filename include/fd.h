@@ -182,6 +182,43 @@ FD_API fd_status fd_decode(const fd_problem* p, const void* q, const void* k_cac
                     void* out, float* lse, void* workspace,
                     size_t workspace_bytes, fd_stream_t stream);
 
+/* Partial decode over a shard of each sequence's history, for merging
+ * across GPUs (sequence-parallel decode).
+ * When each GPU holds a contiguous slice of every sequence's cached tokens,
+ * each GPU calls this on its own slice. The call returns the exact attention
+ * over that slice: a normalised fp32 output and its log-sum-exp. After the
+ * R results are gathered in one place (for example with an NCCL all-gather),
+ * fd_combine merges them into the attention over the whole history. This is
+ * the same log-sum-exp reduction that merges the splits of one GPU (page
+ * "What is Flash-Decoding, and when does it speed up LLMs?", section "Why
+ * decode needs a different schedule").
+ * Arguments are those of fd_decode, except two outputs:
+ *   out_f32  [B, Hq, D] fp32, 16-byte aligned (required)
+ *   lse      [B, Hq] fp32 (required)
+ * An empty slice gives out_f32 = 0 and lse = -inf, which weighs nothing in
+ * fd_combine. */
+FD_API fd_status fd_decode_partial(const fd_problem* p, const void* q, const void* k_cache,
+                                   const void* v_cache, const int32_t* seqlens,
+                                   const int32_t* block_table, float scale, int num_splits,
+                                   float* out_f32, float* lse, void* workspace,
+                                   size_t workspace_bytes, fd_stream_t stream);
+
+/* Merges R partial results into the final output. Each part covers a
+ * disjoint slice of the history, for example one per GPU from
+ * fd_decode_partial:
+ *   m = max_r lse_r,  out = sum_r e^(lse_r - m) O_r / sum_r e^(lse_r - m),
+ *   lse = m + ln sum_r e^(lse_r - m).
+ *   part_o    [R, B, Hq, D] fp32, 16-byte aligned (parts outermost, as an
+ *             all-gather along a new leading dimension lays them out)
+ *   part_lse  [R, B, Hq] fp32
+ *   out       [B, Hq, D] bf16, round-to-nearest-even, 16-byte aligned
+ *   lse       [B, Hq] fp32 or NULL
+ * R is in [1, 1024] and D is 64 or 128. A row whose parts are all empty gives
+ * out = 0 and lse = -inf. Parts are summed in index order, so the result is
+ * deterministic. It runs asynchronously on `stream`. */
+FD_API fd_status fd_combine(int R, int B, int Hq, int D, const float* part_o,
+                            const float* part_lse, void* out, float* lse, fd_stream_t stream);
+
 /* Largest workspace, in bytes, that fd_decode_static_workspace can use. */
 #define FD_STATIC_WORKSPACE_BYTES (8u << 20)
 

@@ -28,8 +28,8 @@ FD_ERR_DEVICE_TIMEOUT = -5
 
 # Entry points declared in include/fd.h.
 EXPORTS = ("fd_plan", "fd_plan_sm", "fd_plan_seqlens", "fd_split_chunk", "fd_workspace_bytes", "fd_decode",
-           "fd_decode_static_workspace", "fd_check_device_error", "fd_selftest_device_timeout",
-           "fd_status_string")
+           "fd_decode_partial", "fd_combine", "fd_decode_static_workspace", "fd_check_device_error",
+           "fd_selftest_device_timeout", "fd_status_string")
 
 # Mirrors FD_STATIC_WORKSPACE_BYTES in include/fd.h.
 FD_STATIC_WORKSPACE_BYTES = 8 << 20
@@ -77,6 +77,11 @@ def load_library(path: str = LIB_PATH):
         lib.fd_decode.argtypes = [ctypes.POINTER(fd_problem), vp, vp, vp, vp, vp, F, I, vp, vp,
                                   vp, sz, vp]
         lib.fd_decode.restype = I
+        lib.fd_decode_partial.argtypes = [ctypes.POINTER(fd_problem), vp, vp, vp, vp, vp, F, I,
+                                          vp, vp, vp, sz, vp]
+        lib.fd_decode_partial.restype = I
+        lib.fd_combine.argtypes = [I, I, I, I, vp, vp, vp, vp, vp]
+        lib.fd_combine.restype = I
         lib.fd_decode_static_workspace.argtypes = [ctypes.POINTER(fd_problem), vp, vp, vp, vp,
                                                    vp, F, I, vp, vp, vp]
         lib.fd_decode_static_workspace.restype = I
@@ -148,6 +153,24 @@ def fd_decode(problem: fd_problem, q, k_cache, v_cache, seqlens, block_table, sc
     return f(ctypes.byref(problem), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens),
              _ptr(block_table), scale, num_splits, _ptr(out), _ptr(lse), _ptr(workspace),
              workspace_bytes, _stream(stream))
+
+
+def fd_decode_partial(problem: fd_problem, q, k_cache, v_cache, seqlens, block_table,
+                      scale: float, num_splits: int, out_f32, lse, workspace,
+                      workspace_bytes: int, stream=None) -> int:
+    """Call the C fd_decode_partial: exact attention over this shard of the
+    history as fp32 output and lse, for fd_combine.  Returns the status."""
+    return int(load_library().fd_decode_partial(
+        ctypes.byref(problem), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens),
+        _ptr(block_table), scale, num_splits, _ptr(out_f32), _ptr(lse), _ptr(workspace),
+        workspace_bytes, _stream(stream)))
+
+
+def fd_combine(R: int, B: int, Hq: int, D: int, part_o, part_lse, out, lse, stream=None) -> int:
+    """Call the C fd_combine: merge R partials [R, B, Hq, D] / [R, B, Hq].
+    Returns the status."""
+    return int(load_library().fd_combine(R, B, Hq, D, _ptr(part_o), _ptr(part_lse), _ptr(out),
+                                         _ptr(lse), _stream(stream)))
 
 
 def fd_decode_static_workspace(problem: fd_problem, q, k_cache, v_cache, seqlens, block_table,

@@ -356,6 +356,93 @@ int pick_splits(int max_len, Model model) {
   return best;
 }
 
+// One decode call.  The result goes to `out` (bf16) or, for a partial over a
+// shard of the history, to `out_f32` (fp32); exactly one of them is set.
+fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
+                      const void* v_cache, const int32_t* seqlens, const int32_t* block_table,
+                      float scale, int num_splits, void* out, float* out_f32, float* lse,
+                      void* workspace, size_t workspace_bytes, fd_stream_t stream) {
+  // ---- host-side checks: nothing is launched for an invalid call
+  if (!p || !q || !k_cache || !v_cache || (!out == !out_f32)) return FD_ERR_INVALID_ARGUMENT;
+  const fd_status st = check_shape(p->B, p->Hq, p->Hkv, p->D, p->max_len, p->block_size);
+  if (st != FD_OK) return st;
+  const bool paged = p->block_size != 0;
+  if (paged != (block_table != nullptr)) return FD_ERR_INVALID_ARGUMENT;
+  if (paged) {
+    if (p->num_blocks < 1 || p->max_blocks_per_seq < 1) return FD_ERR_INVALID_ARGUMENT;
+    if (static_cast<long long>(p->max_blocks_per_seq) * p->block_size < p->max_len)
+      return FD_ERR_INVALID_ARGUMENT;
+  }
+  if (p->kv_layout != FD_LAYOUT_HND && p->kv_layout != FD_LAYOUT_NHD) return FD_ERR_INVALID_ARGUMENT;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return FD_ERR_INVALID_ARGUMENT;
+  if (num_splits < 1 || num_splits > kMaxSplits) return FD_ERR_INVALID_ARGUMENT;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+      !aligned(out_f32, 16) ||
+      !aligned(lse, 4) || !aligned(workspace, 16) || !aligned(seqlens, 4) ||
+      !aligned(block_table, 4))
+    return FD_ERR_INVALID_ARGUMENT;
+
+  const int B = p->B, Hq = p->Hq, Hkv = p->Hkv, D = p->D, G = Hq / Hkv;
+  const int chunk = chunk_for(p->max_len, num_splits);
+  const int n_splits = effective_splits(p->max_len, chunk);
+  float* part_o = nullptr;
+  float* part_lse = nullptr;
+  if (n_splits > 1) {
+    const size_t need = fd_workspace_bytes(B, Hq, D, n_splits);
+    if (!workspace || workspace_bytes < need) return FD_ERR_WORKSPACE;
+    const size_t rows = static_cast<size_t>(B) * Hq * n_splits;
+    char* w = static_cast<char*>(workspace);
+    part_o = reinterpret_cast<float*>(w);
+    part_lse = reinterpret_cast<float*>(w + round256(rows * D * 4));
+  }
+
+  int dev = 0;
+  if (current_device(&dev) != FD_OK) return FD_ERR_CUDA;
+  const fd_status arch = device_is_sm100(dev);
+  if (arch != FD_OK) return arch;
+
+  // ---- tensor maps over the caches
+  CUtensorMap tk, tv;
+  const int layout = p->kv_layout;
+  const long long rows = paged ? p->block_size : (p->max_len > 0 ? p->max_len : 1);
+  const long long planes = paged ? p->num_blocks : B;
+  const int box_rows = paged ? std::min(p->block_size, fd::kTile) : fd::kTile;
+  if (cached_cache_map(&tk, MapKey{k_cache, rows, planes, D, Hkv, layout, box_rows, dev}) != FD_OK ||
+      cached_cache_map(&tv, MapKey{v_cache, rows, planes, D, Hkv, layout, box_rows, dev}) != FD_OK)
+    return FD_ERR_CUDA;
+
+  fd::SplitArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.seqlens = seqlens;
+  a.block_table = block_table;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.out_f32 = out_f32;
+  a.lse = lse;
+  a.part_o = part_o;
+  a.part_lse = part_lse;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.G = G;
+  a.max_len = p->max_len;
+  a.block_size = paged ? p->block_size : 0;
+  a.log2_block_size = paged ? ilog2(p->block_size) : 0;
+  a.log2_box_rows = ilog2(box_rows);
+  a.max_blocks_per_seq = paged ? p->max_blocks_per_seq : 0;
+  a.chunk = chunk;
+  a.n_splits = n_splits;
+  a.scale_log2 = scale * 1.4426950408889634074f;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  fd_status r;
+  if (D == 128)
+    r = paged ? dispatch_split<128, true>(G, tk, tv, a, n_splits, Hkv, B, s)
+              : dispatch_split<128, false>(G, tk, tv, a, n_splits, Hkv, B, s);
+  else
+    r = paged ? dispatch_split<64, true>(G, tk, tv, a, n_splits, Hkv, B, s)
+              : dispatch_split<64, false>(G, tk, tv, a, n_splits, Hkv, B, s);
+  return r;
+}
+
 }  // namespace
 
 extern "C" {
@@ -421,83 +508,49 @@ fd_status fd_decode(const fd_problem* p, const void* q, const void* k_cache,
                     const void* v_cache, const int32_t* seqlens, const int32_t* block_table,
                     float scale, int num_splits, void* out, float* lse, void* workspace,
                     size_t workspace_bytes, fd_stream_t stream) {
-  // ---- host-side checks: nothing is launched for an invalid call
-  if (!p || !q || !k_cache || !v_cache || !out) return FD_ERR_INVALID_ARGUMENT;
-  const fd_status st = check_shape(p->B, p->Hq, p->Hkv, p->D, p->max_len, p->block_size);
-  if (st != FD_OK) return st;
-  const bool paged = p->block_size != 0;
-  if (paged != (block_table != nullptr)) return FD_ERR_INVALID_ARGUMENT;
-  if (paged) {
-    if (p->num_blocks < 1 || p->max_blocks_per_seq < 1) return FD_ERR_INVALID_ARGUMENT;
-    if (static_cast<long long>(p->max_blocks_per_seq) * p->block_size < p->max_len)
-      return FD_ERR_INVALID_ARGUMENT;
-  }
-  if (p->kv_layout != FD_LAYOUT_HND && p->kv_layout != FD_LAYOUT_NHD) return FD_ERR_INVALID_ARGUMENT;
-  if (!std::isfinite(scale) || !(scale > 0.f)) return FD_ERR_INVALID_ARGUMENT;
-  if (num_splits < 1 || num_splits > kMaxSplits) return FD_ERR_INVALID_ARGUMENT;
-  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
-      !aligned(lse, 4) || !aligned(workspace, 16) || !aligned(seqlens, 4) ||
-      !aligned(block_table, 4))
+  if (!out) return FD_ERR_INVALID_ARGUMENT;
+  return decode_impl(p, q, k_cache, v_cache, seqlens, block_table, scale, num_splits, out,
+                     nullptr, lse, workspace, workspace_bytes, stream);
+}
+
+fd_status fd_decode_partial(const fd_problem* p, const void* q, const void* k_cache,
+                            const void* v_cache, const int32_t* seqlens,
+                            const int32_t* block_table, float scale, int num_splits,
+                            float* out_f32, float* lse, void* workspace, size_t workspace_bytes,
+                            fd_stream_t stream) {
+  if (!out_f32 || !lse) return FD_ERR_INVALID_ARGUMENT;
+  return decode_impl(p, q, k_cache, v_cache, seqlens, block_table, scale, num_splits, nullptr,
+                     out_f32, lse, workspace, workspace_bytes, stream);
+}
+
+fd_status fd_combine(int R, int B, int Hq, int D, const float* part_o, const float* part_lse,
+                     void* out, float* lse, fd_stream_t stream) {
+  if (R < 1 || R > kMaxSplits || B < 1 || Hq < 1 || !part_o || !part_lse || !out)
     return FD_ERR_INVALID_ARGUMENT;
-
-  const int B = p->B, Hq = p->Hq, Hkv = p->Hkv, D = p->D, G = Hq / Hkv;
-  const int chunk = chunk_for(p->max_len, num_splits);
-  const int n_splits = effective_splits(p->max_len, chunk);
-  float* part_o = nullptr;
-  float* part_lse = nullptr;
-  if (n_splits > 1) {
-    const size_t need = fd_workspace_bytes(B, Hq, D, n_splits);
-    if (!workspace || workspace_bytes < need) return FD_ERR_WORKSPACE;
-    const size_t rows = static_cast<size_t>(B) * Hq * n_splits;
-    char* w = static_cast<char*>(workspace);
-    part_o = reinterpret_cast<float*>(w);
-    part_lse = reinterpret_cast<float*>(w + round256(rows * D * 4));
-  }
-
+  if (D != 64 && D != 128) return FD_ERR_UNSUPPORTED;
+  if (!aligned(part_o, 16) || !aligned(part_lse, 4) || !aligned(out, 16) || !aligned(lse, 4))
+    return FD_ERR_INVALID_ARGUMENT;
+  const long long rows = static_cast<long long>(B) * Hq;
+  if (rows > (1ll << 30)) return FD_ERR_INVALID_ARGUMENT;
   int dev = 0;
   if (current_device(&dev) != FD_OK) return FD_ERR_CUDA;
   const fd_status arch = device_is_sm100(dev);
   if (arch != FD_OK) return arch;
-
-  // ---- tensor maps over the caches
-  CUtensorMap tk, tv;
-  const int layout = p->kv_layout;
-  const long long rows = paged ? p->block_size : (p->max_len > 0 ? p->max_len : 1);
-  const long long planes = paged ? p->num_blocks : B;
-  const int box_rows = paged ? std::min(p->block_size, fd::kTile) : fd::kTile;
-  if (cached_cache_map(&tk, MapKey{k_cache, rows, planes, D, Hkv, layout, box_rows, dev}) != FD_OK ||
-      cached_cache_map(&tv, MapKey{v_cache, rows, planes, D, Hkv, layout, box_rows, dev}) != FD_OK)
-    return FD_ERR_CUDA;
-
-  fd::SplitArgs a{};
-  a.q = static_cast<const __nv_bfloat16*>(q);
-  a.seqlens = seqlens;
-  a.block_table = block_table;
-  a.out = static_cast<__nv_bfloat16*>(out);
-  a.lse = lse;
-  a.part_o = part_o;
-  a.part_lse = part_lse;
-  a.Hq = Hq;
-  a.Hkv = Hkv;
-  a.G = G;
-  a.max_len = p->max_len;
-  a.block_size = paged ? p->block_size : 0;
-  a.log2_block_size = paged ? ilog2(p->block_size) : 0;
-  a.log2_box_rows = ilog2(box_rows);
-  a.max_blocks_per_seq = paged ? p->max_blocks_per_seq : 0;
-  a.chunk = chunk;
-  a.n_splits = n_splits;
-  a.scale_log2 = scale * 1.4426950408889634074f;
-
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  fd_status r;
-  if (D == 128)
-    r = paged ? dispatch_split<128, true>(G, tk, tv, a, n_splits, Hkv, B, s)
-              : dispatch_split<128, false>(G, tk, tv, a, n_splits, Hkv, B, s);
-  else
-    r = paged ? dispatch_split<64, true>(G, tk, tv, a, n_splits, Hkv, B, s)
-              : dispatch_split<64, false>(G, tk, tv, a, n_splits, Hkv, B, s);
-  return r;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>((rows + 3) / 4));
+  cfg.blockDim = dim3(128);
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
+  const int r = static_cast<int>(rows);
+  const cudaError_t e = D == 128
+      ? cudaLaunchKernelEx(&cfg, fd::fd_merge_kernel<128>, part_o, part_lse, R, r, o, lse)
+      : cudaLaunchKernelEx(&cfg, fd::fd_merge_kernel<64>, part_o, part_lse, R, r, o, lse);
+  return e == cudaSuccess ? FD_OK : FD_ERR_CUDA;
 }
 
 // Scratch of fd_decode_static_workspace: a file-scope device array, so that

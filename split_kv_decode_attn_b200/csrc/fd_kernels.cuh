@@ -49,7 +49,8 @@ struct SplitArgs {
   const __nv_bfloat16* q;       // [B, Hq, D]
   const int32_t* seqlens;       // [B] or null
   const int32_t* block_table;   // [B, max_blocks_per_seq] or null
-  __nv_bfloat16* out;           // [B, Hq, D]          (one split)
+  __nv_bfloat16* out;           // [B, Hq, D] bf16 result (null when out_f32 is set)
+  float* out_f32;               // [B, Hq, D] fp32 result instead (partial over a shard)
   float* lse;                   // [B, Hq] or null     (one split)
   float* part_o;                // [B, Hq, S, D]       (several splits)
   float* part_lse;              // [B, Hq, S]          (several splits)
@@ -82,13 +83,18 @@ __device__ __forceinline__ void raise_device_error(unsigned int code) {
 }
 
 // Merge the n_parts partials of one (sequence, query head) row; one warp,
-// lanes cover D.  Partials written by other CTAs are read through L2
-// (ld.global.cg).  The first 16 split rows are requested together with the
-// lse values, so a row with up to 16 splits costs one round trip.  Splits
-// are summed in index order, so the result is deterministic.
+// lanes cover D.  Partial s of the row sits at po + s * o_stride (D floats)
+// and pl[s * l_stride].  Partials written by other CTAs are read through L2
+// (ld.global.cg).  The first 16 partials are requested together with the
+// lse values, so a row with up to 16 of them costs one round trip.  They are
+// summed in index order, so the result is deterministic.  A row whose
+// partials are all empty (lse = -inf) gives 0 and -inf.  The result goes to
+// orow (bf16) or, when orow_f32 is set, to orow_f32 (fp32).
 template <int D>
 __device__ __forceinline__ void combine_row(const float* po, const float* pl, int n_parts,
-                                            __nv_bfloat16* orow, float* lse_out, int lane) {
+                                            size_t o_stride, size_t l_stride,
+                                            __nv_bfloat16* orow, float* orow_f32,
+                                            float* lse_out, int lane) {
   constexpr int VPL = D / 32;  // 4 or 2 values per lane
   constexpr int BATCH = 16;
   constexpr float kLog2e = 1.4426950408889634074f;
@@ -98,12 +104,12 @@ __device__ __forceinline__ void combine_row(const float* po, const float* pl, in
 #pragma unroll
     for (int j = 0; j < BATCH; ++j) {
       if (s0 + j < n_parts) {
-        lb[j] = __ldcg(pl + s0 + j);
+        lb[j] = __ldcg(pl + (s0 + j) * l_stride);
         if constexpr (VPL == 4) {
-          const float4 v = __ldcg(reinterpret_cast<const float4*>(col + (s0 + j) * D));
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(col + (s0 + j) * o_stride));
           ob[j][0] = v.x; ob[j][1] = v.y; ob[j][2] = v.z; ob[j][3] = v.w;
         } else {
-          const float2 v = __ldcg(reinterpret_cast<const float2*>(col + (s0 + j) * D));
+          const float2 v = __ldcg(reinterpret_cast<const float2*>(col + (s0 + j) * o_stride));
           ob[j][0] = v.x; ob[j][1] = v.y;
         }
       }
@@ -111,27 +117,32 @@ __device__ __forceinline__ void combine_row(const float* po, const float* pl, in
   };
   load_batch(0);
   float mx = -INFINITY;
-  for (int s = lane; s < n_parts; s += 32) mx = fmaxf(mx, __ldcg(pl + s));
+  for (int s = lane; s < n_parts; s += 32) mx = fmaxf(mx, __ldcg(pl + s * l_stride));
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
   float acc[VPL];
 #pragma unroll
   for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
   float W = 0.f;
-  for (int s0 = 0; s0 < n_parts; s0 += BATCH) {
-    if (s0 > 0) load_batch(s0);
+  if (mx != -INFINITY) {
+    for (int s0 = 0; s0 < n_parts; s0 += BATCH) {
+      if (s0 > 0) load_batch(s0);
 #pragma unroll
-    for (int j = 0; j < BATCH; ++j) {
-      if (s0 + j < n_parts) {
-        const float w = ex2((lb[j] - mx) * kLog2e);
-        W += w;
+      for (int j = 0; j < BATCH; ++j) {
+        if (s0 + j < n_parts) {
+          const float w = ex2((lb[j] - mx) * kLog2e);  // an empty partial weighs 0
+          W += w;
 #pragma unroll
-        for (int i = 0; i < VPL; ++i) acc[i] += w * ob[j][i];
+          for (int i = 0; i < VPL; ++i) acc[i] += w * ob[j][i];
+        }
       }
     }
   }
-  const float inv = 1.f / W;
-  if constexpr (VPL == 4) {
+  const float inv = W > 0.f ? 1.f / W : 0.f;
+  if (orow_f32) {
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) orow_f32[lane * VPL + i] = acc[i] * inv;
+  } else if constexpr (VPL == 4) {
     uint2 pk;
     pk.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
     pk.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
@@ -139,7 +150,7 @@ __device__ __forceinline__ void combine_row(const float* po, const float* pl, in
   } else {
     *reinterpret_cast<uint32_t*>(orow + lane * VPL) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
   }
-  if (lse_out && lane == 0) *lse_out = mx + logf(W);
+  if (lse_out && lane == 0) *lse_out = mx == -INFINITY ? -INFINITY : mx + logf(W);
 }
 
 template <int D, int NB, int STAGES>
@@ -429,7 +440,10 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
     }
     const size_t row = static_cast<size_t>(b) * a.Hq + h0 + g;
     if (direct) {
-      a.out[row * D + d] = __float2bfloat16_rn(O);
+      if (a.out_f32)
+        a.out_f32[row * D + d] = O;
+      else
+        a.out[row * D + d] = __float2bfloat16_rn(O);
       if (d == 0 && a.lse) a.lse[row] = f[L::kSplitLse + g];
     } else {
       a.part_o[(row * a.n_splits + split) * D + d] = O;
@@ -490,8 +504,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     // Empty split.  Split 0 is empty only for an empty sequence, whose
     // result is out = 0, lse = -inf; other empty splits take no part.
     if (split == 0) {
-      for (int i = threadIdx.x; i < a.G * D; i += kThreads)
-        a.out[(static_cast<size_t>(b) * a.Hq + h0) * D + i] = __float2bfloat16_rn(0.f);
+      const size_t base = (static_cast<size_t>(b) * a.Hq + h0) * D;
+      for (int i = threadIdx.x; i < a.G * D; i += kThreads) {
+        if (a.out_f32)
+          a.out_f32[base + i] = 0.f;
+        else
+          a.out[base + i] = __float2bfloat16_rn(0.f);
+      }
       if (a.lse && threadIdx.x < a.G) a.lse[static_cast<size_t>(b) * a.Hq + h0 + threadIdx.x] = -INFINITY;
     }
     return;
@@ -594,8 +613,26 @@ __global__ void __launch_bounds__(128) fd_combine_kernel(const SplitArgs a, int 
   const int n_parts = min((n + a.chunk - 1) / a.chunk, a.n_splits);
   if (n_parts <= 1) return;
   combine_row<D>(a.part_o + static_cast<size_t>(row) * a.n_splits * D,
-                 a.part_lse + static_cast<size_t>(row) * a.n_splits, n_parts,
-                 a.out + static_cast<size_t>(row) * D, a.lse ? a.lse + row : nullptr, lane);
+                 a.part_lse + static_cast<size_t>(row) * a.n_splits, n_parts, D, 1,
+                 a.out_f32 ? nullptr : a.out + static_cast<size_t>(row) * D,
+                 a.out_f32 ? a.out_f32 + static_cast<size_t>(row) * D : nullptr,
+                 a.lse ? a.lse + row : nullptr, lane);
+}
+
+// Merge of R partial results laid out [R][rows][D] (fp32) and [R][rows]
+// (lse): one warp per row, partial r at stride rows * D.
+template <int D>
+__global__ void __launch_bounds__(128) fd_merge_kernel(const float* part_o, const float* part_lse,
+                                                       int R, int rows, __nv_bfloat16* out,
+                                                       float* lse) {
+  grid_dependency_wait();
+  grid_dependents_launch();
+  const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  combine_row<D>(part_o + static_cast<size_t>(row) * D, part_lse + row, R,
+                 static_cast<size_t>(rows) * D, static_cast<size_t>(rows),
+                 out + static_cast<size_t>(row) * D, nullptr, lse ? lse + row : nullptr, lane);
 }
 
 // Diagnostic: waits, with the kernels' bounded wait, on an mbarrier that

@@ -230,3 +230,16 @@ def test_plan_seqlens_edge_cases():
     assert fd.load_library().fd_plan_seqlens(B200_SMS, 2, 8, 8, 128, 4096, 0, None) == \
         fd.FD_ERR_INVALID_ARGUMENT
     assert fd.fd_plan_seqlens(B200_SMS, 2, 8, 8, 96, 4096, 0, [1, 2]) == fd.FD_ERR_UNSUPPORTED
+
+
+def test_partial_and_combine_reject_bad_arguments():
+    lib = fd.load_library()
+    assert lib.fd_decode_partial(ctypes.byref(P()), Q, K, V, None, None, ctypes.c_float(0.125), 1,
+                                 None, 0x70000, None, 0, None) == fd.FD_ERR_INVALID_ARGUMENT
+    assert lib.fd_decode_partial(ctypes.byref(P()), Q, K, V, None, None, ctypes.c_float(0.125), 1,
+                                 O, None, None, 0, None) == fd.FD_ERR_INVALID_ARGUMENT
+    # stream 0: the legacy default stream (no torch stream lookup on a CPU machine)
+    assert fd.fd_combine(0, 1, 8, 128, Q, K, O, None, 0) == fd.FD_ERR_INVALID_ARGUMENT
+    assert fd.fd_combine(2, 1, 8, 96, Q, K, O, None, 0) == fd.FD_ERR_UNSUPPORTED
+    assert fd.fd_combine(2, 1, 8, 128, Q + 4, K, O, None, 0) == fd.FD_ERR_INVALID_ARGUMENT
+    assert fd.fd_combine(2, 1, 8, 128, None, K, O, None, 0) == fd.FD_ERR_INVALID_ARGUMENT

@@ -67,3 +67,76 @@ def test_single_rank_needs_no_process_group():
     import bench
     assert bench.max_over_ranks(torch, 12.5, 1) == 12.5
     assert bench.job_throughput(2e6, 10.0, 10, 1) == pytest.approx(2e6 / 1e-3 / 1e9)
+
+
+def _sharded_worker(rank, world, port, q_out):
+    """One rank of a sequence-parallel decode on CPU: the partial over this
+    rank's slice comes from the fp64 oracle, the merge is the log-sum-exp
+    formula written out in numpy; the gather is the package's own code."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+    from split_kv_decode_attn_b200 import sharded
+    from split_kv_decode_attn_b200 import workloads as wl
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = wl.make_problem(3, 8, 2, 64, 300, seed=77, seqlens=[300, 120, 0])
+        lo, hi = sharded.shard_bounds(w.max_len, world, rank)
+        sl_shard = sharded.shard_lengths(w.seqlens, lo, hi)
+        k_shard = np.ascontiguousarray(w.k[:, :, lo:hi])
+        v_shard = np.ascontiguousarray(w.v[:, :, lo:hi])
+
+        def partial(q, k, v, seqlens):
+            o, lse = oracle.decode(q, k, v, w.scale, seqlens=seqlens, nthreads=1)
+            return torch.from_numpy(o), torch.from_numpy(lse)
+
+        def merge(o_all, lse_all):
+            o_all, lse_all = o_all.numpy(), lse_all.numpy()
+            m = lse_all.max(axis=0)
+            with np.errstate(invalid="ignore"):
+                wgt = np.where(np.isneginf(lse_all), 0.0, np.exp(lse_all - m))
+            tot = wgt.sum(axis=0)
+            out = np.where(tot[..., None] > 0,
+                           (wgt[..., None] * o_all).sum(axis=0) / np.where(tot > 0, tot, 1)[..., None], 0.0)
+            lse = np.where(tot > 0, m + np.log(np.where(tot > 0, tot, 1)), -np.inf)
+            return out, lse
+
+        out, lse = sharded.decode_sequence_sharded(w.q, k_shard, v_shard, np.array(sl_shard, np.int32),
+                                                   partial=partial, merge=merge)
+        ref, ref_lse = oracle.decode(w.q, w.k, w.v, w.scale, seqlens=w.seqlens, nthreads=1)
+        q_out.put((rank, float(np.max(np.abs(out - ref))),
+                   bool(np.all(np.isneginf(lse[2]))),
+                   float(np.max(np.abs(lse[:2] - ref_lse[:2])))))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_sequence_sharded_decode_orchestration(world):
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_sharded_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+        assert p.exitcode == 0
+    res = [q.get(timeout=10) for _ in range(world)]
+    for rank, err, empty_ok, lse_err in res:
+        assert err < 1e-12 and lse_err < 1e-12 and empty_ok, (rank, err, lse_err)
+
+
+def test_shard_bounds_cover_the_history_once():
+    sys.path.insert(0, ROOT)
+    from split_kv_decode_attn_b200 import sharded
+    for total in (0, 1, 7, 300, 4096):
+        for world in (1, 2, 3, 8):
+            ranges = [sharded.shard_bounds(total, world, r) for r in range(world)]
+            covered = [t for lo, hi in ranges for t in range(lo, hi)]
+            assert covered == list(range(total))
+    assert sharded.shard_lengths([300, 120, 0], 100, 200) == [100, 20, 0]
