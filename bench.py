@@ -63,6 +63,8 @@ def parse_args():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="codellama34b")
     ap.add_argument("--L", type=int, default=None, help="cache length of the codellama34b workload")
     ap.add_argument("--splits", type=int, default=None, help="override the planner's split count")
+    ap.add_argument("--kv-dtype", choices=["bf16", "fp8"], default="bf16",
+                    help="cache element type (fp8: e4m3 codes with per-tensor scales)")
     ap.add_argument("--layout", choices=["HND", "NHD"], default="HND",
                     help="cache dimension order (heads outside tokens, or tokens outside heads)")
     ap.add_argument("--shard-sequence", action="store_true",
@@ -187,6 +189,15 @@ def dev_bf16(torch, a, device):
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(torch.bfloat16)
 
 
+def host_cache(torch, a):
+    """Cache array as a host tensor of its storage type (bf16 bits or e4m3 codes)."""
+    import numpy as np
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint8:
+        return torch.from_numpy(a)
+    return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+
+
 class Call:
     """Device buffers and a bound fd_decode call for one workload; `copies`
     rotating cache copies keep L2 from serving K/V."""
@@ -194,14 +205,15 @@ class Call:
     def __init__(self, torch, fd, w, device, num_splits=None, copies=1):
         self.torch, self.fd, self.w = torch, fd, w
         self.q = dev_bf16(torch, w.q, device)
-        k = dev_bf16(torch, w.k, device)
-        v = dev_bf16(torch, w.v, device)
+        k = host_cache(torch, w.k).to(device)
+        v = host_cache(torch, w.v).to(device)
         self.ks = [k] + [k.clone() for _ in range(copies - 1)]
         self.vs = [v] + [v.clone() for _ in range(copies - 1)]
         self.seqlens = None if w.seqlens is None else torch.from_numpy(w.seqlens).to(device)
         self.table = None if w.block_table is None else torch.from_numpy(w.block_table).to(device)
         self.prob = fd.make_problem(w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size, w.num_blocks,
-                                    w.max_blocks_per_seq, w.kv_layout)
+                                    w.max_blocks_per_seq, w.kv_layout, w.kv_dtype_code,
+                                    w.k_scale, w.v_scale)
         if num_splits:
             self.S = num_splits
         elif w.seqlens is not None:  # lengths known on the host: length-aware planner
@@ -304,25 +316,56 @@ def copies_for(torch, nbytes, device):
     return max(2, math.ceil(4 * l2 / max(nbytes, 1))), l2
 
 
-def make_workload(name, L, rank, nthreads=None, layout="HND"):
+def make_workload(name, L, rank, nthreads=None, layout="HND", kv_dtype="bf16"):
     from split_kv_decode_attn_b200 import workloads as wl
     idx, default_L = WORKLOADS[name]
     if idx == 2:
         w = wl.config(2, L=L or default_L, nthreads=nthreads)
     else:
         w = wl.config(idx, nthreads=nthreads)
-    if rank or layout != "HND":
-        # replicas: each rank decodes its own sequences (same shapes)
+    if rank or layout != "HND" or kv_dtype != "bf16":
         # replicas: rank r decodes its own sequences (same shapes); the token-
-        # major layout draws its cache in that storage order
+        # major layout draws its cache in that storage order, fp8 caches
+        # hold e4m3 codes
+        suffix = ("" if layout == "HND" else "-NHD") + ("" if kv_dtype == "bf16" else "-fp8")
         w2 = wl.make_problem(w.B, w.Hq, w.Hkv, w.D, w.max_len, wl.CONFIG_SEED_BASE + 1000 * rank + idx,
                              seqlens=w.seqlens, nan_pad=w.seqlens is not None and not w.paged,
-                             block_size=w.block_size, name=w.name + ("" if layout == "HND" else "-NHD"),
-                             nthreads=nthreads, layout=layout)
-        if "dominant_positions" in w.meta and layout == "HND":
+                             block_size=w.block_size, name=w.name + suffix,
+                             nthreads=nthreads, layout=layout, kv_dtype=kv_dtype)
+        if "dominant_positions" in w.meta and layout == "HND" and kv_dtype == "bf16":
             wl.plant_dominant_keys(w2, 64, wl.CONFIG_SEED_BASE + 1000 * rank + idx)
         w = w2
     return w
+
+
+def oracle_sequence(w, b, off, n, threads):
+    """The oracle on tokens [off, off + n) of sequence b, every query head.
+    Returns the algorithmic K+V bytes of that window."""
+    import numpy as np
+    import oracle
+    if w.kv_dtype == "fp8":  # dequantised cache: one fp64 oracle call per KV head
+        from concurrent.futures import ThreadPoolExecutor
+        from split_kv_decode_attn_b200 import workloads as wl
+        G = w.G
+
+        def head(h):
+            k, v = w.logical_kv(b, h)
+            k = float(np.float32(w.k_scale)) * wl.e4m3_bits_to_f64(k[off:off + n])
+            v = float(np.float32(w.v_scale)) * wl.e4m3_bits_to_f64(v[off:off + n])
+            oracle.attend_f64(wl.bf16_bits_to_f64(w.q[b, h * G:(h + 1) * G]), k, v,
+                              float(np.float32(w.scale)))
+        with ThreadPoolExecutor(max_workers=min(threads, w.Hkv)) as ex:
+            list(ex.map(head, range(w.Hkv)))
+        return n * w.Hkv * w.D * 2
+    if w.paged or w.layout != "HND":
+        kv = [w.logical_kv(b, h) for h in range(w.Hkv)]
+        k = np.stack([x[0][off:off + n] for x in kv])[None]
+        v = np.stack([x[1][off:off + n] for x in kv])[None]
+    else:
+        k, v = w.k[b:b + 1, :, off:off + n], w.v[b:b + 1, :, off:off + n]
+    oracle.decode(w.q[b:b + 1], np.ascontiguousarray(k), np.ascontiguousarray(v), w.scale,
+                  nthreads=threads)
+    return n * w.Hkv * w.D * 4
 
 
 def cpu_baseline(w, seconds):
@@ -330,26 +373,15 @@ def cpu_baseline(w, seconds):
     oracle call (all its query heads, threads over heads), cycling through
     the batch until `seconds` of wall time have passed.  GB/s of algorithmic
     K+V bytes."""
-    import numpy as np
-    import oracle
     cores = os.cpu_count() or 1
-    threads = min(cores, w.Hq)
+    threads = min(cores, w.Hq if w.kv_dtype == "bf16" else w.Hkv)
     lengths = w.lengths()
     t0 = time.perf_counter()
     done = 0
     calls = 0
     while True:
         b = calls % w.B
-        n = int(lengths[b])
-        if w.paged or w.layout != "HND":
-            kv = [w.logical_kv(b, h) for h in range(w.Hkv)]
-            k = np.stack([x[0] for x in kv])[None]
-            v = np.stack([x[1] for x in kv])[None]
-        else:
-            k, v = w.k[b:b + 1, :, :n], w.v[b:b + 1, :, :n]
-        oracle.decode(w.q[b:b + 1], np.ascontiguousarray(k), np.ascontiguousarray(v), w.scale,
-                      nthreads=threads)
-        done += n * w.Hkv * w.D * 4
+        done += oracle_sequence(w, b, 0, int(lengths[b]), threads)
         calls += 1
         if time.perf_counter() - t0 >= seconds:
             break
@@ -376,7 +408,7 @@ def run_fd(args):
     device = torch.device("cuda", torch.cuda.current_device())
     fd.load_library()
 
-    w = make_workload(args.workload, args.L, rank, layout=args.layout)
+    w = make_workload(args.workload, args.L, rank, layout=args.layout, kv_dtype=args.kv_dtype)
     kvb = w.kv_bytes()
     copies, l2 = copies_for(torch, (w.k.nbytes + w.v.nbytes), device)
     call = Call(torch, fd, w, device, args.splits, copies)
@@ -397,7 +429,8 @@ def run_fd(args):
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
         "us_per_call": round(per_call_s * 1e6, 3), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": "bf16" if w.kv_dtype == "bf16" else "e4m3 cache, f16 mma",
+        "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
                    "max_len": w.max_len, "block_size": w.block_size, "num_splits": call.S,
                    "effective_splits": call.s_eff, "kv_bytes_per_call": kvb,
@@ -435,8 +468,8 @@ def e2e(torch, fd, call, w, device, steps, warmup, barrier, world):
     D2H of out and lse, all inside the timed region on one stream."""
     import numpy as np
     hq = torch.from_numpy(np.ascontiguousarray(w.q).view(np.int16)).view(torch.bfloat16).pin_memory()
-    hk = torch.from_numpy(np.ascontiguousarray(w.k).view(np.int16)).view(torch.bfloat16).pin_memory()
-    hv = torch.from_numpy(np.ascontiguousarray(w.v).view(np.int16)).view(torch.bfloat16).pin_memory()
+    hk = host_cache(torch, w.k).pin_memory()
+    hv = host_cache(torch, w.v).pin_memory()
     dq, dk, dv = torch.empty_like(hq, device=device), torch.empty_like(hk, device=device), \
         torch.empty_like(hv, device=device)
     ho = torch.empty(call.out.shape, dtype=torch.bfloat16).pin_memory()
@@ -452,7 +485,7 @@ def e2e(torch, fd, call, w, device, steps, warmup, barrier, world):
 
     ms = max_over_ranks(torch, timed(torch, step, steps, warmup, barrier), world, device)
     per = ms / 1e3 / steps
-    h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2
+    h2d = hq.numel() * 2 + hk.numel() * hk.element_size() + hv.numel() * hv.element_size()
     d2h = ho.numel() * 2 + hl.numel() * 4
     return {"value": round(job_throughput(w.kv_bytes(), ms, steps, world), 2), "unit": "GB/s",
             "us_per_call": round(per * 1e6, 1), "h2d_bytes_per_step": h2d,
@@ -625,11 +658,9 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    import numpy as np
-    import oracle
-    w = make_workload(args.workload, args.L, 0, layout=args.layout)
+    w = make_workload(args.workload, args.L, 0, layout=args.layout, kv_dtype=args.kv_dtype)
     cores = os.cpu_count() or 1
-    threads = min(cores, w.Hq)
+    threads = min(cores, w.Hq if w.kv_dtype == "bf16" else w.Hkv)
     lengths = w.lengths()
     seqs = [b for b in range(w.B) if lengths[b] > 0]
     budget_per_step = 120.0 / max(args.steps + args.warmup, 1)
@@ -638,15 +669,7 @@ def run_reference(args):
         b = seqs[i % len(seqs)]
         n = min(n_tok, int(lengths[b]))
         off = (i * 7919) % max(int(lengths[b]) - n + 1, 1)
-        if w.paged or w.layout != "HND":
-            kv = [w.logical_kv(b, h) for h in range(w.Hkv)]
-            k = np.stack([x[0][off:off + n] for x in kv])[None]
-            v = np.stack([x[1][off:off + n] for x in kv])[None]
-        else:
-            k, v = w.k[b:b + 1, :, off:off + n], w.v[b:b + 1, :, off:off + n]
-        oracle.decode(w.q[b:b + 1], np.ascontiguousarray(k), np.ascontiguousarray(v), w.scale,
-                      nthreads=threads)
-        return n * w.Hkv * w.D * 4
+        return oracle_sequence(w, b, off, n, threads)
 
     n_tok = 1024
     t0 = time.perf_counter()

@@ -74,6 +74,12 @@ typedef enum fd_kv_layout {
   FD_LAYOUT_NHD = 1
 } fd_kv_layout;
 
+/* Element type of the K/V cache. */
+typedef enum fd_kv_dtype {
+  FD_KV_BF16 = 0,     /* bf16 */
+  FD_KV_FP8_E4M3 = 1  /* OCP fp8 e4m3 (bias 7, max 448, no inf); value = scale * code */
+} fd_kv_dtype;
+
 /* Shape of one decode-attention call.
  *   B           sequences in the batch (1 .. 65535)
  *   Hq, Hkv     query heads and KV heads (Hkv .. 65535, Hq % Hkv == 0)
@@ -84,7 +90,13 @@ typedef enum fd_kv_layout {
  *   block_size  0 for a contiguous cache; otherwise tokens per page
  *   num_blocks  paged cache: pages in the pool (ignored when contiguous)
  *   max_blocks_per_seq  paged cache: row length of block_table
- *   kv_layout   an fd_kv_layout value (FD_LAYOUT_HND when zero-initialised) */
+ *   kv_layout   an fd_kv_layout value (FD_LAYOUT_HND when zero-initialised)
+ *   kv_dtype    an fd_kv_dtype value (FD_KV_BF16 when zero-initialised)
+ *   k_scale, v_scale
+ *               fp8 caches: the real K and V are k_scale * code and
+ *               v_scale * code (finite, > 0). Ignored for bf16 caches.
+ *               An fp8 cache needs D = 128, and the contraction runs on f16
+ *               tensor cores: q must be finite in f16 (|q| < 65504). */
 typedef struct fd_problem {
   int32_t B;
   int32_t Hq;
@@ -95,6 +107,9 @@ typedef struct fd_problem {
   int32_t num_blocks;
   int32_t max_blocks_per_seq;
   int32_t kv_layout;
+  int32_t kv_dtype;
+  float k_scale;
+  float v_scale;
 } fd_problem;
 
 /* Split-count planner.
@@ -146,6 +161,7 @@ FD_API size_t fd_workspace_bytes(int B, int Hq, int D, int num_splits);
  *   p            shape (see fd_problem)
  *   q            [B, Hq, D] bf16, 16-byte aligned
  *   k_cache, v_cache
+ *                (elements bf16, or fp8 e4m3 bytes when kv_dtype says so)
  *                FD_LAYOUT_HND contiguous: [B, Hkv, max_len, D] bf16;
  *                FD_LAYOUT_HND paged:      [num_blocks, Hkv, block_size, D];
  *                FD_LAYOUT_NHD contiguous: [B, max_len, Hkv, D];

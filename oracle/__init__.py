@@ -47,6 +47,8 @@ def _load():
         lib.oracle_attend_split.restype = None
         lib.oracle_decode.argtypes = [I, I, I, I, L, vp, vp, vp, vp, F, vp, vp, I]
         lib.oracle_decode.restype = I
+        lib.oracle_attend_f64.argtypes = [L, I, I, vp, vp, vp, L, ctypes.c_double, vp, vp]
+        lib.oracle_attend_f64.restype = None
         _lib = lib
     return _lib
 
@@ -69,6 +71,20 @@ def attend(q, k, v, scale: float):
     lse = np.empty(G, np.float64)
     _load().oracle_attend(n, D, G, q.ctypes.data, k.ctypes.data, v.ctypes.data, D,
                           np.float32(scale), out.ctypes.data, lse.ctypes.data)
+    return out, lse
+
+
+def attend_f64(q, k, v, scale: float):
+    """attend() on fp64 values (for caches whose real values are not bf16,
+    such as dequantised fp8).  q [G, D], k/v [n, D] float64."""
+    q, k, v = (np.ascontiguousarray(x, dtype=np.float64) for x in (q, k, v))
+    G, D = q.shape
+    n = k.shape[0]
+    assert k.shape == (n, D) and v.shape == (n, D)
+    out = np.empty((G, D), np.float64)
+    lse = np.empty(G, np.float64)
+    _load().oracle_attend_f64(n, D, G, q.ctypes.data, k.ctypes.data, v.ctypes.data, D,
+                              float(scale), out.ctypes.data, lse.ctypes.data)
     return out, lse
 
 

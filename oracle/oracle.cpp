@@ -28,7 +28,8 @@
 //     M = max_s lse_s,  w_s = exp(lse_s - M)
 //     O = sum_s w_s O_s / sum_s w_s,   lse = M + ln sum_s w_s
 //
-// Inputs are bf16 bit patterns (uint16), widened exactly to double.
+// Inputs are bf16 bit patterns (uint16), widened exactly to double, or fp64
+// values (dequantised caches whose real values need not be bf16).
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -46,11 +47,14 @@ double bf16_to_double(uint16_t bits) {
   return static_cast<double>(f);
 }
 
+double load(const uint16_t* p, long i) { return bf16_to_double(p[i]); }
+double load(const double* p, long i) { return p[i]; }
+
 // One query head against n cached rows.  k and v are row-major [n, D] with
 // row stride `ld` elements.
-void attend_one_head(long n, int D, const uint16_t* q, const uint16_t* k,
-                     const uint16_t* v, long ld, double sc, double* out,
-                     double* lse) {
+template <class T>
+void attend_one_head(long n, int D, const T* q, const T* k, const T* v, long ld, double sc,
+                     double* out, double* lse) {
   const double ninf = -std::numeric_limits<double>::infinity();
   if (n <= 0) {
     for (int d = 0; d < D; ++d) out[d] = 0.0;
@@ -60,7 +64,7 @@ void attend_one_head(long n, int D, const uint16_t* q, const uint16_t* k,
   std::vector<double> s(static_cast<size_t>(n));
   for (long j = 0; j < n; ++j) {
     double dot = 0.0;
-    for (int d = 0; d < D; ++d) dot += bf16_to_double(q[d]) * bf16_to_double(k[j * ld + d]);
+    for (int d = 0; d < D; ++d) dot += load(q, d) * load(k, j * ld + d);
     s[j] = sc * dot;
   }
   double m = ninf;
@@ -70,7 +74,7 @@ void attend_one_head(long n, int D, const uint16_t* q, const uint16_t* k,
   for (int d = 0; d < D; ++d) out[d] = 0.0;
   for (long j = 0; j < n; ++j) {
     double p = std::exp(s[j] - m);
-    for (int d = 0; d < D; ++d) out[d] += p * bf16_to_double(v[j * ld + d]);
+    for (int d = 0; d < D; ++d) out[d] += p * load(v, j * ld + d);
   }
   for (int d = 0; d < D; ++d) out[d] /= Z;
   *lse = m + std::log(Z);
@@ -132,6 +136,14 @@ void parallel_for(long count, int nthreads, F f) {
 }  // namespace
 
 extern "C" {
+
+// The same with fp64 inputs and an fp64 scale.
+void oracle_attend_f64(long n, int D, int G, const double* q, const double* k,
+                       const double* v, long ld, double scale, double* out, double* lse) {
+  for (int g = 0; g < G; ++g)
+    attend_one_head(n, D, q + static_cast<long>(g) * D, k, v, ld, scale,
+                    out + static_cast<long>(g) * D, lse + g);
+}
 
 // G query heads that share one KV head: q [G, D]; k, v [n, ld] row-major.
 void oracle_attend(long n, int D, int G, const uint16_t* q, const uint16_t* k,

@@ -44,13 +44,17 @@ class FdError(RuntimeError):
 
 FD_LAYOUT_HND = 0  # cache [.., Hkv, tokens, D]
 FD_LAYOUT_NHD = 1  # cache [.., tokens, Hkv, D]
+FD_KV_BF16 = 0       # bf16 cache
+FD_KV_FP8_E4M3 = 1   # fp8 e4m3 cache, real value = scale * code
 
 
 class fd_problem(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
                 ("D", ctypes.c_int32), ("max_len", ctypes.c_int32),
                 ("block_size", ctypes.c_int32), ("num_blocks", ctypes.c_int32),
-                ("max_blocks_per_seq", ctypes.c_int32), ("kv_layout", ctypes.c_int32)]
+                ("max_blocks_per_seq", ctypes.c_int32), ("kv_layout", ctypes.c_int32),
+                ("kv_dtype", ctypes.c_int32), ("k_scale", ctypes.c_float),
+                ("v_scale", ctypes.c_float)]
 
 
 _lib = None
@@ -195,9 +199,9 @@ def fd_selftest_device_timeout(limit_us: int, stream=None) -> int:
 # ---- convenience wrapper -----------------------------------------------------
 
 def make_problem(B, Hq, Hkv, D, max_len, block_size=0, num_blocks=0, max_blocks_per_seq=0,
-                 kv_layout=FD_LAYOUT_HND):
+                 kv_layout=FD_LAYOUT_HND, kv_dtype=FD_KV_BF16, k_scale=1.0, v_scale=1.0):
     return fd_problem(B, Hq, Hkv, D, max_len, block_size, num_blocks, max_blocks_per_seq,
-                      kv_layout)
+                      kv_layout, kv_dtype, k_scale, v_scale)
 
 
 def decode(q, k_cache, v_cache, seqlens=None, block_table=None, *, max_len: Optional[int] = None,

@@ -203,22 +203,29 @@ fd_status encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
 // A plane is a sequence (contiguous) or a page (paged).  Coordinates outside
 // the view read zeros.
 fd_status make_cache_map(CUtensorMap* tm, const void* base, int D, int Hkv, long long rows,
-                         long long planes, int layout, int box_rows) {
+                         long long planes, int layout, int box_rows, bool fp8) {
   PFN_cuTensorMapEncodeTiled_v12000 enc;
   if (encoder(&enc) != FD_OK) return FD_ERR_CUDA;
-  const cuuint64_t row_bytes = static_cast<cuuint64_t>(D) * 2;
+  // An fp8 row of 128 entries is one 128-byte swizzle row; a bf16 row of D
+  // entries is D/64 of them.
+  const int elem = fp8 ? 1 : 2;
+  const int inner = 128 / elem;
+  const cuuint64_t row_bytes = static_cast<cuuint64_t>(D) * elem;
   const cuuint64_t head_stride =
       layout == FD_LAYOUT_HND ? static_cast<cuuint64_t>(rows) * row_bytes : row_bytes;
   const cuuint64_t row_stride =
       layout == FD_LAYOUT_HND ? row_bytes : static_cast<cuuint64_t>(Hkv) * row_bytes;
   const cuuint64_t plane_stride = static_cast<cuuint64_t>(Hkv) * rows * row_bytes;
-  const int halves = D / 64;
-  cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(Hkv), static_cast<cuuint64_t>(rows),
-                        static_cast<cuuint64_t>(halves), static_cast<cuuint64_t>(planes)};
+  const int halves = static_cast<int>(row_bytes / 128);
+  cuuint64_t dims[5] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(Hkv),
+                        static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(halves),
+                        static_cast<cuuint64_t>(planes)};
   cuuint64_t strides[4] = {head_stride, row_stride, 128, plane_stride};
-  cuuint32_t box[5] = {64, 1, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(halves), 1};
+  cuuint32_t box[5] = {static_cast<cuuint32_t>(inner), 1, static_cast<cuuint32_t>(box_rows),
+                       static_cast<cuuint32_t>(halves), 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims,
+  CUresult r = enc(tm, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
+                   const_cast<void*>(base), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -232,9 +239,10 @@ struct MapKey {
   const void* base;
   long long rows, planes;
   int D, Hkv, layout, box_rows, dev;
+  bool fp8;
   bool operator==(const MapKey& o) const {
     return base == o.base && rows == o.rows && planes == o.planes && D == o.D && Hkv == o.Hkv &&
-           layout == o.layout && box_rows == o.box_rows && dev == o.dev;
+           layout == o.layout && box_rows == o.box_rows && dev == o.dev && fp8 == o.fp8;
   }
 };
 
@@ -254,7 +262,7 @@ fd_status cached_cache_map(CUtensorMap* tm, const MapKey& key) {
     }
   }
   const fd_status st = make_cache_map(tm, key.base, key.D, key.Hkv, key.rows, key.planes,
-                                      key.layout, key.box_rows);
+                                      key.layout, key.box_rows, key.fp8);
   if (st != FD_OK) return st;
   entries[next] = Entry{key, *tm, true};
   next = (next + 1) % kEntries;
@@ -263,12 +271,13 @@ fd_status cached_cache_map(CUtensorMap* tm, const MapKey& key) {
 
 // --------------------------------------------------------------- launches
 
-template <int D, int NB, int MODE, bool PAGED>
+template <int D, int NB, int MODE, bool PAGED, bool FP8 = false>
 fd_status launch_split(const CUtensorMap& tk, const CUtensorMap& tv, const fd::SplitArgs& a,
                        int n_splits, int Hkv, int B, cudaStream_t stream) {
-  constexpr int STAGES = D == 128 ? 3 : 6;
-  using L = fd::SplitSmem<D, NB, STAGES>;
-  auto kern = fd::fd_split_kernel<D, NB, MODE, PAGED, STAGES>;
+  // About 96 KB of stages: two CTAs per SM.
+  constexpr int STAGES = (D == 128 && !FP8) ? 3 : 6;
+  using L = fd::SplitSmem<D, NB, STAGES, FP8>;
+  auto kern = fd::fd_split_kernel<D, NB, MODE, PAGED, STAGES, FP8>;
   // The shared-memory opt-in is per device; remember which devices have it.
   static std::atomic<unsigned long long> attr_done{0};
   int dev = 0;
@@ -312,12 +321,21 @@ fd_status launch_combine(const fd::SplitArgs& a, int B, cudaStream_t stream) {
 }
 
 // Launches the split kernel and, with several splits, the combine kernel.
-template <int D, int NB, int MODE, bool PAGED>
+template <int D, int NB, int MODE, bool PAGED, bool FP8 = false>
 fd_status launch_call(const CUtensorMap& tk, const CUtensorMap& tv, const fd::SplitArgs& a,
                       int n_splits, int Hkv, int B, cudaStream_t s) {
-  fd_status r = launch_split<D, NB, MODE, PAGED>(tk, tv, a, n_splits, Hkv, B, s);
+  fd_status r = launch_split<D, NB, MODE, PAGED, FP8>(tk, tv, a, n_splits, Hkv, B, s);
   if (r == FD_OK && n_splits > 1) r = launch_combine<D>(a, B, s);
   return r;
+}
+
+// fp8 caches (D = 128): f16 contraction, bf16(p) residuals not needed.
+template <bool PAGED>
+fd_status dispatch_split_fp8(int G, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const fd::SplitArgs& a, int n_splits, int Hkv, int B,
+                             cudaStream_t s) {
+  if (G <= 8) return launch_call<128, 1, fd::kHi, PAGED, true>(tk, tv, a, n_splits, Hkv, B, s);
+  return launch_call<128, 2, fd::kHi, PAGED, true>(tk, tv, a, n_splits, Hkv, B, s);
 }
 
 template <int D, bool PAGED>
@@ -374,6 +392,14 @@ fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
       return FD_ERR_INVALID_ARGUMENT;
   }
   if (p->kv_layout != FD_LAYOUT_HND && p->kv_layout != FD_LAYOUT_NHD) return FD_ERR_INVALID_ARGUMENT;
+  if (p->kv_dtype != FD_KV_BF16 && p->kv_dtype != FD_KV_FP8_E4M3) return FD_ERR_INVALID_ARGUMENT;
+  const bool fp8 = p->kv_dtype == FD_KV_FP8_E4M3;
+  if (fp8) {
+    if (p->D != 128) return FD_ERR_UNSUPPORTED;
+    if (!std::isfinite(p->k_scale) || !(p->k_scale > 0.f) || !std::isfinite(p->v_scale) ||
+        !(p->v_scale > 0.f))
+      return FD_ERR_INVALID_ARGUMENT;
+  }
   if (!std::isfinite(scale) || !(scale > 0.f)) return FD_ERR_INVALID_ARGUMENT;
   if (num_splits < 1 || num_splits > kMaxSplits) return FD_ERR_INVALID_ARGUMENT;
   if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
@@ -407,8 +433,8 @@ fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
   const long long rows = paged ? p->block_size : (p->max_len > 0 ? p->max_len : 1);
   const long long planes = paged ? p->num_blocks : B;
   const int box_rows = paged ? std::min(p->block_size, fd::kTile) : fd::kTile;
-  if (cached_cache_map(&tk, MapKey{k_cache, rows, planes, D, Hkv, layout, box_rows, dev}) != FD_OK ||
-      cached_cache_map(&tv, MapKey{v_cache, rows, planes, D, Hkv, layout, box_rows, dev}) != FD_OK)
+  if (cached_cache_map(&tk, MapKey{k_cache, rows, planes, D, Hkv, layout, box_rows, dev, fp8}) != FD_OK ||
+      cached_cache_map(&tv, MapKey{v_cache, rows, planes, D, Hkv, layout, box_rows, dev, fp8}) != FD_OK)
     return FD_ERR_CUDA;
 
   fd::SplitArgs a{};
@@ -430,11 +456,15 @@ fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
   a.max_blocks_per_seq = paged ? p->max_blocks_per_seq : 0;
   a.chunk = chunk;
   a.n_splits = n_splits;
-  a.scale_log2 = scale * 1.4426950408889634074f;
+  a.scale_log2 = scale * (fp8 ? p->k_scale : 1.f) * 1.4426950408889634074f;
+  a.v_scale = fp8 ? p->v_scale : 1.f;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   fd_status r;
-  if (D == 128)
+  if (fp8)
+    r = paged ? dispatch_split_fp8<true>(G, tk, tv, a, n_splits, Hkv, B, s)
+              : dispatch_split_fp8<false>(G, tk, tv, a, n_splits, Hkv, B, s);
+  else if (D == 128)
     r = paged ? dispatch_split<128, true>(G, tk, tv, a, n_splits, Hkv, B, s)
               : dispatch_split<128, false>(G, tk, tv, a, n_splits, Hkv, B, s);
   else

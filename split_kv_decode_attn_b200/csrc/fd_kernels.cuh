@@ -21,6 +21,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cstdint>
 
 #include "fd_ptx.cuh"
@@ -61,11 +62,17 @@ struct SplitArgs {
   int max_blocks_per_seq;
   int chunk;                    // tokens per split, a multiple of kTile
   int n_splits;                 // effective split count = gridDim.x
-  float scale_log2;             // scale * log2(e)
+  float scale_log2;             // scale * k_scale * log2(e)
+  float v_scale;                // dequantisation scale of an fp8 V cache (1 for bf16)
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
@@ -153,9 +160,11 @@ __device__ __forceinline__ void combine_row(const float* po, const float* pl, in
   if (lse_out && lane == 0) *lse_out = mx == -INFINITY ? -INFINITY : mx + logf(W);
 }
 
-template <int D, int NB, int STAGES>
+template <int D, int NB, int STAGES, bool FP8 = false>
 struct SplitSmem {
-  static constexpr int kHalves = D / 64;               // 128-byte swizzle rows
+  // Rows are stored in 128-byte swizzle rows: a bf16 row of D = 128 takes two
+  // (its column halves), an fp8 row of 128 takes one.
+  static constexpr int kHalves = FP8 ? 1 : D / 64;
   static constexpr int kHalfBytes = kTile * 128;       // one 64-column half tile
   static constexpr int kTileBytes = kHalves * kHalfBytes;
   static constexpr int kStageBytes = 2 * kTileBytes;   // K tile + V tile
@@ -177,20 +186,40 @@ struct SplitSmem {
 // split's tiles, then the merge of the four warps' softmax states into this
 // split's result, which goes to `out` (the sequence has one split) or to the
 // global partials (several splits).
-template <int D, int NB, int MODE, int STAGES>
+template <int D, int NB, int MODE, int STAGES, bool FP8>
 __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* smem,
                                                 uint32_t smem_base, uint32_t bar_full,
                                                 uint32_t bar_empty, volatile int* cta_error,
                                                 int warp, int lane, int b, int h0, int split,
                                                 int start, int end, int n_tiles, int n_parts) {
-  using L = SplitSmem<D, NB, STAGES>;
+  using L = SplitSmem<D, NB, STAGES, FP8>;
   constexpr int KSTEPS = D / 16;   // k-steps of the score MMA (over D)
   constexpr int DBLK = D / 16;     // m-blocks of the P.V MMA (over D)
   constexpr int NCOL = NB * 8;     // MMA columns (query heads, maybe doubled)
+  static_assert(!FP8 || (D == 128 && MODE == kHi), "fp8 caches: D = 128, bf16-only P modes off");
 
   // B fragments of Q^T (k = head dim, n = query head), loaded once.
   uint32_t qf[NB][KSTEPS][2];
-  {
+  if constexpr (FP8) {
+    // f16 fragments, k order permuted to match the fp8 K fragments: k-step
+    // c covers head-dim entries 16c..16c+15; slots 2t, 2t+1 hold 16c+4t,
+    // 16c+4t+1 and slots 2t+8, 2t+9 hold 16c+4t+2, 16c+4t+3 (t = lane & 3).
+    const int ncol = lane >> 2;
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      const int head = nb * 8 + ncol;
+      const bool live = head < a.G;
+      const __nv_bfloat16* qrow = a.q + (static_cast<size_t>(b) * a.Hq + h0 + (live ? head : 0)) * D;
+#pragma unroll
+      for (int ks = 0; ks < KSTEPS; ++ks) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(qrow + ks * 16 + 4 * (lane & 3));
+        const __nv_bfloat162 q01 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+        const __nv_bfloat162 q23 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+        qf[nb][ks][0] = live ? pack_f16x2(__low2float(q01), __high2float(q01)) : 0u;
+        qf[nb][ks][1] = live ? pack_f16x2(__low2float(q23), __high2float(q23)) : 0u;
+      }
+    }
+  } else {
     const int ncol = lane >> 2;
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
@@ -226,7 +255,7 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
   const uint32_t x7 = lane & 7;
   const uint32_t lgr = a.log2_box_rows;
   const uint32_t half_bytes = 128u << lgr;                    // one column half of a box
-  const uint32_t box_bytes = half_bytes * (D / 64);
+  const uint32_t box_bytes = half_bytes * L::kHalves;
   const uint32_t offK = (rowK >> lgr) * box_bytes + (rowK & ((1u << lgr) - 1)) * 128;
   const uint32_t offV = (rowV >> lgr) * box_bytes + (rowV & ((1u << lgr) - 1)) * 128;
   const int r_lo = warp * 16 + (lane >> 2);   // token rows of the C fragment
@@ -254,14 +283,39 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
       for (int c = 0; c < 2; ++c)
 #pragma unroll
         for (int i = 0; i < 4; ++i) sc[nb][c][i] = 0.f;
+    if constexpr (FP8) {
+      // One ldmatrix brings 16 bytes (16 head-dim entries) of 8 token rows
+      // per matrix: tokens 0-7 and 8-15 of chunks 2kp and 2kp+1.  A lane's
+      // register holds 4 consecutive entries of one token, converted to two
+      // f16 pairs in the permuted k order of the q fragments.
 #pragma unroll
-    for (int ks = 0; ks < KSTEPS; ++ks) {
-      const uint32_t chunk16 = ((ks & 3) << 1) + (lane >> 4);
-      const uint32_t addr = kbase + offK + (ks >> 2) * half_bytes + ((chunk16 ^ x7) << 4);
-      uint32_t af[4];
-      ldmatrix_x4(addr, af[0], af[1], af[2], af[3]);
+      for (int kp = 0; kp < KSTEPS / 2; ++kp) {
+        const uint32_t chunk16 = 2 * kp + (lane >> 4);
+        const uint32_t addr = kbase + offK + ((chunk16 ^ x7) << 4);
+        uint32_t r[4];
+        ldmatrix_x4(addr, r[0], r[1], r[2], r[3]);
 #pragma unroll
-      for (int nb = 0; nb < NB; ++nb) mma_bf16_16816(sc[nb][ks & 1], af, qf[nb][ks][0], qf[nb][ks][1]);
+        for (int h = 0; h < 2; ++h) {
+          const int ks = 2 * kp + h;
+          uint32_t af[4];
+          af[0] = e4m3x2_to_f16x2(r[2 * h]);
+          af[1] = e4m3x2_to_f16x2(r[2 * h + 1]);
+          af[2] = e4m3x2_to_f16x2(r[2 * h] >> 16);
+          af[3] = e4m3x2_to_f16x2(r[2 * h + 1] >> 16);
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) mma_f16_16816(sc[nb][ks & 1], af, qf[nb][ks][0], qf[nb][ks][1]);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int ks = 0; ks < KSTEPS; ++ks) {
+        const uint32_t chunk16 = ((ks & 3) << 1) + (lane >> 4);
+        const uint32_t addr = kbase + offK + (ks >> 2) * half_bytes + ((chunk16 ^ x7) << 4);
+        uint32_t af[4];
+        ldmatrix_x4(addr, af[0], af[1], af[2], af[3]);
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) mma_bf16_16816(sc[nb][ks & 1], af, qf[nb][ks][0], qf[nb][ks][1]);
+      }
     }
 
     // Online softmax in the log2 domain; this lane holds tokens r_lo, r_hi
@@ -311,6 +365,9 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
         const float e3 = lo_lane ? p3 - round_to_bf16(p3) : p3;
         pb[nb][0] = movmatrix_trans(pack_bf16x2(e0, e1));
         pb[nb][1] = movmatrix_trans(pack_bf16x2(e2, e3));
+      } else if constexpr (FP8) {
+        pb[nb][0] = movmatrix_trans(pack_f16x2(p0, p1));
+        pb[nb][1] = movmatrix_trans(pack_f16x2(p2, p3));
       } else {
         pb[nb][0] = movmatrix_trans(pack_bf16x2(p0, p1));
         pb[nb][1] = movmatrix_trans(pack_bf16x2(p2, p3));
@@ -330,6 +387,35 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
       vmask_lo = (tk < tile_valid ? 0x0000ffffu : 0u) | (tk + 1 < tile_valid ? 0xffff0000u : 0u);
       vmask_hi = (tk + 8 < tile_valid ? 0x0000ffffu : 0u) | (tk + 9 < tile_valid ? 0xffff0000u : 0u);
     }
+    if constexpr (FP8) {
+      // ldmatrix.trans on the fp8 V tile, 16-bit units: a lane's register
+      // holds entries (16c + 2p, 16c + 2p + 1) of tokens 2t and 2t + 1
+      // (p = lane / 4, t = lane & 3).  Byte-permute to (token 2t, token 2t+1)
+      // pairs of one entry and convert: rows g (g < 8) of the A fragment hold
+      // entry 16c + 2g, rows g + 8 hold 16c + 2g + 1.
+#pragma unroll
+      for (int dp = 0; dp < DBLK / 2; ++dp) {
+        const uint32_t chunk16 = 2 * dp + (lane >> 4);
+        const uint32_t addr = vbase + offK + ((chunk16 ^ x7) << 4);
+        uint32_t r[4];
+        ldmatrix_x4_trans(addr, r[0], r[1], r[2], r[3]);
+        r[0] &= vmask_lo;
+        r[1] &= vmask_hi;
+        r[2] &= vmask_lo;
+        r[3] &= vmask_hi;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int db = 2 * dp + h;
+          uint32_t vf[4];
+          vf[0] = e4m3x2_to_f16x2(__byte_perm(r[2 * h], 0, 0x0020));
+          vf[1] = e4m3x2_to_f16x2(__byte_perm(r[2 * h], 0, 0x0031));
+          vf[2] = e4m3x2_to_f16x2(__byte_perm(r[2 * h + 1], 0, 0x0020));
+          vf[3] = e4m3x2_to_f16x2(__byte_perm(r[2 * h + 1], 0, 0x0031));
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) mma_f16_16816(acc[nb][db], vf, pb[nb][0], pb[nb][1]);
+        }
+      }
+    } else {
 #pragma unroll
     for (int db = 0; db < DBLK; ++db) {
       const uint32_t chunk16 = ((db & 3) << 1) + ((lane >> 3) & 1);
@@ -347,6 +433,7 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
         mma_bf16_16816(acc[nb][db], vf, pb[nb][0], pb[nb][1]);
         if constexpr (MODE == kHiLo) mma_bf16_16816(acc[nb][db], vf, plo[nb][0], plo[nb][1]);
       }
+    }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(bar_empty + 8 * s);
@@ -381,13 +468,17 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
       float* base = f + L::kRedAcc + (warp * NCOL + nb * 8 + j0) * D;
+      // Accumulator rows g and g + 8 of d-block db: head-dim entries
+      // 16db + g and 16db + g + 8, or 16db + 2g and 16db + 2g + 1 on the fp8
+      // path (its V fragments permute the rows).
+      const int dstep = FP8 ? 1 : 8;
 #pragma unroll
       for (int db = 0; db < DBLK; ++db) {
-        const int d = db * 16 + (lane >> 2);
+        const int d = db * 16 + (FP8 ? 2 : 1) * (lane >> 2);
         base[d] = acc[nb][db][0];
         base[D + d] = acc[nb][db][1];
-        base[d + 8] = acc[nb][db][2];
-        base[D + d + 8] = acc[nb][db][3];
+        base[d + dstep] = acc[nb][db][2];
+        base[D + d + dstep] = acc[nb][db][3];
       }
       if (lane < 4) {
         f[L::kRedM + warp * NCOL + nb * 8 + j0] = m_run[nb][0];
@@ -419,7 +510,7 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
         e[w] = ex2(mw[w] - M);
         Ls += e[w] * f[L::kRedL + w * NCOL + t];
       }
-      const float inv = 1.f / Ls;
+      const float inv = a.v_scale / Ls;  // an fp8 V cache is dequantised here
 #pragma unroll
       for (int w = 0; w < kConsumerWarps; ++w) f[L::kRedW + w * NCOL + t] = e[w] * inv;
       f[L::kSplitLse + t] = (M + log2f(Ls)) * 0.69314718055994530942f;
@@ -452,12 +543,13 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
   }
 }
 
-// Split kernel: one CTA per (split, KV head, sequence).
-template <int D, int NB, int MODE, bool PAGED, int STAGES>
+// Split kernel: one CTA per (split, KV head, sequence).  FP8: the cache
+// holds e4m3 values (D = 128); the contraction runs on f16 tensor cores.
+template <int D, int NB, int MODE, bool PAGED, int STAGES, bool FP8>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     fd_split_kernel(const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const SplitArgs a) {
-  using L = SplitSmem<D, NB, STAGES>;
+  using L = SplitSmem<D, NB, STAGES, FP8>;
   static_assert(MODE != kDup || NB == 1, "duplicated columns need one column block");
 
   extern __shared__ uint8_t smem_raw[];
@@ -595,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
   } else {
     // ------------------------------------------------------------- consumers
-    split_consumers<D, NB, MODE, STAGES>(a, smem, smem_base, bar_full, bar_empty, cta_error,
+    split_consumers<D, NB, MODE, STAGES, FP8>(a, smem, smem_base, bar_full, bar_empty, cta_error,
                                          warp, lane, b, h0, split, start, end, n_tiles,
                                          n_parts);
   }

@@ -140,6 +140,42 @@ def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
     return (b.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
 
 
+# OCP 8-bit floating point, E4M3: sign, 4 exponent bits (bias 7), 3 mantissa
+# bits; exponent field 0 holds subnormals (m * 2^-9); S.1111.111 is NaN and
+# there is no infinity, so the largest finite magnitude is 1.75 * 2^8 = 448.
+E4M3_MAX = 448.0
+
+
+def e4m3_bits_to_f64(c: np.ndarray) -> np.ndarray:
+    c = np.asarray(c, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 7).astype(np.float64)
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((e == 15) & ((c & 7) == 7), np.nan, mag)
+    return sign * mag
+
+
+def f64_to_e4m3_bits(x: np.ndarray) -> np.ndarray:
+    """Round to nearest, ties to even, saturating at +-448 (finite input)."""
+    x = np.asarray(x, dtype=np.float64)
+    sign = (np.signbit(x)).astype(np.int64) << 7
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.clip(e, -6, 8)                      # binade; -6 also covers subnormals
+    step = np.exp2(e - 3)
+    q = np.rint(a / step) * step               # np.rint: ties to even
+    q = np.minimum(q, E4M3_MAX)
+    with np.errstate(divide="ignore"):
+        qe = np.floor(np.log2(np.where(q > 0, q, 1.0)))
+    normal = q >= 2.0 ** -6
+    ef = np.where(normal, qe + 7, 0).astype(np.int64)
+    mf = np.where(normal, q / np.exp2(qe) * 8 - 8, q / 2.0 ** -9)
+    code = sign | (ef << 3) | np.rint(mf).astype(np.int64)
+    return code.astype(np.uint8)
+
+
 @dataclass
 class Workload:
     """One decode-attention problem held on the host.
@@ -163,7 +199,14 @@ class Workload:
     block_size: int = 0
     block_table: Optional[np.ndarray] = None
     layout: str = "HND"
+    kv_dtype: str = "bf16"         # "bf16" (uint16 bits) or "fp8" (e4m3 codes, uint8)
+    k_scale: float = 1.0           # fp8: real K = k_scale * code
+    v_scale: float = 1.0
     meta: dict = field(default_factory=dict)
+
+    @property
+    def kv_dtype_code(self) -> int:
+        return 0 if self.kv_dtype == "bf16" else 1
 
     @property
     def kv_layout(self) -> int:
@@ -191,8 +234,17 @@ class Workload:
         return np.clip(self.seqlens.astype(np.int64), 0, self.max_len)
 
     def kv_bytes(self) -> int:
-        """Algorithmic K+V bytes: valid tokens x Hkv x D x 2 bytes x 2 tensors."""
-        return int(self.lengths().sum()) * self.Hkv * self.D * 4
+        """Algorithmic K+V bytes: valid tokens x Hkv x D x element bytes x 2."""
+        elem = 2 if self.kv_dtype == "bf16" else 1
+        return int(self.lengths().sum()) * self.Hkv * self.D * elem * 2
+
+    def logical_kv_f64(self, b: int, h: int):
+        """Real (dequantised) K, V rows [n, D] of sequence b, KV head h, in fp64."""
+        k, v = self.logical_kv(b, h)
+        if self.kv_dtype == "bf16":
+            return bf16_bits_to_f64(k), bf16_bits_to_f64(v)
+        return (float(np.float32(self.k_scale)) * e4m3_bits_to_f64(k),
+                float(np.float32(self.v_scale)) * e4m3_bits_to_f64(v))
 
     def logical_kv(self, b: int, h: int):
         """K, V rows [n, D] (bf16 bits) of sequence b, KV head h, in token order."""
@@ -215,7 +267,8 @@ class Workload:
 def make_problem(B: int, Hq: int, Hkv: int, D: int, max_len: int, seed: int,
                  seqlens=None, nan_pad: bool = False, block_size: int = 0,
                  num_blocks: Optional[int] = None, name: str = "custom",
-                 nthreads: Optional[int] = None, layout: str = "HND") -> Workload:
+                 nthreads: Optional[int] = None, layout: str = "HND", kv_dtype: str = "bf16",
+                 kv_scale: float = 1.0 / 32) -> Workload:
     """Build a workload with i.i.d. N(0,1) bf16 q, K, V from base `seed`.
 
     Contiguous cache when block_size == 0.  Paged cache otherwise: the
@@ -223,8 +276,10 @@ def make_problem(B: int, Hq: int, Hkv: int, D: int, max_len: int, seed: int,
     sequence) and the block table is a seeded permutation of the pool,
     reshaped [B, max_len / block_size].  `layout` orders the cache dims
     ("HND": heads outside tokens, "NHD": tokens outside heads); K and V are
-    drawn in the storage order of that layout."""
-    assert layout in ("HND", "NHD")
+    drawn in the storage order of that layout.  kv_dtype "fp8": K and V hold
+    e4m3 codes of N(0,1) / kv_scale (so the real values, kv_scale * code, are
+    N(0,1) rounded to e4m3), with k_scale = v_scale = kv_scale."""
+    assert layout in ("HND", "NHD") and kv_dtype in ("bf16", "fp8")
     q = normal_bf16(stream_seed(seed, STREAM_Q), (B, Hq, D), nthreads=nthreads)
     if block_size:
         assert max_len % block_size == 0
@@ -237,21 +292,29 @@ def make_problem(B: int, Hq: int, Hkv: int, D: int, max_len: int, seed: int,
     else:
         table = None
         shape = (B, Hkv, max_len, D) if layout == "HND" else (B, max_len, Hkv, D)
-    k = normal_bf16(stream_seed(seed, STREAM_K), shape, nthreads=nthreads)
-    v = normal_bf16(stream_seed(seed, STREAM_V), shape, nthreads=nthreads)
+    if kv_dtype == "bf16":
+        k = normal_bf16(stream_seed(seed, STREAM_K), shape, nthreads=nthreads)
+        v = normal_bf16(stream_seed(seed, STREAM_V), shape, nthreads=nthreads)
+    else:
+        n = int(np.prod(shape))
+        k = f64_to_e4m3_bits(normal_f64(stream_seed(seed, STREAM_K), n) / kv_scale).reshape(shape)
+        v = f64_to_e4m3_bits(normal_f64(stream_seed(seed, STREAM_V), n) / kv_scale).reshape(shape)
     sl = None if seqlens is None else np.asarray(seqlens, dtype=np.int32)
     if nan_pad and sl is not None:
         assert not block_size
+        nan = BF16_NAN if kv_dtype == "bf16" else np.uint8(0x7F)
         for b in range(B):
             if layout == "HND":
-                k[b, :, int(sl[b]):, :] = BF16_NAN
-                v[b, :, int(sl[b]):, :] = BF16_NAN
+                k[b, :, int(sl[b]):, :] = nan
+                v[b, :, int(sl[b]):, :] = nan
             else:
-                k[b, int(sl[b]):, :, :] = BF16_NAN
-                v[b, int(sl[b]):, :, :] = BF16_NAN
+                k[b, int(sl[b]):, :, :] = nan
+                v[b, int(sl[b]):, :, :] = nan
     return Workload(name=name, B=B, Hq=Hq, Hkv=Hkv, D=D, max_len=max_len, q=q, k=k, v=v,
                     scale=float(np.float32(1.0 / math.sqrt(D))), seqlens=sl,
-                    block_size=block_size, block_table=table, layout=layout)
+                    block_size=block_size, block_table=table, layout=layout, kv_dtype=kv_dtype,
+                    k_scale=kv_scale if kv_dtype == "fp8" else 1.0,
+                    v_scale=kv_scale if kv_dtype == "fp8" else 1.0)
 
 
 def plant_dominant_keys(w: Workload, count: int, seed: int, magnitude: float = 4.0) -> np.ndarray:

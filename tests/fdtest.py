@@ -39,6 +39,11 @@ def dev_i32(a):
     return None if a is None else t.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
 
 
+def dev_u8(a: np.ndarray):
+    t = torch()
+    return t.from_numpy(np.ascontiguousarray(a, dtype=np.uint8)).cuda()
+
+
 def host_bf16(x) -> np.ndarray:
     t = torch()
     return wl.bf16_bits_to_f64(x.view(t.int16).cpu().numpy().view(np.uint16))
@@ -50,15 +55,17 @@ class OnDevice:
     def __init__(self, w: wl.Workload):
         self.w = w
         self.q = dev_bf16(w.q)
-        self.k = dev_bf16(w.k)
-        self.v = dev_bf16(w.v)
+        up = dev_bf16 if w.kv_dtype == "bf16" else dev_u8
+        self.k = up(w.k)
+        self.v = up(w.v)
         self.seqlens = dev_i32(w.seqlens)
         self.table = dev_i32(w.block_table)
 
     def problem(self):
         w = self.w
         return fd.make_problem(w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size, w.num_blocks,
-                               w.max_blocks_per_seq, w.kv_layout)
+                               w.max_blocks_per_seq, w.kv_layout, w.kv_dtype_code, w.k_scale,
+                               w.v_scale)
 
     def plan(self) -> int:
         """The split count the benchmark uses: the length-aware planner when
@@ -102,7 +109,7 @@ def reference(w: wl.Workload, groups=None, nthreads=None):
     computed are NaN.  Paged caches are gathered to logical token order
     first (the oracle only sees logical K/V)."""
     nthreads = nthreads or os.cpu_count() or 1
-    if groups is None and not w.paged and w.layout == "HND":
+    if groups is None and not w.paged and w.layout == "HND" and w.kv_dtype == "bf16":
         return oracle.decode(w.q, w.k, w.v, w.scale, seqlens=w.seqlens, nthreads=nthreads)
     if groups is None:
         groups = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
@@ -112,9 +119,14 @@ def reference(w: wl.Workload, groups=None, nthreads=None):
 
     def one(bh):
         b, h = bh
-        k, v = w.logical_kv(b, h)
-        o, l = oracle.attend(w.q[b, h * G:(h + 1) * G], np.ascontiguousarray(k),
-                             np.ascontiguousarray(v), w.scale)
+        if w.kv_dtype == "bf16":
+            k, v = w.logical_kv(b, h)
+            o, l = oracle.attend(w.q[b, h * G:(h + 1) * G], np.ascontiguousarray(k),
+                                 np.ascontiguousarray(v), w.scale)
+        else:  # dequantised fp8 values in fp64
+            k, v = w.logical_kv_f64(b, h)
+            o, l = oracle.attend_f64(wl.bf16_bits_to_f64(w.q[b, h * G:(h + 1) * G]), k, v,
+                                     float(np.float32(w.scale)))
         return b, h, o, l
 
     with ThreadPoolExecutor(max_workers=nthreads) as ex:

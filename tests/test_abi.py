@@ -177,12 +177,12 @@ def test_decode_rejects_unknown_layout():
 
 def test_problem_struct_matches_header():
     import ctypes
-    # nine int32 fields, in the order of fd_problem in include/fd.h
-    assert ctypes.sizeof(fd.fd_problem) == 9 * 4
+    # ten int32 fields and two floats, in the order of fd_problem in include/fd.h
+    assert ctypes.sizeof(fd.fd_problem) == 12 * 4
     names = [f[0] for f in fd.fd_problem._fields_]
     text = open(os.path.join(ROOT, "include", "fd.h")).read()
     body = text[text.index("typedef struct fd_problem {"):text.index("} fd_problem;")]
-    assert names == re.findall(r"int32_t (\w+);", body)
+    assert names == re.findall(r"(?:int32_t|float) (\w+);", body)
 
 
 def test_decode_rejects_bad_scalars():
@@ -243,3 +243,18 @@ def test_partial_and_combine_reject_bad_arguments():
     assert fd.fd_combine(2, 1, 8, 96, Q, K, O, None, 0) == fd.FD_ERR_UNSUPPORTED
     assert fd.fd_combine(2, 1, 8, 128, Q + 4, K, O, None, 0) == fd.FD_ERR_INVALID_ARGUMENT
     assert fd.fd_combine(2, 1, 8, 128, None, K, O, None, 0) == fd.FD_ERR_INVALID_ARGUMENT
+
+
+def test_fp8_cache_checks():
+    prob = P(D=128)
+    prob.kv_dtype = 1
+    prob.k_scale, prob.v_scale = 0.0, 1.0
+    assert decode(prob) == fd.FD_ERR_INVALID_ARGUMENT      # scale must be > 0
+    prob.k_scale, prob.v_scale = 1.0, float("nan")
+    assert decode(prob) == fd.FD_ERR_INVALID_ARGUMENT
+    prob = P(D=64)
+    prob.kv_dtype, prob.k_scale, prob.v_scale = 1, 1.0, 1.0
+    assert decode(prob) == fd.FD_ERR_UNSUPPORTED            # fp8 needs D = 128
+    prob = P()
+    prob.kv_dtype = 7
+    assert decode(prob) == fd.FD_ERR_INVALID_ARGUMENT

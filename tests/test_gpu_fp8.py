@@ -1,0 +1,124 @@
+"""GPU parity of the fp8 e4m3 KV-cache path against the fp64 oracle.
+
+The oracle sees the dequantised cache (k_scale * code, v_scale * code, exact
+in fp64) and the bf16 queries; the kernel multiplies the codes in f16 on the
+tensor cores and applies the scales in fp32.  Same tolerances as the bf16
+path.  Covers every group size, ragged lengths with NaN-coded padding, forced
+split counts, paged versus contiguous and token-major versus head-major bit
+identity, determinism, unequal non-power-of-two scales and a long context."""
+import dataclasses
+
+import numpy as np
+import pytest
+
+from split_kv_decode_attn_b200 import workloads as wl
+
+from fdtest import OnDevice, assert_close, free_device, reference, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _gpu(cuda_device):
+    yield
+    free_device()
+
+
+def contiguous_copy(p: wl.Workload) -> wl.Workload:
+    """The same logical fp8 cache as a contiguous [B, Hkv, L, D] array."""
+    kc = np.zeros((p.B, p.Hkv, p.max_len, p.D), np.uint8)
+    vc = np.zeros_like(kc)
+    for b in range(p.B):
+        for h in range(p.Hkv):
+            k, v = p.logical_kv(b, h)
+            kc[b, h, :len(k)] = k
+            vc[b, h, :len(v)] = v
+    return dataclasses.replace(p, name="contig", k=kc, v=vc, block_table=None, block_size=0,
+                               layout="HND")
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
+def test_fp8_group_sizes_and_ragged_lengths(G):
+    Hkv = 2
+    lens = [0, 1, 63, 64, 65, 200, 777, 2000]
+    w = wl.make_problem(len(lens), G * Hkv, Hkv, 128, 2000, seed=300 + G, seqlens=lens,
+                        nan_pad=True, kv_dtype="fp8")
+    d = OnDevice(w)
+    ref, rl = reference(w)
+    for S in (1, 2, 3, 7, 16, 32):
+        got, gl, _ = run_gpu(d, S)
+        assert_close(got, gl, ref, rl, f"fp8 G={G} S={S}")
+
+
+@pytest.mark.parametrize("layout", ["HND", "NHD"])
+@pytest.mark.parametrize("bs", [16, 64, 256])
+def test_fp8_paged_matches_contiguous_bit_for_bit(bs, layout):
+    B, Hq, Hkv, L = 3, 64, 8, 1024
+    p = wl.make_problem(B, Hq, Hkv, 128, L, seed=340 + bs, seqlens=[1024, 517, 64],
+                        block_size=bs, num_blocks=B * L // bs + 3, layout=layout,
+                        kv_dtype="fp8")
+    c = contiguous_copy(p)
+    dp, dc = OnDevice(p), OnDevice(c)
+    ref, rl = reference(c)
+    for S in (1, 5):
+        gp, lp, _ = run_gpu(dp, S)
+        gc_, lc, _ = run_gpu(dc, S)
+        assert_close(gp, lp, ref, rl, f"fp8 paged {layout} bs={bs} S={S}")
+        assert np.array_equal(gp, gc_) and np.array_equal(lp, lc)
+
+
+def test_fp8_token_major_matches_head_major():
+    B, Hkv, L = 3, 4, 1500
+    n = wl.make_problem(B, 16 * Hkv // 4, Hkv, 128, L, seed=360, seqlens=[1500, 9, 640],
+                        nan_pad=True, layout="NHD", kv_dtype="fp8")
+    h = dataclasses.replace(n, name="hnd", layout="HND",
+                            k=np.ascontiguousarray(n.k.transpose(0, 2, 1, 3)),
+                            v=np.ascontiguousarray(n.v.transpose(0, 2, 1, 3)))
+    dn, dh = OnDevice(n), OnDevice(h)
+    ref, rl = reference(h)
+    for S in (1, 6):
+        gn, ln_, _ = run_gpu(dn, S)
+        gh, lh, _ = run_gpu(dh, S)
+        assert_close(gn, ln_, ref, rl, f"fp8 NHD S={S}")
+        assert np.array_equal(gn, gh) and np.array_equal(ln_, lh)
+
+
+def test_fp8_unequal_scales():
+    w = wl.make_problem(2, 32, 4, 128, 3000, seed=370, seqlens=[3000, 1234], kv_dtype="fp8")
+    w = dataclasses.replace(w, k_scale=0.0217, v_scale=0.0461)
+    d = OnDevice(w)
+    ref, rl = reference(w)
+    for S in (1, 4, 11):
+        got, gl, _ = run_gpu(d, S)
+        assert_close(got, gl, ref, rl, f"fp8 scales S={S}")
+
+
+def test_fp8_single_token_returns_scaled_v0_exactly():
+    w = wl.make_problem(2, 16, 2, 128, 64, seed=380, seqlens=[1, 1], kv_dtype="fp8")
+    d = OnDevice(w)
+    got, _, _ = run_gpu(d, 1)
+    for b in range(2):
+        for h in range(16):
+            v0 = w.v_scale * wl.e4m3_bits_to_f64(w.v[b, h // w.G, 0])
+            assert np.array_equal(got[b, h], v0)
+
+
+def test_fp8_repeated_runs_are_bit_identical():
+    w = wl.make_problem(2, 64, 8, 128, 5000, seed=390, seqlens=[5000, 2999], kv_dtype="fp8")
+    d = OnDevice(w)
+    for S in (1, 9):
+        a, la, _ = run_gpu(d, S)
+        for _ in range(2):
+            b, lb, _ = run_gpu(d, S)
+            assert np.array_equal(a, b) and np.array_equal(la, lb)
+
+
+def test_fp8_codellama34b_shape_long_context():
+    """B=1, Hq=64, Hkv=8, L=65536 in the planner's split count; the oracle
+    computes two KV heads (16 query rows)."""
+    w = wl.make_problem(1, 64, 8, 128, 65536, seed=395, kv_dtype="fp8")
+    d = OnDevice(w)
+    got, gl, S = run_gpu(d)
+    ref, rl = reference(w, groups=[(0, 0), (0, 5)])
+    e = assert_close(got, gl, ref, rl, f"fp8 L=64K S={S}")
+    print(f"fp8 64K planner S={S} errors {e}")

@@ -20,10 +20,10 @@ MUTANTS = {
     "lse without max": ("*lse = m + std::log(Z);", "*lse = std::log(Z);"),
     "output not normalised": ("for (int d = 0; d < D; ++d) out[d] /= Z;",
                               "for (int d = 0; d < D; ++d) out[d] /= (Z + 1.0);"),
-    "value read from keys": ("out[d] += p * bf16_to_double(v[j * ld + d]);",
-                             "out[d] += p * bf16_to_double(k[j * ld + d]);"),
-    "key read from values": ("dot += bf16_to_double(q[d]) * bf16_to_double(k[j * ld + d]);",
-                             "dot += bf16_to_double(q[d]) * bf16_to_double(v[j * ld + d]);"),
+    "value read from keys": ("out[d] += p * load(v, j * ld + d);",
+                             "out[d] += p * load(k, j * ld + d);"),
+    "key read from values": ("dot += load(q, d) * load(k, j * ld + d);",
+                             "dot += load(q, d) * load(v, j * ld + d);"),
     "GQA interleaved mapping": ("kv = h / G;", "kv = h % Hkv;"),
     "chunk end off by one": ("long end = (s + 1) * C < n ? (s + 1) * C : n;",
                              "long end = (s + 1) * C - 1 < n ? (s + 1) * C - 1 : n;"),

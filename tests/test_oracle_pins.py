@@ -291,3 +291,21 @@ def test_split_of_empty_sequence():
     k = np.zeros((0, 8), np.uint16)
     out, lse = oracle.attend_split(q, k, k, 0.5, 16)
     assert np.all(out == 0) and np.all(np.isneginf(lse))
+
+
+def test_f64_inputs_match_bf16_inputs_exactly():
+    """The fp64 entry point runs the same arithmetic on already-widened values."""
+    n, D = 123, 64
+    q, k, v = rnd_bf16(60, (4, D)), rnd_bf16(61, (n, D)), rnd_bf16(62, (n, D))
+    out, lse = oracle.attend(q, k, v, 0.125)
+    out2, lse2 = oracle.attend_f64(f64(q), f64(k), f64(v), float(np.float32(0.125)))
+    assert np.array_equal(out, out2) and np.array_equal(lse, lse2)
+
+
+def test_f64_inputs_against_scipy_on_non_bf16_values():
+    rng = np.random.default_rng(5)
+    q, k, v = rng.normal(size=(2, 16)), rng.normal(size=(40, 16)), rng.normal(size=(40, 16))
+    out, lse = oracle.attend_f64(q, k, v, 0.3)
+    s = 0.3 * (q @ k.T)
+    np.testing.assert_allclose(out, scipy.special.softmax(s, axis=1) @ v, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(lse, scipy.special.logsumexp(s, axis=1), rtol=1e-13)

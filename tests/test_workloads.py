@@ -103,3 +103,29 @@ def test_token_major_layouts():
     assert p.k.shape == (12, 16, 2, 64)
     k, v = p.logical_kv(0, 1)
     assert np.array_equal(k[16:32], p.k[p.block_table[0, 1], :, 1])
+
+
+def test_e4m3_codec_against_the_format_definition():
+    """OCP FP8 E4M3: bias 7, 3 mantissa bits, subnormals m * 2^-9, S.1111.111
+    is NaN, largest finite 448."""
+    table = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6,
+             0x38: 1.0, 0x39: 1.125, 0x3F: 1.875, 0x40: 2.0, 0x7E: 448.0, 0xB8: -1.0,
+             0xFE: -448.0}
+    for c, val in table.items():
+        assert wl.e4m3_bits_to_f64(np.array([c]))[0] == val
+    assert np.isnan(wl.e4m3_bits_to_f64(np.array([0x7F, 0xFF]))).all()
+    finite = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
+    back = wl.f64_to_e4m3_bits(wl.e4m3_bits_to_f64(finite))
+    assert np.array_equal(back, finite)
+    # nearest, ties to even, saturation
+    x = np.array([1.0625, 1.1875, 2.0 ** -10, 3 * 2.0 ** -11, 500.0, -1e9, 0.3])
+    assert list(wl.f64_to_e4m3_bits(x)) == [0x38, 0x3A, 0x00, 0x01, 0x7E, 0xFE, 0x2A]
+
+
+def test_fp8_workload_recipe():
+    w = wl.make_problem(2, 8, 2, 128, 64, seed=4, seqlens=[64, 10], nan_pad=True, kv_dtype="fp8")
+    assert w.k.dtype == np.uint8 and w.kv_dtype_code == 1 and w.k_scale == 1 / 32
+    assert np.all(w.k[1, :, 10:] == 0x7F)
+    k, _ = w.logical_kv_f64(0, 1)
+    assert np.isfinite(k).all() and 0.8 < np.std(k) < 1.2
+    assert w.kv_bytes() == (64 + 10) * 2 * 128 * 2
