@@ -70,7 +70,7 @@ def parse_args():
     ap.add_argument("--shard-sequence", action="store_true",
                     help="sequence-parallel: the ranks split one history (strong scaling)")
     ap.add_argument("--crossover", action="store_true",
-                    help="concurrency sweep: batch x cache length, planner pick vs one split")
+                    help="planner sweep: split-count ladders over batch, length, element type")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -109,8 +109,9 @@ def kernel_source_hash() -> str:
 
 
 def ncu_traffic(workload: str):
-    """Per-launch DRAM bytes of the split kernel from the committed ncu summary,
-    if it was taken on the current kernel sources; else None."""
+    """DRAM bytes (read + write) per launch of the split kernel, the dominant
+    kernel, from the committed ncu summary, if it was taken on the current
+    kernel sources; else None."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
@@ -118,7 +119,7 @@ def ncu_traffic(workload: str):
         if j.get("source_hash") != kernel_source_hash():
             return None
         entry = j.get("workloads", {}).get(workload)
-        return None if entry is None else float(entry["bytes_per_call"])
+        return None if entry is None else float(entry["split_kernel_bytes"])
     except Exception:
         return None
 
@@ -216,11 +217,8 @@ class Call:
                                     w.k_scale, w.v_scale)
         if num_splits:
             self.S = num_splits
-        elif w.seqlens is not None:  # lengths known on the host: length-aware planner
-            self.S = fd.fd_plan_seqlens(0, w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size,
-                                        w.seqlens)
-        else:
-            self.S = fd.fd_plan(w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size)
+        else:  # the planner over the whole problem, lengths included when known
+            self.S = fd.fd_plan_problem(0, self.prob, w.seqlens)
         assert self.S >= 1, fd.fd_status_string(self.S)
         chunk = fd.fd_split_chunk(w.max_len, self.S)
         self.s_eff = max(1, -(-w.max_len // chunk)) if w.max_len else 1
@@ -437,11 +435,16 @@ def run_fd(args):
                    "l2": f"inputs rotate over {copies} cache copies "
                          f"({copies * (w.k.nbytes + w.v.nbytes) / 1e6:.0f} MB, L2 {l2 / 1e6:.0f} MB)",
                    "parallelism": f"replicas{world}" if world > 1 else "single"},
+        # achieved: algorithmic bytes over the whole call's event-timed duration
+        # (the split kernel, the dominant one, plus the combine), so it is a
+        # lower bound for the split kernel alone; traffic: the split kernel's
+        # DRAM bytes per launch from ncu
         "roofline": {"bound": "hbm", "kernel": "fd_decode (split + combine)",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                      "frac_of_spec_8tbs": round(achieved / SPEC_HBM_GBS, 4),
-                     "traffic": ncu_traffic(w.name)},
+                     "traffic": ncu_traffic(w.name), "traffic_kernel": "fd_split_kernel",
+                     "algorithmic_bytes": kvb},
         "gpu_launches": args.steps * call.launches_per_call,
         "clocks": clocks,
     }
@@ -608,43 +611,64 @@ def run_sharded(args):
 
 
 def crossover(args):
-    """Batch size x cache length on the CodeLlama-34B head shape (Hq=64,
-    Hkv=8, D=128, contiguous): one split, the planner's pick, and a ladder of
-    split counts, timed on the device from CUDA-graph replays (the call's own
-    cost; eager calls below ~2K tokens are bound by the host's launch work).
-    One JSON line per (B, L) on stdout."""
+    """Split-count sweep for the planner: device microseconds per fd_decode
+    call over a ladder of split counts, timed from CUDA-graph replays (the
+    call's own cost; eager calls below ~2K tokens are bound by the host's
+    launch work), with cache copies rotated past L2.  Shapes: the CodeLlama-34B
+    head shape (Hq=64, Hkv=8, D=128) at B=1 over L = 512..128K and at B = 2..40
+    over L = 2K..64K, bf16 and fp8 caches; G=4; the varlen, paged and peaked
+    workloads.  One JSON line per shape on stdout, with the planner's pick
+    (fd_plan_problem) and its regret against the fastest measured count."""
     import torch
     import split_kv_decode_attn_b200 as fd
     from split_kv_decode_attn_b200 import workloads as wl
     torch.cuda.set_device(0)
     device = torch.device("cuda", 0)
     fd.load_library()
-    peak, _ = measured_peak()
-    for B in (1, 4, 16, 64, 256):
-        for L in (512, 2048, 8192, 16384, 65536):
-            kv = B * 8 * L * 128 * 4
-            if kv > 9e9:
+    ladder = (1, 2, 3, 4, 6, 8, 12, 16, 20, 24, 28, 32, 40, 48, 64)
+
+    def run(w, Ss, tag):
+        copies, _ = copies_for(torch, w.k.nbytes + w.v.nbytes, device)
+        prob = fd.make_problem(w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size, w.num_blocks,
+                               w.max_blocks_per_seq, w.kv_layout, w.kv_dtype_code, w.k_scale,
+                               w.v_scale)
+        plan = fd.fd_plan_problem(0, prob, w.seqlens)
+        times = {}
+        for S in sorted(set(Ss) | {plan}):
+            call = Call(torch, fd, w, device, S, copies)
+            est = timed_graph(torch, call, copies, 3, warmup=1)
+            times[S] = timed_graph(torch, call, copies, max(3, int(60000 / max(est, 1.0) / copies)))
+            del call
+        torch.cuda.empty_cache()
+        best = min(times, key=times.get)
+        kv = w.kv_bytes()
+        print(json.dumps({"tag": tag, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "L": w.max_len,
+                          "bs": w.block_size, "kv": w.kv_dtype, "kv_bytes": kv, "plan": plan,
+                          "us": {str(k): round(v, 2) for k, v in sorted(times.items())},
+                          "best": best, "plan_regret": round(times[plan] / times[best] - 1, 4),
+                          "plan_GBs": round(kv / times[plan] / 1e3, 1)}), flush=True)
+
+    for L in (512, 1024, 2048, 4096, 8192, 16384, 32768, 65536, 131072):
+        for kvd in ("bf16", "fp8"):
+            w = make_workload("codellama34b", L, 0, kv_dtype=kvd)
+            run(w, [s for s in ladder if s <= L // 64], f"B1-L{L}-{kvd}")
+    for L in (16384, 65536):
+        run(wl.make_problem(1, 32, 8, 128, L, wl.CONFIG_SEED_BASE + 300, name="g4"),
+            [s for s in ladder if s <= L // 64], f"G4-B1-L{L}")
+    for B in (2, 4, 8, 16, 32, 40):
+        for L in (2048, 8192, 16384, 65536):
+            if B * 8 * L * 128 * 4 > 4.5e9:
                 continue
-            w = wl.make_problem(B, 64, 8, 128, L, wl.CONFIG_SEED_BASE + 200 + B, name=f"B{B}-L{L}")
-            copies, _ = copies_for(torch, w.k.nbytes + w.v.nbytes, device)
-            plan = fd.fd_plan(B, 64, 8, 128, L, 0)
-            times = {}
-            for S in sorted({1, plan, 2, 4, 8, 16, 24, 32}):
-                if S > max(1, L // 64):
-                    continue
-                call = Call(torch, fd, w, device, S, copies)
-                est = timed(torch, call, 3, 2) / 3
-                steps = int(max(10, min(5000, 150.0 / max(est, 1e-3))))
-                times[S] = timed_graph(torch, call, copies, max(1, steps // copies))
-                del call
-            torch.cuda.empty_cache()
-            best = min(times, key=times.get)
-            print(json.dumps({"B": B, "L": L, "kv_bytes": kv, "plan": plan,
-                              "us": {str(k): round(v, 2) for k, v in times.items()},
-                              "best": best, "plan_regret": round(times[plan] / times[best] - 1, 4),
-                              "split_gain_vs_1": round(times[1] / times[plan], 3),
-                              "plan_GBs": round(kv / times[plan] / 1e3, 1),
-                              "plan_frac": round(kv / times[plan] / 1e3 / peak, 4)}), flush=True)
+            for kvd in (("bf16", "fp8") if B in (4, 16) else ("bf16",)):
+                w = wl.make_problem(B, 64, 8, 128, L, wl.CONFIG_SEED_BASE + 200 + B,
+                                    name=f"B{B}-L{L}", kv_dtype=kvd)
+                run(w, [s for s in (1, 2, 3, 4, 6, 8, 12, 16, 24, 32) if s <= L // 64],
+                    f"B{B}-L{L}-{kvd}")
+    for kvd in ("bf16", "fp8"):
+        run(make_workload("varlen", None, 0, kv_dtype=kvd), [1, 2, 3, 4, 6, 8], f"varlen-{kvd}")
+    run(make_workload("paged", None, 0), [1, 2, 3, 4, 6, 8], "paged-bf16")
+    run(make_workload("peaked", None, 0), [8, 12, 16, 20, 24, 32, 48, 64], "peaked-bf16")
+    assert fd.fd_check_device_error() == 0
 
 
 # ------------------------------------------------------- reference arm

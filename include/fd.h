@@ -143,6 +143,20 @@ FD_API int fd_plan_sm(int num_sms, int B, int Hq, int Hkv, int D, int max_len,
 FD_API int fd_plan_seqlens(int num_sms, int B, int Hq, int Hkv, int D, int max_len,
                            int block_size, const int32_t* seqlens);
 
+/* The planner for a whole problem description: the same cost model, with
+ * the cache's element type (an fp8 CTA moves half the bytes of a bf16 one
+ * at the same token rate, so fp8 caches want more CTAs in flight) and, when
+ * given, the lengths. fd_plan and fd_plan_seqlens plan for bf16 caches.
+ *   num_sms   SM count to plan for; <= 0 means the current device's
+ *   p         HOST pointer to the problem as passed to fd_decode (pointers
+ *             and scales are not read)
+ *   seqlens   HOST array [B] of valid tokens per sequence, or NULL when
+ *             every sequence holds max_len
+ * Returns S >= 1, or a negative fd_status: FD_ERR_INVALID_ARGUMENT for a
+ * NULL p, a bad shape or an unknown kv_dtype; FD_ERR_UNSUPPORTED for an fp8
+ * cache with D != 128. Host only and deterministic. */
+FD_API int fd_plan_problem(int num_sms, const fd_problem* p, const int32_t* seqlens);
+
 /* Tokens per split for a given split count. This is ceil(max_len /
  * num_splits) rounded up to the 64-token tile. Split s covers tokens
  * [s*chunk, (s+1)*chunk) of every sequence, and splits past a sequence's end

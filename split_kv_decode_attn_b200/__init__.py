@@ -27,7 +27,7 @@ FD_ERR_CUDA = -4
 FD_ERR_DEVICE_TIMEOUT = -5
 
 # Entry points declared in include/fd.h.
-EXPORTS = ("fd_plan", "fd_plan_sm", "fd_plan_seqlens", "fd_split_chunk", "fd_workspace_bytes", "fd_decode",
+EXPORTS = ("fd_plan", "fd_plan_sm", "fd_plan_seqlens", "fd_plan_problem", "fd_split_chunk", "fd_workspace_bytes", "fd_decode",
            "fd_decode_partial", "fd_combine", "fd_decode_static_workspace", "fd_check_device_error",
            "fd_selftest_device_timeout", "fd_status_string")
 
@@ -74,6 +74,8 @@ def load_library(path: str = LIB_PATH):
         lib.fd_plan_sm.restype = I
         lib.fd_plan_seqlens.argtypes = [I] * 7 + [vp]
         lib.fd_plan_seqlens.restype = I
+        lib.fd_plan_problem.argtypes = [I, ctypes.POINTER(fd_problem), vp]
+        lib.fd_plan_problem.restype = I
         lib.fd_split_chunk.argtypes = [I, I]
         lib.fd_split_chunk.restype = I
         lib.fd_workspace_bytes.argtypes = [I, I, I, I]
@@ -138,6 +140,15 @@ def fd_plan_seqlens(num_sms: int, B: int, Hq: int, Hkv: int, D: int, max_len: in
     sl = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32))
     return int(load_library().fd_plan_seqlens(num_sms, B, Hq, Hkv, D, max_len, block_size,
                                               sl.ctypes.data))
+
+
+def fd_plan_problem(num_sms: int, prob: "fd_problem", seqlens=None) -> int:
+    """Planner for a whole problem (element type included); `seqlens` is a
+    host sequence of B ints or None (every sequence holds max_len)."""
+    import numpy as np
+    sl = None if seqlens is None else np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32))
+    return int(load_library().fd_plan_problem(num_sms, ctypes.byref(prob),
+                                              None if sl is None else sl.ctypes.data))
 
 
 def fd_split_chunk(max_len: int, num_splits: int) -> int:
@@ -206,26 +217,31 @@ def make_problem(B, Hq, Hkv, D, max_len, block_size=0, num_blocks=0, max_blocks_
 
 def decode(q, k_cache, v_cache, seqlens=None, block_table=None, *, max_len: Optional[int] = None,
            kv_layout: int = FD_LAYOUT_HND, scale: Optional[float] = None,
-           num_splits: Optional[int] = None, out=None, lse=None, workspace=None, stream=None):
+           num_splits: Optional[int] = None, out=None, lse=None, workspace=None, stream=None,
+           k_scale: float = 1.0, v_scale: float = 1.0):
     """Decode attention on torch CUDA tensors.
 
-    q [B, Hq, D] bf16.  Caches (bf16): FD_LAYOUT_HND contiguous
-    [B, Hkv, max_len, D] or paged [num_blocks, Hkv, block_size, D];
-    FD_LAYOUT_NHD contiguous [B, max_len, Hkv, D] or paged
-    [num_blocks, block_size, Hkv, D].  Paged caches come with block_table
-    [B, max_blocks] int32.  seqlens [B] int32 or None.  Returns
-    (out [B, Hq, D] bf16, lse [B, Hq] fp32).  num_splits defaults to
-    fd_plan's choice."""
+    q [B, Hq, D] bf16.  Caches: bf16, or E4M3 codes (torch.uint8 or
+    torch.float8_e4m3fn, D = 128) whose real values are k_scale * code and
+    v_scale * code.  FD_LAYOUT_HND contiguous [B, Hkv, max_len, D] or paged
+    [num_blocks, Hkv, block_size, D]; FD_LAYOUT_NHD contiguous
+    [B, max_len, Hkv, D] or paged [num_blocks, block_size, Hkv, D].  Paged
+    caches come with block_table [B, max_blocks] int32.  seqlens [B] int32
+    or None.  Returns (out [B, Hq, D] bf16, lse [B, Hq] fp32).  num_splits
+    defaults to fd_plan_problem's choice."""
     import torch
     B, Hq, D = q.shape
     block_size = 0
+    fp8 = k_cache.element_size() == 1
+    kv_dtype = FD_KV_FP8_E4M3 if fp8 else FD_KV_BF16
     if block_table is None:
         if kv_layout == FD_LAYOUT_HND:
             _, Hkv, L, _ = k_cache.shape
         else:
             _, L, Hkv, _ = k_cache.shape
         max_len = L if max_len is None else max_len
-        prob = make_problem(B, Hq, Hkv, D, max_len, kv_layout=kv_layout)
+        prob = make_problem(B, Hq, Hkv, D, max_len, kv_layout=kv_layout, kv_dtype=kv_dtype,
+                            k_scale=k_scale, v_scale=v_scale)
     else:
         if kv_layout == FD_LAYOUT_HND:
             nb, Hkv, bs, _ = k_cache.shape
@@ -234,13 +250,14 @@ def decode(q, k_cache, v_cache, seqlens=None, block_table=None, *, max_len: Opti
         block_size = bs
         mbps = block_table.shape[1]
         max_len = mbps * bs if max_len is None else max_len
-        prob = make_problem(B, Hq, Hkv, D, max_len, bs, nb, mbps, kv_layout)
+        prob = make_problem(B, Hq, Hkv, D, max_len, bs, nb, mbps, kv_layout, kv_dtype, k_scale,
+                            v_scale)
     if scale is None:
         scale = 1.0 / (D ** 0.5)
     if num_splits is None:
-        num_splits = fd_plan(B, Hq, Hkv, D, max_len, block_size)
+        num_splits = fd_plan_problem(0, prob)
         if num_splits < 0:
-            raise FdError(num_splits, "fd_plan")
+            raise FdError(num_splits, "fd_plan_problem")
     if out is None:
         out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
     if lse is None:

@@ -18,31 +18,38 @@
 namespace {
 
 constexpr int kMaxSplits = 1024;
+// Tiles a split CTA may prefetch into L2 before its inputs are released.
+constexpr int kPrefetchTiles = 4;
 constexpr int kMaxDevices = 64;
 
 // ---------------------------------------------------------------- planner
 
 // Cost model of one call, in microseconds, used to pick the split count.
 // It models device time: the constants were fitted to split-count sweeps
-// measured on B200 from CUDA-graph replays (free of the host's launch work),
-// over the five workload shapes and a batch x length grid (B = 1..256,
-// L = 512..64K) on the CodeLlama-34B head shape.  Over those shapes the
-// planner's pick is the fastest measured split count or within 3.5 % of it.
-//   kHbmGBs      streaming rate of the whole device
-//   kCtaGBs      rate of one CTA alone on an SM (contiguous cache)
-//   kCtaPagedGBs the same when pages hold fewer than 64 tokens (one TMA box
-//                per page instead of one per tile)
-//   kSmPairGBs   rate of an SM running two CTAs, both together
-//   kCtaFixedUs  per-CTA fixed cost within a wave
-//   kCombineUs   extra device time of a call with several splits (the
-//                combine kernel after its dependency)
+// measured on B200 from CUDA-graph replays (free of the host's launch work)
+// over 51 shapes: the CodeLlama-34B head shape at B = 1 and L = 512..128K,
+// B = 2..32 at L = 2K..64K, G = 4, the varlen, paged and peaked workloads,
+// bf16 and fp8 caches.  The pick is the fastest measured split count or
+// within 4 % of it, except varlen fp8 (9 %); the mean regret is 1 %.
+//
+// A CTA streams its tokens at a rate of its own (the tile loop's latency,
+// independent of the element type), unless the device's HBM bandwidth,
+// shared by the CTAs in flight, is lower:
+//   kHbmGBs            streaming rate of the whole device
+//   kCtaTokPerUs       tokens per microsecond of one CTA (any residency)
+//   kCtaPagedTokPerUs  the same alone on an SM when pages hold fewer than 64
+//                      tokens (one TMA box per page instead of one per tile)
+//   kCtaFixedUs        per-CTA fixed cost within a wave
+//   kCombineUs         device time added by a call with several splits (the
+//                      combine kernel after its dependency) ...
+//   kCombinePer16Us    ... plus this per 16 splits merged
 struct PlanModel {
-  static constexpr double kHbmGBs = 6500.0;
-  static constexpr double kCtaGBs = 50.0;
-  static constexpr double kCtaPagedGBs = 45.0;
-  static constexpr double kSmPairGBs = 54.0;
-  static constexpr double kCtaFixedUs = 0.2;
-  static constexpr double kCombineUs = 0.5;
+  static constexpr double kHbmGBs = 6800.0;
+  static constexpr double kCtaTokPerUs = 100.0;
+  static constexpr double kCtaPagedTokPerUs = 60.0;
+  static constexpr double kCtaFixedUs = 0.5;
+  static constexpr double kCombineUs = 1.5;
+  static constexpr double kCombinePer16Us = 1.5;
 };
 
 int tile_round_up(long long x) {
@@ -60,50 +67,53 @@ int effective_splits(int max_len, int chunk) {
   return static_cast<int>((static_cast<long long>(max_len) + chunk - 1) / chunk);
 }
 
-// Time of one wave of k equal CTAs of cta_bytes each.  CTAs are spread over
+// What the model needs to know of a problem besides its lengths.
+struct PlanShape {
+  int num_sms;
+  int Hkv;
+  double token_bytes;  // K + V bytes of one token of one KV head
+  bool small_pages;    // pages of fewer than 64 tokens
+};
+
+// Time of one wave of k CTAs of `tokens` tokens each.  CTAs are spread over
 // the SMs first one per SM, then two per SM.
-double wave_time_us(double cta_bytes, double k, int num_sms, double solo_gbs) {
-  const double share = PlanModel::kHbmGBs / k;
-  const double limit = k <= num_sms ? solo_gbs : PlanModel::kSmPairGBs / 2.0;
-  return cta_bytes / (std::min(share, limit) * 1e3) + PlanModel::kCtaFixedUs;
+double wave_time_us(const PlanShape& ps, double tokens, double k) {
+  const double hbm_tok = PlanModel::kHbmGBs * 1e3 / (k * ps.token_bytes);
+  const double own = (k <= ps.num_sms && ps.small_pages) ? PlanModel::kCtaPagedTokPerUs
+                                                          : PlanModel::kCtaTokPerUs;
+  return tokens / std::min(hbm_tok, own) + PlanModel::kCtaFixedUs;
 }
 
-// Time of one call whose split kernel runs n_ctas non-empty CTAs moving
-// bytes_total bytes, the largest CTA moving max_cta bytes.  The larger of two
-// estimates: waves of CTAs of the mean size, and the largest CTA on its own
-// (which decides the end when lengths differ).
-double model_time_us(int num_sms, int block_size, double n_ctas, double bytes_total,
-                     double max_cta, int s_eff) {
+// Time of one call whose split kernel runs n_ctas non-empty CTAs over
+// `tokens` KV-head tokens, the largest CTA holding max_cta of them.  The
+// larger of two estimates: waves of CTAs of the mean size, and the largest
+// CTA on its own (which decides the end when lengths differ).
+double model_time_us(const PlanShape& ps, double n_ctas, double tokens, double max_cta,
+                     int s_eff) {
   if (n_ctas <= 0) return PlanModel::kCtaFixedUs;
-  const double slots = static_cast<double>(num_sms) * fd::kCtasPerSm;
-  const double solo = (block_size > 0 && block_size < fd::kTile) ? PlanModel::kCtaPagedGBs
-                                                                 : PlanModel::kCtaGBs;
-  const double mean = bytes_total / n_ctas;
+  const double slots = static_cast<double>(ps.num_sms) * fd::kCtasPerSm;
+  const double mean = tokens / n_ctas;
   const double full_waves = std::floor(n_ctas / slots);
   const double rem = n_ctas - full_waves * slots;
   double waves = 0.0;
-  if (full_waves > 0) waves += full_waves * wave_time_us(mean, slots, num_sms, solo);
-  if (rem > 0) waves += wave_time_us(mean, rem, num_sms, solo);
-  const double longest = wave_time_us(max_cta, std::min(n_ctas, slots), num_sms, solo);
+  if (full_waves > 0) waves += full_waves * wave_time_us(ps, mean, slots);
+  if (rem > 0) waves += wave_time_us(ps, mean, rem);
+  const double longest = wave_time_us(ps, max_cta, std::min(n_ctas, slots));
   double t = std::max(waves, longest);
-  if (s_eff > 1) t += PlanModel::kCombineUs;
+  if (s_eff > 1) t += PlanModel::kCombineUs + PlanModel::kCombinePer16Us * std::ceil(s_eff / 16.0);
   return t;
 }
 
 // The model for a batch whose sequences all hold max_len tokens.
-double model_time_uniform(int num_sms, int B, int Hkv, int D, int max_len, int block_size,
-                          int S) {
+double model_time_uniform(const PlanShape& ps, int B, int max_len, int S) {
   const int chunk = chunk_for(max_len, S);
   const int s_eff = effective_splits(max_len, chunk);
-  const double units = static_cast<double>(B) * Hkv;
-  const double bytes = units * max_len * D * 4.0;
-  const double max_cta = std::min<double>(chunk, max_len) * D * 4.0;
-  return model_time_us(num_sms, block_size, units * s_eff, bytes, max_cta, s_eff);
+  const double units = static_cast<double>(B) * ps.Hkv;
+  return model_time_us(ps, units * s_eff, units * max_len, std::min(chunk, max_len), s_eff);
 }
 
 // The model for given per-sequence lengths (clamped to [0, max_len]).
-double model_time_lengths(int num_sms, int B, int Hkv, int D, int max_len, int block_size,
-                          const int32_t* lens, int S) {
+double model_time_lengths(const PlanShape& ps, int B, int max_len, const int32_t* lens, int S) {
   const int chunk = chunk_for(max_len, S);
   const int s_eff = effective_splits(max_len, chunk);
   double n_ctas = 0.0, tokens = 0.0, max_tok = 0.0;
@@ -113,8 +123,7 @@ double model_time_lengths(int num_sms, int B, int Hkv, int D, int max_len, int b
     tokens += n;
     max_tok = std::max(max_tok, std::min<double>(n, chunk));
   }
-  return model_time_us(num_sms, block_size, n_ctas * Hkv, tokens * Hkv * D * 4.0,
-                       max_tok * D * 4.0, s_eff);
+  return model_time_us(ps, n_ctas * ps.Hkv, tokens * ps.Hkv, max_tok, s_eff);
 }
 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
@@ -458,6 +467,10 @@ fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
   a.n_splits = n_splits;
   a.scale_log2 = scale * (fp8 ? p->k_scale : 1.f) * 1.4426950408889634074f;
   a.v_scale = fp8 ? p->v_scale : 1.f;
+  // L2 prefetch ahead of the wait on the previous grid (contiguous caches):
+  // half the split's tiles, at most kPrefetchTiles.  Swept on B200 over
+  // 0..12 tiles at 4K..64K tokens, bf16 and fp8, S = 16 and 32.
+  a.prefetch_tiles = paged ? 0 : std::min(kPrefetchTiles, std::max(1, chunk / fd::kTile / 2));
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   fd_status r;
@@ -471,6 +484,21 @@ fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
     r = paged ? dispatch_split<64, true>(G, tk, tv, a, n_splits, Hkv, B, s)
               : dispatch_split<64, false>(G, tk, tv, a, n_splits, Hkv, B, s);
   return r;
+}
+
+// The planner over every input it uses.  elem_bytes: bytes of one cache
+// element; seqlens: host lengths or null (every sequence holds max_len).
+int plan_impl(int num_sms, int B, int Hkv, int D, int max_len, int block_size, int elem_bytes,
+              const int32_t* seqlens) {
+  // Two CTAs per slot from the batch alone: no split (this also bounds the
+  // planning cost for large batches).
+  if (static_cast<long long>(B) * Hkv >= 2LL * num_sms * fd::kCtasPerSm) return 1;
+  const PlanShape ps{num_sms, Hkv, 2.0 * D * elem_bytes, block_size > 0 && block_size < fd::kTile};
+  if (seqlens)
+    return pick_splits(max_len, [&](int S) {
+      return model_time_lengths(ps, B, max_len, seqlens, S);
+    });
+  return pick_splits(max_len, [&](int S) { return model_time_uniform(ps, B, max_len, S); });
 }
 
 }  // namespace
@@ -498,11 +526,7 @@ int fd_plan_sm(int num_sms, int B, int Hq, int Hkv, int D, int max_len, int bloc
   if (num_sms < 1) return FD_ERR_INVALID_ARGUMENT;
   const fd_status st = check_shape(B, Hq, Hkv, D, max_len, block_size);
   if (st != FD_OK) return st;
-  // Enough (sequence, KV head) units to fill every CTA slot: no split.
-  if (static_cast<long long>(B) * Hkv >= static_cast<long long>(num_sms) * fd::kCtasPerSm) return 1;
-  return pick_splits(max_len, [&](int S) {
-    return model_time_uniform(num_sms, B, Hkv, D, max_len, block_size, S);
-  });
+  return plan_impl(num_sms, B, Hkv, D, max_len, block_size, 2, nullptr);
 }
 
 int fd_plan_seqlens(int num_sms, int B, int Hq, int Hkv, int D, int max_len, int block_size,
@@ -514,9 +538,21 @@ int fd_plan_seqlens(int num_sms, int B, int Hq, int Hkv, int D, int max_len, int
     int dev = 0;
     if (current_device(&dev) != FD_OK || device_sms(dev, &num_sms) != FD_OK) return FD_ERR_CUDA;
   }
-  return pick_splits(max_len, [&](int S) {
-    return model_time_lengths(num_sms, B, Hkv, D, max_len, block_size, seqlens, S);
-  });
+  return plan_impl(num_sms, B, Hkv, D, max_len, block_size, 2, seqlens);
+}
+
+int fd_plan_problem(int num_sms, const fd_problem* p, const int32_t* seqlens) {
+  if (!p) return FD_ERR_INVALID_ARGUMENT;
+  const fd_status st = check_shape(p->B, p->Hq, p->Hkv, p->D, p->max_len, p->block_size);
+  if (st != FD_OK) return st;
+  if (p->kv_dtype != FD_KV_BF16 && p->kv_dtype != FD_KV_FP8_E4M3) return FD_ERR_INVALID_ARGUMENT;
+  if (p->kv_dtype == FD_KV_FP8_E4M3 && p->D != 128) return FD_ERR_UNSUPPORTED;
+  if (num_sms < 1) {
+    int dev = 0;
+    if (current_device(&dev) != FD_OK || device_sms(dev, &num_sms) != FD_OK) return FD_ERR_CUDA;
+  }
+  return plan_impl(num_sms, p->B, p->Hkv, p->D, p->max_len, p->block_size,
+                   p->kv_dtype == FD_KV_FP8_E4M3 ? 1 : 2, seqlens);
 }
 
 int fd_plan(int B, int Hq, int Hkv, int D, int max_len, int block_size) {

@@ -64,6 +64,8 @@ struct SplitArgs {
   int n_splits;                 // effective split count = gridDim.x
   float scale_log2;             // scale * k_scale * log2(e)
   float v_scale;                // dequantisation scale of an fp8 V cache (1 for bf16)
+  int prefetch_tiles;           // contiguous caches: tiles per CTA prefetched into L2 before
+                                // the wait on the previous grid (0 = none)
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -578,6 +580,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
   }
+  if constexpr (!PAGED) {
+    // While the previous grid finishes, pull the first tiles of this split
+    // into L2, one tile per lane.  Only kernel arguments are used (the
+    // lengths may still be in flight), so the range stops at max_len.
+    if (warp == kConsumerWarps && lane < a.prefetch_tiles) {
+      const int t0 = split * a.chunk + lane * kTile;
+      if (lane * kTile < a.chunk && t0 < a.max_len) {
+        tma_prefetch_l2_5d(&tmK, 0, kvh, t0, 0, b);
+        tma_prefetch_l2_5d(&tmV, 0, kvh, t0, 0, b);
+      }
+    }
+  }
   __syncthreads();
 
   // Inputs may be produced by the previous kernel on the stream.
@@ -696,7 +710,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 template <int D>
 __global__ void __launch_bounds__(128) fd_combine_kernel(const SplitArgs a, int B) {
   grid_dependency_wait();     // partials come from the split kernel
-  grid_dependents_launch();   // the next call's split kernel may start its prologue
+  // The next call's split kernel may now start its prologue, which pulls its
+  // first tiles into L2 while this kernel merges.  (Triggering before the
+  // wait lets it become resident while the split kernel still streams; its
+  // prefetched tiles then sit in L2 for the whole split and were measured to
+  // be evicted and read twice at 16K tokens.)
+  grid_dependents_launch();
   const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= B * a.Hq) return;

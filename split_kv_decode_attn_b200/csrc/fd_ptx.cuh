@@ -91,6 +91,17 @@ __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* tm,
       : "memory");
 }
 
+// Prefetch a 5-D box into L2 (no shared-memory destination, no completion).
+// L2 is the device's point of coherence, so this is safe ahead of the wait
+// on the previous grid: a later load still sees that grid's writes.
+__device__ __forceinline__ void tma_prefetch_l2_5d(const CUtensorMap* tm, int c0, int c1, int c2,
+                                                   int c3, int c4) {
+  asm volatile("cp.async.bulk.prefetch.tensor.5d.L2.global.tile [%0, {%1, %2, %3, %4, %5}];"
+               ::"l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+               "r"(c4)
+               : "memory");
+}
+
 // ---- warp-level tensor-core fragments ---------------------------------------
 
 __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1,

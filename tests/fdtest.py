@@ -68,14 +68,9 @@ class OnDevice:
                                w.v_scale)
 
     def plan(self) -> int:
-        """The split count the benchmark uses: the length-aware planner when
-        the lengths are known, else fd_plan."""
-        w = self.w
-        if w.seqlens is not None:
-            s = fd.fd_plan_seqlens(0, w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size,
-                                   w.seqlens)
-        else:
-            s = fd.fd_plan(w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size)
+        """The split count the benchmark uses: fd_plan_problem over the whole
+        problem, with the lengths when they are known."""
+        s = fd.fd_plan_problem(0, self.problem(), self.w.seqlens)
         assert s >= 1, fd.fd_status_string(s)
         return s
 

@@ -68,8 +68,9 @@ B200_SMS = 148
 
 
 def test_plan_large_batch_does_not_split():
-    # B*Hkv = 256 + 64 units >= 2 CTAs per SM on 148 SMs: enough work already
-    assert fd.fd_plan_sm(B200_SMS, 40, 32, 8, 128, 32768, 0) == 1
+    # B*Hkv = 640 units >= two CTAs per slot (2 per SM on 148 SMs): enough work
+    assert fd.fd_plan_sm(B200_SMS, 80, 32, 8, 128, 32768, 0) == 1
+    assert fd.fd_plan_sm(B200_SMS, 256, 64, 8, 128, 8192, 0) == 1
 
 
 def test_plan_short_history_does_not_split():
@@ -88,25 +89,67 @@ def test_plan_long_history_fills_the_device():
         assert ctas <= 4 * 2 * B200_SMS, (L, S, ctas)
 
 
-# Split counts that were fastest, or within 6 %, in device-time sweeps
-# measured on B200 (the planner's constants were fitted to those sweeps).
+# Split counts that were fastest, or within 5 %, in device-time sweeps
+# measured on B200 from CUDA-graph replays (the planner's constants were fitted
+# to those sweeps; summary and command in the planner profile under profiles/).
+# shape: (B, Hq, Hkv, D, max_len, block_size), bf16 cache.
 @pytest.mark.parametrize("shape,good", [
-    ((1, 64, 8, 128, 512, 0), {4, 8}),          # 8 units: even 8 tiles pay to split
-    ((4, 64, 8, 128, 512, 0), {1, 4}),
-    ((1, 64, 8, 128, 2048, 0), {16, 24}),
-    ((1, 64, 8, 128, 8192, 0), {12, 16, 18}),
-    ((1, 64, 8, 128, 16384, 0), {16, 18, 20}),
-    ((1, 64, 8, 128, 32768, 0), {16, 18, 24}),
-    ((1, 64, 8, 128, 65536, 0), {16, 18, 24}),
-    ((4, 64, 8, 128, 16384, 0), {4, 8}),
-    ((16, 64, 8, 128, 2048, 0), {1}),           # large batch: no split
-    ((16, 64, 8, 128, 65536, 0), {1, 4, 8}),
-    ((64, 64, 8, 128, 8192, 0), {1}),
-    ((8, 32, 8, 128, 131072, 16), {4, 18}),
-    ((1, 32, 8, 128, 262144, 0), {16, 18, 24, 32}),
+    ((1, 64, 8, 128, 512, 0), {8}),             # 8 units: even 8 tiles pay to split
+    ((1, 64, 8, 128, 2048, 0), {16, 20, 24, 28}),
+    ((1, 64, 8, 128, 4096, 0), {16, 20}),
+    ((1, 64, 8, 128, 8192, 0), {16, 28}),
+    ((1, 64, 8, 128, 16384, 0), {16}),
+    ((1, 64, 8, 128, 32768, 0), {16, 24, 28, 32}),
+    ((1, 64, 8, 128, 65536, 0), {16, 20, 24, 28, 32}),
+    ((1, 32, 8, 128, 16384, 0), {16}),
+    ((2, 64, 8, 128, 2048, 0), {8}),
+    ((4, 64, 8, 128, 8192, 0), {4, 6, 8}),
+    ((4, 64, 8, 128, 16384, 0), {4, 6, 8, 16}),
+    ((8, 64, 8, 128, 8192, 0), {2, 3, 4, 8}),
+    ((16, 64, 8, 128, 2048, 0), {1, 2}),        # large batch: little or no split
+    ((16, 64, 8, 128, 16384, 0), {1, 2, 4, 6, 8}),
+    ((32, 64, 8, 128, 2048, 0), {1}),
+    ((8, 32, 8, 128, 131072, 16), {3, 4, 8}),
+    ((1, 32, 8, 128, 262144, 0), {16, 17, 20, 24, 32, 64}),
 ])
 def test_plan_matches_measured_sweeps(shape, good):
     assert fd.fd_plan_sm(B200_SMS, *shape) in good
+    # fd_plan_problem on a bf16 problem is the same planner
+    B, Hq, Hkv, D, L, bs = shape
+    prob = fd.make_problem(B, Hq, Hkv, D, L, bs, 1 if bs else 0, L // bs if bs else 0)
+    assert fd.fd_plan_problem(B200_SMS, prob) == fd.fd_plan_sm(B200_SMS, *shape)
+
+
+# The same for fp8 E4M3 caches: an fp8 CTA streams tokens at the bf16 rate,
+# half the bytes, so the fastest split counts put more CTAs in flight.
+@pytest.mark.parametrize("shape,good", [
+    ((1, 64, 8, 128, 4096), {16, 20}),
+    ((1, 64, 8, 128, 16384), {16, 32, 40}),
+    ((1, 64, 8, 128, 32768), {32}),
+    ((1, 64, 8, 128, 65536), {32}),
+    ((1, 64, 8, 128, 131072), {32}),
+    ((4, 64, 8, 128, 16384), {8}),
+    ((16, 64, 8, 128, 8192), {2}),              # 128 units: fp8 still wants 2 CTAs per SM
+    ((16, 64, 8, 128, 16384), {2, 4, 8}),
+])
+def test_plan_problem_fp8_matches_measured_sweeps(shape, good):
+    prob = fd.make_problem(*shape, kv_dtype=fd.FD_KV_FP8_E4M3)
+    assert fd.fd_plan_problem(B200_SMS, prob) in good
+
+
+def test_plan_problem_checks_and_lengths():
+    lib = fd.load_library()
+    assert lib.fd_plan_problem(B200_SMS, None, None) == fd.FD_ERR_INVALID_ARGUMENT
+    bad = fd.make_problem(1, 8, 8, 64, 100, kv_dtype=fd.FD_KV_FP8_E4M3)
+    assert fd.fd_plan_problem(B200_SMS, bad) == fd.FD_ERR_UNSUPPORTED
+    assert fd.fd_plan_problem(B200_SMS, fd.make_problem(1, 8, 8, 128, 100, kv_dtype=5)) == \
+        fd.FD_ERR_INVALID_ARGUMENT
+    assert fd.fd_plan_problem(B200_SMS, fd.make_problem(1, 6, 4, 128, 100)) == \
+        fd.FD_ERR_INVALID_ARGUMENT
+    lens = [30000, 1200, 7, 0]
+    prob = fd.make_problem(4, 32, 8, 128, 32768)
+    assert fd.fd_plan_problem(B200_SMS, prob, lens) == \
+        fd.fd_plan_seqlens(B200_SMS, 4, 32, 8, 128, 32768, 0, lens)
 
 
 def test_plan_splits_grow_with_length_and_are_deterministic():
