@@ -441,6 +441,10 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
     if (lane == 0) mbar_arrive(bar_empty + 8 * s);
   }
 
+  // The combine kernel (or the next call) may launch once every CTA is past
+  // its tile loop: launched at the start it sat resident through the whole
+  // split and measured 0.4-1.4 us slower per call.
+  grid_dependents_launch();
   if (failed) {
     if (lane == 0) {
       raise_device_error(1u);
@@ -456,8 +460,6 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1)
         l_run[nb][j] += __shfl_xor_sync(0xffffffffu, l_run[nb][j], off);
-
-  // Every consumer warp is past its last shared-memory read of the pipeline.
 
   // Every consumer warp is past its last shared-memory read of the pipeline,
   // so the drained buffers hold the epilogue scratch.
@@ -596,7 +598,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
   // Inputs may be produced by the previous kernel on the stream.
   grid_dependency_wait();
-  grid_dependents_launch();
 
   const int n = seq_length(a.seqlens, b, a.max_len);
   const int start = split * a.chunk;
