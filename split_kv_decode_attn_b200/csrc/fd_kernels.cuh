@@ -178,9 +178,7 @@ struct SplitSmem {
   static constexpr int kRedAcc = 0;                                   // [warp][col][D]
   static constexpr int kRedM = kRedAcc + kConsumerWarps * kNcol * D;  // [warp][col]
   static constexpr int kRedL = kRedM + kConsumerWarps * kNcol;        // [warp][col]
-  static constexpr int kRedW = kRedL + kConsumerWarps * kNcol;        // [warp][col]
-  static constexpr int kSplitLse = kRedW + kConsumerWarps * kNcol;    // [col]: this split's lse
-  static constexpr int kScratchFloats = kSplitLse + kNcol;
+  static constexpr int kScratchFloats = kRedL + kConsumerWarps * kNcol;
   static_assert(kScratchFloats * 4 <= kBarOffset, "epilogue scratch must fit the pipeline buffers");
 };
 
@@ -462,9 +460,9 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
         l_run[nb][j] += __shfl_xor_sync(0xffffffffu, l_run[nb][j], off);
 
   // Every consumer warp is past its last shared-memory read of the pipeline,
-  // so the drained buffers hold the epilogue scratch.
+  // so the drained buffers hold the epilogue scratch: each warp's
+  // accumulator [warp][col][D] and its running max and sum per column.
   named_barrier_sync(1, kConsumerWarps * 32);
-  const int t = threadIdx.x;
   float* f = reinterpret_cast<float*>(smem);
   const bool live = !*cta_error;
   if (live) {
@@ -493,56 +491,81 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
     }
   }
   named_barrier_sync(1, kConsumerWarps * 32);
-  // Per head: the weight of each warp's state and this split's lse.
-  if (live && t < a.G) {
+  if (!live) return;
+
+  // One pass with no further barrier.  Each thread merges the four warp
+  // states for 8 head-dim entries of one head (4 at d0 and 4 at d0 + D/2, so
+  // that a warp's 16-byte reads and writes are contiguous) and computes that
+  // head's weights itself from a few broadcast reads.  (A separate per-head
+  // pass behind two more barriers took about 1.5 us per CTA.)
+  constexpr int kChunks = D / 8;  // chunks of 8 entries per head
+  const bool direct = n_parts == 1;
+  for (int c = threadIdx.x; c < a.G * kChunks; c += kConsumerWarps * 32) {
+    const int g = c / kChunks;
+    const int d0 = (c - g * kChunks) * 4;
     float mw[kConsumerWarps];
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) {
-      mw[w] = f[L::kRedM + w * NCOL + t];
+      mw[w] = f[L::kRedM + w * NCOL + g];
       M = fmaxf(M, mw[w]);
     }
+    float wt[kConsumerWarps];
+    float lse_s = -INFINITY;
     if (M == -INFINITY) {  // no token in this split
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) f[L::kRedW + w * NCOL + t] = 0.f;
-      f[L::kSplitLse + t] = -INFINITY;
+      for (int w = 0; w < kConsumerWarps; ++w) wt[w] = 0.f;
     } else {
-      float e[kConsumerWarps];
       float Ls = 0.f;
 #pragma unroll
       for (int w = 0; w < kConsumerWarps; ++w) {
-        e[w] = ex2(mw[w] - M);
-        Ls += e[w] * f[L::kRedL + w * NCOL + t];
+        wt[w] = ex2(mw[w] - M);
+        Ls += wt[w] * f[L::kRedL + w * NCOL + g];
       }
       const float inv = a.v_scale / Ls;  // an fp8 V cache is dequantised here
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) f[L::kRedW + w * NCOL + t] = e[w] * inv;
-      f[L::kSplitLse + t] = (M + log2f(Ls)) * 0.69314718055994530942f;
+      for (int w = 0; w < kConsumerWarps; ++w) wt[w] *= inv;
+      lse_s = (M + log2f(Ls)) * 0.69314718055994530942f;
     }
-  }
-  named_barrier_sync(1, kConsumerWarps * 32);
-  if (!live) return;
-
-  const bool direct = n_parts == 1;
-  for (int idx = t; idx < a.G * D; idx += kConsumerWarps * 32) {
-    const int g = idx / D, d = idx - (idx / D) * D;
-    float O = 0.f;
+    float4 o[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) {
-      float v = f[L::kRedAcc + (w * NCOL + g) * D + d];
-      if constexpr (MODE == kDup) v += f[L::kRedAcc + (w * NCOL + g + 4) * D + d];
-      O += f[L::kRedW + w * NCOL + g] * v;
+      const float* src = f + L::kRedAcc + (w * NCOL + g) * D + d0;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float4 v = *reinterpret_cast<const float4*>(src + h * (D / 2));
+        if constexpr (MODE == kDup) {  // columns g + 4 hold the bf16 residuals
+          const float4 r = *reinterpret_cast<const float4*>(src + 4 * D + h * (D / 2));
+          v.x += r.x;
+          v.y += r.y;
+          v.z += r.z;
+          v.w += r.w;
+        }
+        o[h].x += wt[w] * v.x;
+        o[h].y += wt[w] * v.y;
+        o[h].z += wt[w] * v.z;
+        o[h].w += wt[w] * v.w;
+      }
     }
     const size_t row = static_cast<size_t>(b) * a.Hq + h0 + g;
     if (direct) {
-      if (a.out_f32)
-        a.out_f32[row * D + d] = O;
-      else
-        a.out[row * D + d] = __float2bfloat16_rn(O);
-      if (d == 0 && a.lse) a.lse[row] = f[L::kSplitLse + g];
+      if (a.out_f32) {
+        float* dst = a.out_f32 + row * D + d0;
+        *reinterpret_cast<float4*>(dst) = o[0];
+        *reinterpret_cast<float4*>(dst + D / 2) = o[1];
+      } else {
+        __nv_bfloat16* dst = a.out + row * D + d0;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          *reinterpret_cast<uint2*>(dst + h * (D / 2)) =
+              make_uint2(pack_bf16x2(o[h].x, o[h].y), pack_bf16x2(o[h].z, o[h].w));
+      }
+      if (d0 == 0 && a.lse) a.lse[row] = lse_s;
     } else {
-      a.part_o[(row * a.n_splits + split) * D + d] = O;
-      if (d == 0) a.part_lse[row * a.n_splits + split] = f[L::kSplitLse + g];
+      float* dst = a.part_o + (row * a.n_splits + split) * D + d0;
+      *reinterpret_cast<float4*>(dst) = o[0];
+      *reinterpret_cast<float4*>(dst + D / 2) = o[1];
+      if (d0 == 0) a.part_lse[row * a.n_splits + split] = lse_s;
     }
   }
 }
