@@ -370,23 +370,37 @@ def cpu_baseline(w, seconds):
     """The fp64 oracle, as it stands, on this host's cores: one sequence per
     oracle call (all its query heads, threads over heads), cycling through
     the batch until `seconds` of wall time have passed.  GB/s of algorithmic
-    K+V bytes."""
+    K+V bytes.  Then the same on one thread for a third of that time, over a
+    window of each history sized to fit it."""
     cores = os.cpu_count() or 1
     threads = min(cores, w.Hq if w.kv_dtype == "bf16" else w.Hkv)
     lengths = w.lengths()
-    t0 = time.perf_counter()
-    done = 0
-    calls = 0
-    while True:
-        b = calls % w.B
-        done += oracle_sequence(w, b, 0, int(lengths[b]), threads)
-        calls += 1
-        if time.perf_counter() - t0 >= seconds:
-            break
-    dt = time.perf_counter() - t0
+
+    def run(nthreads, limit, window):
+        t0 = time.perf_counter()
+        done = 0
+        calls = 0
+        while True:
+            b = calls % w.B
+            done += oracle_sequence(w, b, 0, min(window, int(lengths[b])), nthreads)
+            calls += 1
+            if time.perf_counter() - t0 >= limit:
+                break
+        return done, calls, time.perf_counter() - t0
+
+    done, calls, dt = run(threads, seconds, int(lengths.max()))
+    t1 = time.perf_counter()
+    oracle_sequence(w, 0, 0, min(1024, int(lengths[0])), 1)
+    per_tok = (time.perf_counter() - t1) / max(min(1024, int(lengths[0])), 1)
+    window = int(max(64, min(int(lengths.max()), seconds / 3 / 4 / max(per_tok, 1e-9))))
+    done1, calls1, dt1 = run(1, seconds / 3, window)
     return {"value": round(done / dt / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "hardware_threads": cores,
             "sample": f"{calls} oracle calls, each one whole sequence of the workload "
-                      f"({w.Hq} query heads over its full history), {dt:.1f} s wall"}
+                      f"({w.Hq} query heads over its full history), {dt:.1f} s wall",
+            "single_thread": {"value": round(done1 / dt1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                              "sample": f"{calls1} oracle calls over the first {window} tokens "
+                                        f"of a sequence, {dt1:.1f} s wall"}}
 
 
 def run_fd(args):

@@ -126,9 +126,15 @@ __device__ __forceinline__ void combine_row(const float* po, const float* pl, in
   };
   load_batch(0);
   float mx = -INFINITY;
-  for (int s = lane; s < n_parts; s += 32) mx = fmaxf(mx, __ldcg(pl + s * l_stride));
+  if (n_parts <= BATCH) {  // every lane holds all the lse values already
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    for (int j = 0; j < BATCH; ++j)
+      if (j < n_parts) mx = fmaxf(mx, lb[j]);
+  } else {
+    for (int s = lane; s < n_parts; s += 32) mx = fmaxf(mx, __ldcg(pl + s * l_stride));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  }
   float acc[VPL];
 #pragma unroll
   for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
@@ -733,6 +739,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
 template <int D>
 __global__ void __launch_bounds__(128) fd_combine_kernel(const SplitArgs a, int B) {
+  const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  // The lengths may be read before the wait: the split kernel, the grid this
+  // one depends on, does not write them, and this grid launches only after
+  // every split CTA passed its own wait, i.e. after all earlier writes to
+  // them completed.  Read through L2 (coherent), not L1.
+  int n = 0;
+  if (row < B * a.Hq) {
+    n = a.seqlens ? __ldcg(a.seqlens + row / a.Hq) : a.max_len;
+    n = n < 0 ? 0 : (n > a.max_len ? a.max_len : n);
+  }
   grid_dependency_wait();     // partials come from the split kernel
   // The next call's split kernel may now start its prologue, which pulls its
   // first tiles into L2 while this kernel merges.  (Triggering before the
@@ -740,11 +757,7 @@ __global__ void __launch_bounds__(128) fd_combine_kernel(const SplitArgs a, int 
   // prefetched tiles then sit in L2 for the whole split and were measured to
   // be evicted and read twice at 16K tokens.)
   grid_dependents_launch();
-  const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
   if (row >= B * a.Hq) return;
-  const int b = row / a.Hq;
-  const int n = seq_length(a.seqlens, b, a.max_len);
   const int n_parts = min((n + a.chunk - 1) / a.chunk, a.n_splits);
   if (n_parts <= 1) return;
   combine_row<D>(a.part_o + static_cast<size_t>(row) * a.n_splits * D,
