@@ -99,19 +99,19 @@ def measured_peak():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the device code (the kernels and their PTX helpers)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "split_kv_decode_attn_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in ("fd_kernels.cuh", "fd_ptx.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(workload: str):
+def ncu_traffic(workload: str, num_splits: int):
     """DRAM bytes (read + write) per launch of the split kernel, the dominant
     kernel, from the committed ncu summary, if it was taken on the current
-    kernel sources; else None."""
+    device code at the same split count; else None."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
@@ -119,7 +119,9 @@ def ncu_traffic(workload: str):
         if j.get("source_hash") != kernel_source_hash():
             return None
         entry = j.get("workloads", {}).get(workload)
-        return None if entry is None else float(entry["split_kernel_bytes"])
+        if entry is None or int(entry["num_splits"]) != num_splits:
+            return None
+        return float(entry["split_kernel_bytes"])
     except Exception:
         return None
 
@@ -457,7 +459,7 @@ def run_fd(args):
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                      "frac_of_spec_8tbs": round(achieved / SPEC_HBM_GBS, 4),
-                     "traffic": ncu_traffic(w.name), "traffic_kernel": "fd_split_kernel",
+                     "traffic": ncu_traffic(w.name, call.S), "traffic_kernel": "fd_split_kernel",
                      "algorithmic_bytes": kvb},
         "gpu_launches": args.steps * call.launches_per_call,
         "clocks": clocks,

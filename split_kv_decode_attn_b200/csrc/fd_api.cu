@@ -25,31 +25,34 @@ constexpr int kMaxDevices = 64;
 // ---------------------------------------------------------------- planner
 
 // Cost model of one call, in microseconds, used to pick the split count.
-// It models device time: the constants were fitted to split-count sweeps
+// It models device time: the constants were fitted to a split-count sweep
 // measured on B200 from CUDA-graph replays (free of the host's launch work)
-// over 51 shapes: the CodeLlama-34B head shape at B = 1 and L = 512..128K,
-// B = 2..32 at L = 2K..64K, G = 4, the varlen, paged and peaked workloads,
+// over 54 shapes: the CodeLlama-34B head shape at B = 1 and L = 512..128K,
+// B = 2..40 at L = 2K..64K, G = 4, the varlen, paged and peaked workloads,
 // bf16 and fp8 caches.  The pick is the fastest measured split count or
-// within 4 % of it, except varlen fp8 (9 %); the mean regret is 1 %.
+// within 5.5 % of it; the mean regret is 0.5 %.
 //
 // A CTA streams its tokens at a rate of its own (the tile loop's latency,
 // independent of the element type), unless the device's HBM bandwidth,
 // shared by the CTAs in flight, is lower:
 //   kHbmGBs            streaming rate of the whole device
-//   kCtaTokPerUs       tokens per microsecond of one CTA (any residency)
-//   kCtaPagedTokPerUs  the same alone on an SM when pages hold fewer than 64
-//                      tokens (one TMA box per page instead of one per tile)
+//   kCtaTokPerUs       tokens per microsecond of one CTA
+//   kCtaDeepTokPerUs   the same for a bf16 D = 128 grid of at most one CTA
+//                      per SM, which runs the deeper ring
+//   kCtaPagedTokPerUs  alone on an SM when pages hold fewer than 64 tokens
+//                      (one TMA box per page instead of one per tile)
 //   kCtaFixedUs        per-CTA fixed cost within a wave
 //   kCombineUs         device time added by a call with several splits (the
 //                      combine kernel after its dependency) ...
 //   kCombinePer16Us    ... plus this per 16 splits merged
 struct PlanModel {
-  static constexpr double kHbmGBs = 6800.0;
-  static constexpr double kCtaTokPerUs = 100.0;
-  static constexpr double kCtaPagedTokPerUs = 60.0;
-  static constexpr double kCtaFixedUs = 0.5;
-  static constexpr double kCombineUs = 1.5;
-  static constexpr double kCombinePer16Us = 1.5;
+  static constexpr double kHbmGBs = 6500.0;
+  static constexpr double kCtaTokPerUs = 90.0;
+  static constexpr double kCtaDeepTokPerUs = 100.0;
+  static constexpr double kCtaPagedTokPerUs = 50.0;
+  static constexpr double kCtaFixedUs = 0.3;
+  static constexpr double kCombineUs = 1.0;
+  static constexpr double kCombinePer16Us = 2.0;
 };
 
 int tile_round_up(long long x) {
@@ -70,17 +73,20 @@ int effective_splits(int max_len, int chunk) {
 // What the model needs to know of a problem besides its lengths.
 struct PlanShape {
   int num_sms;
+  int B;
   int Hkv;
   double token_bytes;  // K + V bytes of one token of one KV head
   bool small_pages;    // pages of fewer than 64 tokens
+  bool deep_ring;      // bf16, D = 128: a grid of <= num_sms CTAs gets the deep ring
 };
 
-// Time of one wave of k CTAs of `tokens` tokens each.  CTAs are spread over
-// the SMs first one per SM, then two per SM.
-double wave_time_us(const PlanShape& ps, double tokens, double k) {
+// Time of one wave of k CTAs of `tokens` tokens each, in a grid of
+// `grid` CTAs.  CTAs are spread over the SMs first one per SM, then two.
+double wave_time_us(const PlanShape& ps, double tokens, double k, double grid) {
   const double hbm_tok = PlanModel::kHbmGBs * 1e3 / (k * ps.token_bytes);
-  const double own = (k <= ps.num_sms && ps.small_pages) ? PlanModel::kCtaPagedTokPerUs
-                                                          : PlanModel::kCtaTokPerUs;
+  double own = PlanModel::kCtaTokPerUs;
+  if (k <= ps.num_sms && ps.small_pages) own = PlanModel::kCtaPagedTokPerUs;
+  else if (ps.deep_ring && grid <= ps.num_sms) own = PlanModel::kCtaDeepTokPerUs;
   return tokens / std::min(hbm_tok, own) + PlanModel::kCtaFixedUs;
 }
 
@@ -92,13 +98,14 @@ double model_time_us(const PlanShape& ps, double n_ctas, double tokens, double m
                      int s_eff) {
   if (n_ctas <= 0) return PlanModel::kCtaFixedUs;
   const double slots = static_cast<double>(ps.num_sms) * fd::kCtasPerSm;
+  const double grid = static_cast<double>(ps.B) * ps.Hkv * s_eff;
   const double mean = tokens / n_ctas;
   const double full_waves = std::floor(n_ctas / slots);
   const double rem = n_ctas - full_waves * slots;
   double waves = 0.0;
-  if (full_waves > 0) waves += full_waves * wave_time_us(ps, mean, slots);
-  if (rem > 0) waves += wave_time_us(ps, mean, rem);
-  const double longest = wave_time_us(ps, max_cta, std::min(n_ctas, slots));
+  if (full_waves > 0) waves += full_waves * wave_time_us(ps, mean, slots, grid);
+  if (rem > 0) waves += wave_time_us(ps, mean, rem, grid);
+  const double longest = wave_time_us(ps, max_cta, std::min(n_ctas, slots), grid);
   double t = std::max(waves, longest);
   if (s_eff > 1) t += PlanModel::kCombineUs + PlanModel::kCombinePer16Us * std::ceil(s_eff / 16.0);
   return t;
@@ -513,7 +520,8 @@ int plan_impl(int num_sms, int B, int Hkv, int D, int max_len, int block_size, i
   // Two CTAs per slot from the batch alone: no split (this also bounds the
   // planning cost for large batches).
   if (static_cast<long long>(B) * Hkv >= 2LL * num_sms * fd::kCtasPerSm) return 1;
-  const PlanShape ps{num_sms, Hkv, 2.0 * D * elem_bytes, block_size > 0 && block_size < fd::kTile};
+  const PlanShape ps{num_sms, B, Hkv, 2.0 * D * elem_bytes,
+                     block_size > 0 && block_size < fd::kTile, elem_bytes == 2 && D == 128};
   if (seqlens)
     return pick_splits(max_len, [&](int S) {
       return model_time_lengths(ps, B, max_len, seqlens, S);

@@ -181,8 +181,13 @@ struct SplitSmem {
   static constexpr int kDynamicBytes = kBytes + 1024;  // room to align to 1 KB
   // Epilogue scratch, laid over the drained pipeline buffers (floats):
   static constexpr int kNcol = NB * 8;
-  static constexpr int kRedAcc = 0;                                   // [warp][col][D]
-  static constexpr int kRedM = kRedAcc + kConsumerWarps * kNcol * D;  // [warp][col]
+  // Rows of D floats padded by 4: the accumulator writes of lanes in
+  // different column pairs then start in different banks.  (With two column
+  // blocks the kernel is at its register cap and the padding's index
+  // arithmetic spilled, so those rows stay unpadded.)
+  static constexpr int kAccStride = NB == 1 ? D + 4 : D;
+  static constexpr int kRedAcc = 0;                                   // [warp][col][kAccStride]
+  static constexpr int kRedM = kRedAcc + kConsumerWarps * kNcol * kAccStride;  // [warp][col]
   static constexpr int kRedL = kRedM + kConsumerWarps * kNcol;        // [warp][col]
   static constexpr int kScratchFloats = kRedL + kConsumerWarps * kNcol;
   static_assert(kScratchFloats * 4 <= kBarOffset, "epilogue scratch must fit the pipeline buffers");
@@ -475,7 +480,7 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
     const int j0 = 2 * (lane & 3);
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
-      float* base = f + L::kRedAcc + (warp * NCOL + nb * 8 + j0) * D;
+      float* base = f + L::kRedAcc + (warp * NCOL + nb * 8 + j0) * L::kAccStride;
       // Accumulator rows g and g + 8 of d-block db: head-dim entries
       // 16db + g and 16db + g + 8, or 16db + 2g and 16db + 2g + 1 on the fp8
       // path (its V fragments permute the rows).
@@ -484,9 +489,9 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
       for (int db = 0; db < DBLK; ++db) {
         const int d = db * 16 + (FP8 ? 2 : 1) * (lane >> 2);
         base[d] = acc[nb][db][0];
-        base[D + d] = acc[nb][db][1];
+        base[L::kAccStride + d] = acc[nb][db][1];
         base[d + dstep] = acc[nb][db][2];
-        base[D + d + dstep] = acc[nb][db][3];
+        base[L::kAccStride + d + dstep] = acc[nb][db][3];
       }
       if (lane < 4) {
         f[L::kRedM + warp * NCOL + nb * 8 + j0] = m_run[nb][0];
@@ -536,12 +541,12 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
     float4 o[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
 #pragma unroll
     for (int w = 0; w < kConsumerWarps; ++w) {
-      const float* src = f + L::kRedAcc + (w * NCOL + g) * D + d0;
+      const float* src = f + L::kRedAcc + (w * NCOL + g) * L::kAccStride + d0;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         float4 v = *reinterpret_cast<const float4*>(src + h * (D / 2));
         if constexpr (MODE == kDup) {  // columns g + 4 hold the bf16 residuals
-          const float4 r = *reinterpret_cast<const float4*>(src + 4 * D + h * (D / 2));
+          const float4 r = *reinterpret_cast<const float4*>(src + 4 * L::kAccStride + h * (D / 2));
           v.x += r.x;
           v.y += r.y;
           v.z += r.z;
