@@ -68,6 +68,12 @@ struct SplitArgs {
                                 // the wait on the previous grid (0 = none)
 };
 
+// Token of row s (0..15) of the fp8 score MMA within a warp's 16-token slice:
+// rows 2t, 2t+1 -> tokens 4t, 4t+1 and rows 8+2t, 8+2t+1 -> tokens 4t+2, 4t+3.
+__host__ __device__ constexpr uint32_t perm16(uint32_t s) {
+  return ((s & 7) >> 1) * 4 + (s >> 3) * 2 + (s & 1);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -261,16 +267,24 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
   // Row of the 16-token slice this lane addresses for ldmatrix, and its
   // 128-byte swizzle phase (row mod 8).  A tile is a stack of TMA boxes of
   // 2^log2_box_rows rows, each laid out [column half][row][128 bytes].
-  const uint32_t rowK = warp * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
-  const uint32_t rowV = warp * 16 + (lane >> 4) * 8 + (lane & 7);
-  const uint32_t x7 = lane & 7;
+  //
+  // FP8: row r of the score MMA is token perm16(r), so that after the P
+  // transpose the k-slots 2t, 2t+1 and 2t+8, 2t+9 of the P.V MMA are tokens
+  // 4t, 4t+1 and 4t+2, 4t+3: the order in which the byte-transposing
+  // ldmatrix delivers V (see ldmatrix_x2_trans_b8).
+  const uint32_t r16 = ((lane >> 3) & 1) * 8 + (lane & 7);
+  const uint32_t rowK = warp * 16 + (FP8 ? perm16(r16) : r16);
+  const uint32_t rowV = warp * 16 + (FP8 ? (lane & 15) : (lane >> 4) * 8 + (lane & 7));
+  const uint32_t x7 = lane & 7;              // swizzle phase of rowV (and of rowK if not FP8)
+  const uint32_t xk = rowK & 7;
   const uint32_t lgr = a.log2_box_rows;
   const uint32_t half_bytes = 128u << lgr;                    // one column half of a box
   const uint32_t box_bytes = half_bytes * L::kHalves;
   const uint32_t offK = (rowK >> lgr) * box_bytes + (rowK & ((1u << lgr) - 1)) * 128;
   const uint32_t offV = (rowV >> lgr) * box_bytes + (rowV & ((1u << lgr) - 1)) * 128;
-  const int r_lo = warp * 16 + (lane >> 2);   // token rows of the C fragment
-  const int r_hi = r_lo + 8;
+  // Token rows of the C fragment held by this lane.
+  const int r_lo = warp * 16 + (FP8 ? perm16(lane >> 2) : (lane >> 2));
+  const int r_hi = warp * 16 + (FP8 ? perm16((lane >> 2) + 8) : (lane >> 2) + 8);
   const float sl2 = a.scale_log2;
   bool failed = false;
 
@@ -302,7 +316,7 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
 #pragma unroll
       for (int kp = 0; kp < KSTEPS / 2; ++kp) {
         const uint32_t chunk16 = 2 * kp + (lane >> 4);
-        const uint32_t addr = kbase + offK + ((chunk16 ^ x7) << 4);
+        const uint32_t addr = kbase + offK + ((chunk16 ^ xk) << 4);
         uint32_t r[4];
         ldmatrix_x4(addr, r[0], r[1], r[2], r[3]);
 #pragma unroll
@@ -391,37 +405,44 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
       }
     }
 
-    // O^T += V^T P^T for this warp's 16 tokens.
+    // O^T += V^T P^T for this warp's 16 tokens.  Rows past the valid length
+    // may hold anything (NaN included): on a partial tile their V values are
+    // zeroed in registers so that 0 * NaN never reaches the accumulator.
     uint32_t vmask_lo = 0xffffffffu, vmask_hi = 0xffffffffu;
     if (partial) {
-      const int tk = warp * 16 + 2 * (lane & 3);
-      vmask_lo = (tk < tile_valid ? 0x0000ffffu : 0u) | (tk + 1 < tile_valid ? 0xffff0000u : 0u);
-      vmask_hi = (tk + 8 < tile_valid ? 0x0000ffffu : 0u) | (tk + 9 < tile_valid ? 0xffff0000u : 0u);
+      if constexpr (FP8) {  // bytes i of a register: token 4t + i
+        const int tk = warp * 16 + 4 * (lane & 3);
+        vmask_lo = (tk < tile_valid ? 0xffu : 0u) | (tk + 1 < tile_valid ? 0xff00u : 0u) |
+                   (tk + 2 < tile_valid ? 0xff0000u : 0u) | (tk + 3 < tile_valid ? 0xff000000u : 0u);
+      } else {
+        const int tk = warp * 16 + 2 * (lane & 3);
+        vmask_lo = (tk < tile_valid ? 0x0000ffffu : 0u) | (tk + 1 < tile_valid ? 0xffff0000u : 0u);
+        vmask_hi = (tk + 8 < tile_valid ? 0x0000ffffu : 0u) | (tk + 9 < tile_valid ? 0xffff0000u : 0u);
+      }
     }
     if constexpr (FP8) {
-      // ldmatrix.trans on the fp8 V tile, 16-bit units: a lane's register
-      // holds entries (16c + 2p, 16c + 2p + 1) of tokens 2t and 2t + 1
-      // (p = lane / 4, t = lane & 3).  Byte-permute to (token 2t, token 2t+1)
-      // pairs of one entry and convert: rows g (g < 8) of the A fragment hold
-      // entry 16c + 2g, rows g + 8 hold 16c + 2g + 1.
+      // The byte-transposing ldmatrix gives a lane, per 16-entry block,
+      // tokens 4t .. 4t+3 of entries g and g + 8: exactly the A fragment
+      // (rows g, g + 8; k-slots 2t, 2t+1 in the low halves, 2t+8, 2t+9 in the
+      // high halves) after one conversion per half.
 #pragma unroll
       for (int dp = 0; dp < DBLK / 2; ++dp) {
         const uint32_t chunk16 = 2 * dp + (lane >> 4);
-        const uint32_t addr = vbase + offK + ((chunk16 ^ x7) << 4);
+        const uint32_t addr = vbase + offV + ((chunk16 ^ x7) << 4);
         uint32_t r[4];
-        ldmatrix_x4_trans(addr, r[0], r[1], r[2], r[3]);
-        r[0] &= vmask_lo;
-        r[1] &= vmask_hi;
-        r[2] &= vmask_lo;
-        r[3] &= vmask_hi;
+        ldmatrix_x2_trans_b8(addr, r[0], r[1], r[2], r[3]);
+        if (partial) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) r[i] &= vmask_lo;
+        }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int db = 2 * dp + h;
           uint32_t vf[4];
-          vf[0] = e4m3x2_to_f16x2(__byte_perm(r[2 * h], 0, 0x0020));
-          vf[1] = e4m3x2_to_f16x2(__byte_perm(r[2 * h], 0, 0x0031));
-          vf[2] = e4m3x2_to_f16x2(__byte_perm(r[2 * h + 1], 0, 0x0020));
-          vf[3] = e4m3x2_to_f16x2(__byte_perm(r[2 * h + 1], 0, 0x0031));
+          vf[0] = e4m3x2_to_f16x2(r[2 * h]);
+          vf[1] = e4m3x2_to_f16x2(r[2 * h + 1]);
+          vf[2] = e4m3x2_to_f16x2(r[2 * h] >> 16);
+          vf[3] = e4m3x2_to_f16x2(r[2 * h + 1] >> 16);
 #pragma unroll
           for (int nb = 0; nb < NB; ++nb) mma_f16_16816(acc[nb][db], vf, pb[nb][0], pb[nb][1]);
         }
@@ -433,12 +454,12 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
       const uint32_t addr = vbase + offV + (db >> 2) * half_bytes + ((chunk16 ^ x7) << 4);
       uint32_t vf[4];
       ldmatrix_x4_trans(addr, vf[0], vf[1], vf[2], vf[3]);
-      // Rows past the valid length may hold anything (NaN included): zero them
-      // so that 0 * NaN never reaches the accumulator.
-      vf[0] &= vmask_lo;
-      vf[1] &= vmask_lo;
-      vf[2] &= vmask_hi;
-      vf[3] &= vmask_hi;
+      if (partial) {
+        vf[0] &= vmask_lo;
+        vf[1] &= vmask_lo;
+        vf[2] &= vmask_hi;
+        vf[3] &= vmask_hi;
+      }
 #pragma unroll
       for (int nb = 0; nb < NB; ++nb) {
         mma_bf16_16816(acc[nb][db], vf, pb[nb][0], pb[nb][1]);
@@ -482,16 +503,14 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
     for (int nb = 0; nb < NB; ++nb) {
       float* base = f + L::kRedAcc + (warp * NCOL + nb * 8 + j0) * L::kAccStride;
       // Accumulator rows g and g + 8 of d-block db: head-dim entries
-      // 16db + g and 16db + g + 8, or 16db + 2g and 16db + 2g + 1 on the fp8
-      // path (its V fragments permute the rows).
-      const int dstep = FP8 ? 1 : 8;
+      // 16db + g and 16db + g + 8.
 #pragma unroll
       for (int db = 0; db < DBLK; ++db) {
-        const int d = db * 16 + (FP8 ? 2 : 1) * (lane >> 2);
+        const int d = db * 16 + (lane >> 2);
         base[d] = acc[nb][db][0];
         base[L::kAccStride + d] = acc[nb][db][1];
-        base[d + dstep] = acc[nb][db][2];
-        base[L::kAccStride + d + dstep] = acc[nb][db][3];
+        base[d + 8] = acc[nb][db][2];
+        base[L::kAccStride + d + 8] = acc[nb][db][3];
       }
       if (lane < 4) {
         f[L::kRedM + warp * NCOL + nb * 8 + j0] = m_run[nb][0];

@@ -118,6 +118,18 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, u
                : "r"(addr));
 }
 
+// Two 16x16 byte matrices, transposed.  Matrix j's 16 rows (16 bytes each)
+// come from the addresses of lanes 16j .. 16j+15.  Lane (g = lane / 4,
+// t = lane % 4) receives, for each matrix, rows 4t .. 4t+3 of column g in its
+// first register and of column g + 8 in its second, row 4t + i in byte i.
+// (Layout checked on B200 with a probe that loads a known matrix.)
+__device__ __forceinline__ void ldmatrix_x2_trans_b8(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                                     uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m16n16.x2.trans.shared.b8 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
 // D = A(16x16, row) * B(16x8, col) + D, bf16 inputs, fp32 accumulators.
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
                                                uint32_t b0, uint32_t b1) {
