@@ -25,12 +25,13 @@ constexpr int kMaxDevices = 64;
 // ---------------------------------------------------------------- planner
 
 // Cost model of one call, in microseconds, used to pick the split count.
-// It models device time: the constants were fitted to a split-count sweep
-// measured on B200 from CUDA-graph replays (free of the host's launch work)
-// over 54 shapes: the CodeLlama-34B head shape at B = 1 and L = 512..128K,
-// B = 2..40 at L = 2K..64K, G = 4, the varlen, paged and peaked workloads,
-// bf16 and fp8 caches.  The pick is the fastest measured split count or
-// within 5.5 % of it; the mean regret is 0.5 %.
+// It models device time: the constants were fitted to split-count sweeps
+// measured on B200 from CUDA-graph replays (free of the host's launch work):
+// 36 bf16 shapes (the CodeLlama-34B head shape at B = 1 and L = 512..128K,
+// B = 2..40 at L = 2K..64K, G = 4, the varlen, paged and peaked workloads)
+// and 12 fp8 shapes (B = 1, 4, 16 and the three workloads).  The pick is the
+// fastest measured split count or within 5.7 % of it; the mean regret is
+// 0.7 %.
 //
 // A CTA streams its tokens at a rate of its own (the tile loop's latency,
 // independent of the element type), unless the device's HBM bandwidth,
@@ -39,8 +40,10 @@ constexpr int kMaxDevices = 64;
 //   kCtaTokPerUs       tokens per microsecond of one CTA
 //   kCtaDeepTokPerUs   the same for a bf16 D = 128 grid of at most one CTA
 //                      per SM, which runs the deeper ring
+//   kCtaFp8TokPerUs    the same for an fp8 cache
 //   kCtaPagedTokPerUs  alone on an SM when pages hold fewer than 64 tokens
-//                      (one TMA box per page instead of one per tile)
+//                      (one TMA box per page instead of one per tile) ...
+//   kCtaPagedSharedTokPerUs  ... and two to an SM (bf16 or fp8)
 //   kCtaFixedUs        per-CTA fixed cost within a wave
 //   kCombineUs         device time added by a call with several splits (the
 //                      combine kernel after its dependency) ...
@@ -49,7 +52,9 @@ struct PlanModel {
   static constexpr double kHbmGBs = 6500.0;
   static constexpr double kCtaTokPerUs = 90.0;
   static constexpr double kCtaDeepTokPerUs = 100.0;
+  static constexpr double kCtaFp8TokPerUs = 100.0;
   static constexpr double kCtaPagedTokPerUs = 50.0;
+  static constexpr double kCtaPagedSharedTokPerUs = 80.0;
   static constexpr double kCtaFixedUs = 0.3;
   static constexpr double kCombineUs = 1.0;
   static constexpr double kCombinePer16Us = 2.0;
@@ -78,6 +83,7 @@ struct PlanShape {
   double token_bytes;  // K + V bytes of one token of one KV head
   bool small_pages;    // pages of fewer than 64 tokens
   bool deep_ring;      // bf16, D = 128: a grid of <= num_sms CTAs gets the deep ring
+  bool fp8;            // fp8 E4M3 cache
 };
 
 // Time of one wave of k CTAs of `tokens` tokens each, in a grid of
@@ -85,7 +91,9 @@ struct PlanShape {
 double wave_time_us(const PlanShape& ps, double tokens, double k, double grid) {
   const double hbm_tok = PlanModel::kHbmGBs * 1e3 / (k * ps.token_bytes);
   double own = PlanModel::kCtaTokPerUs;
-  if (k <= ps.num_sms && ps.small_pages) own = PlanModel::kCtaPagedTokPerUs;
+  if (ps.small_pages)
+    own = k <= ps.num_sms ? PlanModel::kCtaPagedTokPerUs : PlanModel::kCtaPagedSharedTokPerUs;
+  else if (ps.fp8) own = PlanModel::kCtaFp8TokPerUs;
   else if (ps.deep_ring && grid <= ps.num_sms) own = PlanModel::kCtaDeepTokPerUs;
   return tokens / std::min(hbm_tok, own) + PlanModel::kCtaFixedUs;
 }
@@ -521,7 +529,8 @@ int plan_impl(int num_sms, int B, int Hkv, int D, int max_len, int block_size, i
   // planning cost for large batches).
   if (static_cast<long long>(B) * Hkv >= 2LL * num_sms * fd::kCtasPerSm) return 1;
   const PlanShape ps{num_sms, B, Hkv, 2.0 * D * elem_bytes,
-                     block_size > 0 && block_size < fd::kTile, elem_bytes == 2 && D == 128};
+                     block_size > 0 && block_size < fd::kTile, elem_bytes == 2 && D == 128,
+                     elem_bytes == 1};
   if (seqlens)
     return pick_splits(max_len, [&](int S) {
       return model_time_lengths(ps, B, max_len, seqlens, S);

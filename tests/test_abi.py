@@ -121,19 +121,48 @@ def test_plan_matches_measured_sweeps(shape, good):
     assert fd.fd_plan_problem(B200_SMS, prob) == fd.fd_plan_sm(B200_SMS, *shape)
 
 
-# The same for fp8 E4M3 caches: an fp8 CTA streams tokens at the bf16 rate,
-# half the bytes, so the fastest split counts put more CTAs in flight.
+# The same for fp8 E4M3 caches (a separate sweep, fastest or within 6 %): an
+# fp8 CTA streams tokens at the bf16 rate, half the bytes, so the fastest split
+# counts put more CTAs in flight.
 @pytest.mark.parametrize("shape,good", [
-    ((1, 64, 8, 128, 4096), {16, 20}),
+    ((1, 64, 8, 128, 8192), {16, 32, 40}),
     ((1, 64, 8, 128, 16384), {32, 40}),
     ((1, 64, 8, 128, 32768), {32}),
     ((1, 64, 8, 128, 65536), {32}),
-    ((4, 64, 8, 128, 2048), {8}),
-    ((16, 64, 8, 128, 2048), {2}),              # 128 units: fp8 still wants 2 CTAs per SM
+    ((1, 64, 8, 128, 131072), {32, 35}),
+    ((4, 64, 8, 128, 16384), {8, 9}),
+    ((16, 64, 8, 128, 8192), {2}),              # 128 units: fp8 still wants 2 CTAs per SM
+    ((16, 64, 8, 128, 16384), {2, 4, 8, 9}),
+    ((16, 64, 8, 128, 65536), {2, 4, 8, 9, 12}),
 ])
 def test_plan_problem_fp8_matches_measured_sweeps(shape, good):
     prob = fd.make_problem(*shape, kv_dtype=fd.FD_KV_FP8_E4M3)
     assert fd.fd_plan_problem(B200_SMS, prob) in good
+
+
+# The three large workloads with their own caches: split counts fastest or
+# within 6 % in the same kind of sweep (lengths given to the planner).
+VARLEN = (32, 32, 8, 128, 32768, 0, 0, 0)
+PAGED = (8, 32, 8, 128, 131072, 16, 65536, 8192)
+PEAKED = (1, 32, 8, 128, 262144, 0, 0, 0)
+
+
+@pytest.mark.parametrize("shape,kv,good", [
+    (VARLEN, fd.FD_KV_BF16, {3}),
+    (VARLEN, fd.FD_KV_FP8_E4M3, {3, 6, 8, 9, 12, 16}),
+    (PAGED, fd.FD_KV_BF16, {3, 4, 8}),
+    (PAGED, fd.FD_KV_FP8_E4M3, {9}),
+    (PEAKED, fd.FD_KV_BF16, {16, 17, 24, 32, 64}),
+    (PEAKED, fd.FD_KV_FP8_E4M3, {32, 35, 64}),
+])
+def test_plan_problem_workloads(shape, kv, good):
+    from split_kv_decode_attn_b200 import workloads as wl
+    lens = None
+    if shape is VARLEN:  # the varlen workload's seeded lengths
+        lens = wl.uniform_int(wl.stream_seed(wl.CONFIG_SEED_BASE + 3, wl.STREAM_SEQLENS), 32,
+                              1024, 32768)
+    prob = fd.make_problem(*shape, kv_dtype=kv)
+    assert fd.fd_plan_problem(B200_SMS, prob, lens) in good
 
 
 def test_plan_problem_checks_and_lengths():
