@@ -99,12 +99,15 @@ def measured_peak():
 
 
 def kernel_source_hash() -> str:
-    """Hash of the device code (the kernels and their PTX helpers)."""
+    """Hash of the device code (the kernels and their PTX helpers), with
+    comments and blank lines left out so that documentation edits keep it."""
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "split_kv_decode_attn_b200", "csrc")
     for name in ("fd_kernels.cuh", "fd_ptx.cuh"):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + b"\0" + f.read())
+        with open(os.path.join(csrc, name)) as f:
+            code = [re.sub(r"//.*$", "", line).rstrip() for line in f]
+        h.update(name.encode() + b"\0" + "\n".join(x for x in code if x).encode())
     return h.hexdigest()[:16]
 
 

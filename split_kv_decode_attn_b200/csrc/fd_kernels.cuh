@@ -2,9 +2,11 @@
 //
 // Split kernel: one CTA per (split, KV head, sequence).  It streams the
 // split's K/V tiles from HBM through a multi-stage shared-memory pipeline
-// fed by TMA tensor loads (128-byte swizzle), and runs the scores and the
+// fed by TMA tensor loads (128-byte swizzle; the first tiles are prefetched
+// into L2 before the wait on the previous grid), and runs the scores and the
 // P.V product for all G query heads of the KV head on the tensor cores
-// (bf16 mma.sync, fp32 accumulation), with an online softmax in between.
+// (mma.sync in bf16, or f16 for an fp8 E4M3 cache converted in registers;
+// fp32 accumulation), with an online softmax in between.
 // Each split ends with a partial output and a log-sum-exp ("What is
 // Flash-Decoding, and when does it speed up LLMs?", slavadubrov.com, section
 // "Why decode needs a different schedule").  The running maximum and
@@ -40,7 +42,8 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
 //         4..7 carry the rounding residual p - bf16(p); their sum restores p
 //         to ~16 bits at no extra MMA.
 //  kHiLo: G = 8 per column block.  A second P.V MMA adds the residual.
-//  kHi  : G = 8 per column block, bf16(p) only.
+//  kHi  : one P.V MMA with P as is: the fp8 path, whose P is f16 (11
+//         significant bits).
 enum PMode { kDup = 0, kHiLo = 1, kHi = 2 };
 
 // Device error word: set when a bounded wait runs out.
