@@ -67,6 +67,22 @@ def test_fp8_paged_matches_contiguous_bit_for_bit(bs, layout):
         assert np.array_equal(gp, gc_) and np.array_equal(lp, lc)
 
 
+@pytest.mark.parametrize("bs", [8, 32])
+def test_fp8_paged_sixteen_heads_per_group(bs):
+    """G = 16 (two column blocks) on a paged fp8 cache, pages under a tile."""
+    B, Hkv, L = 2, 2, 512
+    p = wl.make_problem(B, 16 * Hkv, Hkv, 128, L, seed=350 + bs, seqlens=[512, 77],
+                        block_size=bs, num_blocks=B * L // bs + 2, kv_dtype="fp8")
+    c = contiguous_copy(p)
+    dp, dc = OnDevice(p), OnDevice(c)
+    ref, rl = reference(c)
+    for S in (1, 3):
+        gp, lp, _ = run_gpu(dp, S)
+        gc_, lc, _ = run_gpu(dc, S)
+        assert_close(gp, lp, ref, rl, f"fp8 paged G=16 bs={bs} S={S}")
+        assert np.array_equal(gp, gc_) and np.array_equal(lp, lc)
+
+
 def test_fp8_token_major_matches_head_major():
     B, Hkv, L = 3, 4, 1500
     n = wl.make_problem(B, 16 * Hkv // 4, Hkv, 128, L, seed=360, seqlens=[1500, 9, 640],

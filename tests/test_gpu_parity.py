@@ -268,3 +268,6 @@ def test_planner_on_device_matches_pure_planner():
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     for L in (512, 16384, 65536):
         assert fd.fd_plan(1, 64, 8, 128, L, 0) == fd.fd_plan_sm(sms, 1, 64, 8, 128, L, 0)
+        for kv in (fd.FD_KV_BF16, fd.FD_KV_FP8_E4M3):
+            prob = fd.make_problem(1, 64, 8, 128, L, kv_dtype=kv)
+            assert fd.fd_plan_problem(0, prob) == fd.fd_plan_problem(sms, prob)
