@@ -19,8 +19,9 @@
  * Conventions shared by every entry point:
  *  - Tensor pointers are DEVICE pointers owned by the caller. The library
  *    keeps no pointer and allocates nothing; the workspace is caller-supplied.
- *  - Element types: q, K, V and out are bf16; lse, the workspace and scale
- *    are fp32; seqlens and block_table are int32.
+ *  - Element types: q and out are bf16; K and V are bf16 or fp8 E4M3 codes
+ *    (fd_problem.kv_dtype); lse, the workspace and scale are fp32; seqlens
+ *    and block_table are int32.
  *  - Errors are return codes. No entry point aborts, throws or prints.
  *    Argument checks run on the host before anything is launched; an invalid
  *    call launches nothing.
@@ -176,7 +177,7 @@ FD_API size_t fd_workspace_bytes(int B, int Hq, int D, int num_splits);
  *   q            [B, Hq, D] bf16, 16-byte aligned
  *   k_cache, v_cache
  *                (elements bf16, or fp8 e4m3 bytes when kv_dtype says so)
- *                FD_LAYOUT_HND contiguous: [B, Hkv, max_len, D] bf16;
+ *                FD_LAYOUT_HND contiguous: [B, Hkv, max_len, D];
  *                FD_LAYOUT_HND paged:      [num_blocks, Hkv, block_size, D];
  *                FD_LAYOUT_NHD contiguous: [B, max_len, Hkv, D];
  *                FD_LAYOUT_NHD paged:      [num_blocks, block_size, Hkv, D];
