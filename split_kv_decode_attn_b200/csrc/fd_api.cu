@@ -29,9 +29,9 @@ constexpr int kMaxDevices = 64;
 // measured on B200 from CUDA-graph replays (free of the host's launch work):
 // 36 bf16 shapes (the CodeLlama-34B head shape at B = 1 and L = 512..128K,
 // B = 2..40 at L = 2K..64K, G = 4, the varlen, paged and peaked workloads)
-// and 12 fp8 shapes (B = 1, 4, 16 and the three workloads).  The pick is the
-// fastest measured split count or within 5.7 % of it; the mean regret is
-// 0.7 %.
+// and 12 fp8 shapes (B = 1, 4, 16 and the three workloads).  On a fresh
+// sweep of 54 shapes the pick is the fastest measured split count or within
+// 4.6 % of it; the mean regret is 0.7 %.
 //
 // A CTA streams its tokens at a rate of its own (the tile loop's latency,
 // independent of the element type), unless the device's HBM bandwidth,
