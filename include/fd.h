@@ -250,6 +250,57 @@ FD_API fd_status fd_decode_partial(const fd_problem* p, const void* q, const voi
 FD_API fd_status fd_combine(int R, int B, int Hq, int D, const float* part_o,
                             const float* part_lse, void* out, float* lse, fd_stream_t stream);
 
+/* Low-bit key codes for fd_decode_sparse ("Faster Than Flash: Exploiting
+ * Attention Sparsity for Efficient Long-Context Decoding", abstract: a scan
+ * over low-bit keys replaces metadata indices). Call it when the cache
+ * changes (in a decode loop, for the blocks that tokens were appended to).
+ * For every 64-token block of every (sequence, KV head):
+ *   k8_scale = max |K| over the block's valid rows / 127 (1 for an all-zero
+ *              block), fp32;
+ *   k8       = rint(K / k8_scale) in [-127, 127], int8; rows at or past the
+ *              sequence's length get 0.
+ *   p         contiguous head-major bf16 cache (block_size 0, FD_LAYOUT_HND,
+ *             FD_KV_BF16), D 64 or 128
+ *   k_cache   [B, Hkv, max_len, D] bf16, 16-byte aligned
+ *   seqlens   [B] int32 or NULL (all max_len)
+ *   k8        [B, Hkv, max_len, D] int8 out, 16-byte aligned
+ *   k8_scale  [B, Hkv, ceil(max_len / 64)] fp32 out
+ * Returns FD_ERR_UNSUPPORTED for a paged, token-major or fp8 cache. */
+FD_API fd_status fd_quantize_keys(const fd_problem* p, const void* k_cache,
+                                  const int32_t* seqlens, int8_t* k8, float* k8_scale,
+                                  fd_stream_t stream);
+
+/* Sparse decode: fd_decode over the blocks a low-bit scan selects (same page,
+ * abstract: a top-delta rule that filters blocks adaptively with no global
+ * synchronisation, selector and computation fused in one kernel). Inside the
+ * split kernel, before any K/V tile is loaded, each CTA (one split of one
+ * KV head of one sequence):
+ *   1. turns each query head of the group into int8: sq = max |q| / 127,
+ *      q8 = rint(q / sq);
+ *   2. computes for every 64-token block of its split, and every head, the
+ *      largest approximate logit ((scale * sq) * k8_scale) * (q8 . k8), with
+ *      the dot product exact in integers and each product rounded to fp32 in
+ *      that order;
+ *   3. keeps a block when some head's block maximum is >= M - delta, M being
+ *      that head's largest block maximum in the split;
+ *   4. runs the exact bf16 attention of fd_decode over the kept blocks only.
+ * The splits then merge as in fd_decode. The result is the exact attention
+ * over the union of the kept blocks. delta = +inf keeps every block and gives
+ * fd_decode's result bit for bit.
+ *   k8, k8_scale  from fd_quantize_keys on the same cache and lengths
+ *   delta         >= 0, natural-log units (NaN is invalid)
+ *   kept          [B, Hkv, ceil(max_len / 64)] uint8 out (1 = kept), or NULL.
+ *                 Blocks at or past a sequence's length are not written.
+ * Other arguments are those of fd_decode with a contiguous head-major bf16
+ * cache. The split count must make the chunk at most 65,536 tokens
+ * (FD_ERR_INVALID_ARGUMENT otherwise). Results are deterministic. */
+FD_API fd_status fd_decode_sparse(const fd_problem* p, const void* q, const void* k_cache,
+                                  const void* v_cache, const int8_t* k8,
+                                  const float* k8_scale, const int32_t* seqlens, float scale,
+                                  float delta, int num_splits, void* out, float* lse,
+                                  uint8_t* kept, void* workspace, size_t workspace_bytes,
+                                  fd_stream_t stream);
+
 /* Largest workspace, in bytes, that fd_decode_static_workspace can use. */
 #define FD_STATIC_WORKSPACE_BYTES (8u << 20)
 

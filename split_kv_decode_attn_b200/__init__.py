@@ -28,7 +28,8 @@ FD_ERR_DEVICE_TIMEOUT = -5
 
 # Entry points declared in include/fd.h.
 EXPORTS = ("fd_plan", "fd_plan_sm", "fd_plan_seqlens", "fd_plan_problem", "fd_split_chunk", "fd_workspace_bytes", "fd_decode",
-           "fd_decode_partial", "fd_combine", "fd_decode_static_workspace", "fd_check_device_error",
+           "fd_decode_partial", "fd_combine", "fd_quantize_keys", "fd_decode_sparse",
+           "fd_decode_static_workspace", "fd_check_device_error",
            "fd_selftest_device_timeout", "fd_status_string")
 
 # Mirrors FD_STATIC_WORKSPACE_BYTES in include/fd.h.
@@ -86,6 +87,11 @@ def load_library(path: str = LIB_PATH):
         lib.fd_decode_partial.argtypes = [ctypes.POINTER(fd_problem), vp, vp, vp, vp, vp, F, I,
                                           vp, vp, vp, sz, vp]
         lib.fd_decode_partial.restype = I
+        lib.fd_quantize_keys.argtypes = [ctypes.POINTER(fd_problem), vp, vp, vp, vp, vp]
+        lib.fd_quantize_keys.restype = I
+        lib.fd_decode_sparse.argtypes = [ctypes.POINTER(fd_problem), vp, vp, vp, vp, vp, vp, F,
+                                         F, I, vp, vp, vp, vp, sz, vp]
+        lib.fd_decode_sparse.restype = I
         lib.fd_combine.argtypes = [I, I, I, I, vp, vp, vp, vp, vp]
         lib.fd_combine.restype = I
         lib.fd_decode_static_workspace.argtypes = [ctypes.POINTER(fd_problem), vp, vp, vp, vp,
@@ -179,6 +185,25 @@ def fd_decode_partial(problem: fd_problem, q, k_cache, v_cache, seqlens, block_t
         ctypes.byref(problem), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens),
         _ptr(block_table), scale, num_splits, _ptr(out_f32), _ptr(lse), _ptr(workspace),
         workspace_bytes, _stream(stream)))
+
+
+def fd_quantize_keys(problem: fd_problem, k_cache, seqlens, k8, k8_scale, stream=None) -> int:
+    """Call the C fd_quantize_keys: int8 key codes and per-64-token-block
+    scales for fd_decode_sparse.  Returns the status."""
+    return int(load_library().fd_quantize_keys(ctypes.byref(problem), _ptr(k_cache),
+                                               _ptr(seqlens), _ptr(k8), _ptr(k8_scale),
+                                               _stream(stream)))
+
+
+def fd_decode_sparse(problem: fd_problem, q, k_cache, v_cache, k8, k8_scale, seqlens,
+                     scale: float, delta: float, num_splits: int, out, lse, kept, workspace,
+                     workspace_bytes: int, stream=None) -> int:
+    """Call the C fd_decode_sparse: the low-bit scan and top-delta block
+    selection, then exact attention over the kept blocks.  Returns the status."""
+    return int(load_library().fd_decode_sparse(
+        ctypes.byref(problem), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k8), _ptr(k8_scale),
+        _ptr(seqlens), scale, delta, num_splits, _ptr(out), _ptr(lse), _ptr(kept),
+        _ptr(workspace), workspace_bytes, _stream(stream)))
 
 
 def fd_combine(R: int, B: int, Hq: int, D: int, part_o, part_lse, out, lse, stream=None) -> int:

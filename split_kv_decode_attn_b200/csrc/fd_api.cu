@@ -302,12 +302,13 @@ constexpr int split_stages() {
   return (D == 128 && !FP8) ? (DEEP ? 4 : 3) : 6;
 }
 
-template <int D, int NB, int MODE, bool PAGED, bool FP8 = false, bool DEEP = false>
+template <int D, int NB, int MODE, bool PAGED, bool FP8 = false, bool DEEP = false,
+          bool SPARSE = false>
 fd_status launch_split(const CUtensorMap& tk, const CUtensorMap& tv, const fd::SplitArgs& a,
                        int n_splits, int Hkv, int B, cudaStream_t stream) {
   constexpr int STAGES = split_stages<D, FP8, DEEP>();
-  using L = fd::SplitSmem<D, NB, STAGES, FP8>;
-  auto kern = fd::fd_split_kernel<D, NB, MODE, PAGED, STAGES, FP8>;
+  using L = fd::SplitSmem<D, NB, STAGES, FP8, SPARSE>;
+  auto kern = fd::fd_split_kernel<D, NB, MODE, PAGED, STAGES, FP8, SPARSE>;
   // The shared-memory opt-in is per device; remember which devices have it.
   static std::atomic<unsigned long long> attr_done{0};
   int dev = 0;
@@ -353,10 +354,24 @@ fd_status launch_combine(const fd::SplitArgs& a, int B, cudaStream_t stream) {
 // Launches the split kernel and, with several splits, the combine kernel.
 // deep: the grid has at most one CTA per SM, so a deeper ring costs no
 // occupancy (bf16, D = 128 only; measured 5 % faster at 16K tokens, S = 16).
+// sparse: the low-bit scan and top-delta selection run first (contiguous
+// bf16 caches only).
 template <int D, int NB, int MODE, bool PAGED, bool FP8 = false>
 fd_status launch_call(const CUtensorMap& tk, const CUtensorMap& tv, const fd::SplitArgs& a,
-                      int n_splits, int Hkv, int B, bool deep, cudaStream_t s) {
-  fd_status r;
+                      int n_splits, int Hkv, int B, bool deep, bool sparse, cudaStream_t s) {
+  fd_status r = FD_ERR_UNSUPPORTED;
+  if constexpr (!PAGED && !FP8) {
+    if (sparse) {
+      if constexpr (D == 128)
+        r = deep ? launch_split<D, NB, MODE, PAGED, FP8, true, true>(tk, tv, a, n_splits, Hkv, B, s)
+                 : launch_split<D, NB, MODE, PAGED, FP8, false, true>(tk, tv, a, n_splits, Hkv, B, s);
+      else
+        r = launch_split<D, NB, MODE, PAGED, FP8, false, true>(tk, tv, a, n_splits, Hkv, B, s);
+      if (r == FD_OK && n_splits > 1) r = launch_combine<D>(a, B, s);
+      return r;
+    }
+  }
+  if (sparse) return FD_ERR_UNSUPPORTED;
   if constexpr (D == 128 && !FP8) {
     r = deep ? launch_split<D, NB, MODE, PAGED, FP8, true>(tk, tv, a, n_splits, Hkv, B, s)
              : launch_split<D, NB, MODE, PAGED, FP8, false>(tk, tv, a, n_splits, Hkv, B, s);
@@ -374,17 +389,19 @@ fd_status dispatch_split_fp8(int G, const CUtensorMap& tk, const CUtensorMap& tv
                              const fd::SplitArgs& a, int n_splits, int Hkv, int B,
                              cudaStream_t s) {
   if (G <= 8)
-    return launch_call<128, 1, fd::kHi, PAGED, true>(tk, tv, a, n_splits, Hkv, B, false, s);
-  return launch_call<128, 2, fd::kHi, PAGED, true>(tk, tv, a, n_splits, Hkv, B, false, s);
+    return launch_call<128, 1, fd::kHi, PAGED, true>(tk, tv, a, n_splits, Hkv, B, false, false, s);
+  return launch_call<128, 2, fd::kHi, PAGED, true>(tk, tv, a, n_splits, Hkv, B, false, false, s);
 }
 
 template <int D, bool PAGED>
 fd_status dispatch_split(int G, const CUtensorMap& tk, const CUtensorMap& tv,
                          const fd::SplitArgs& a, int n_splits, int Hkv, int B, bool deep,
-                         cudaStream_t s) {
-  if (G <= 4) return launch_call<D, 1, fd::kDup, PAGED>(tk, tv, a, n_splits, Hkv, B, deep, s);
-  if (G == 8) return launch_call<D, 1, fd::kHiLo, PAGED>(tk, tv, a, n_splits, Hkv, B, deep, s);
-  return launch_call<D, 2, fd::kHiLo, PAGED>(tk, tv, a, n_splits, Hkv, B, deep, s);
+                         bool sparse, cudaStream_t s) {
+  if (G <= 4)
+    return launch_call<D, 1, fd::kDup, PAGED>(tk, tv, a, n_splits, Hkv, B, deep, sparse, s);
+  if (G == 8)
+    return launch_call<D, 1, fd::kHiLo, PAGED>(tk, tv, a, n_splits, Hkv, B, deep, sparse, s);
+  return launch_call<D, 2, fd::kHiLo, PAGED>(tk, tv, a, n_splits, Hkv, B, deep, sparse, s);
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -414,12 +431,21 @@ int pick_splits(int max_len, Model model) {
   return best;
 }
 
+// Inputs of the sparse decode (null for the dense one).
+struct SparseArgs {
+  const int8_t* k8;
+  const float* k8_scale;
+  uint8_t* kept;
+  float delta;
+};
+
 // One decode call.  The result goes to `out` (bf16) or, for a partial over a
 // shard of the history, to `out_f32` (fp32); exactly one of them is set.
 fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
                       const void* v_cache, const int32_t* seqlens, const int32_t* block_table,
                       float scale, int num_splits, void* out, float* out_f32, float* lse,
-                      void* workspace, size_t workspace_bytes, fd_stream_t stream) {
+                      void* workspace, size_t workspace_bytes, fd_stream_t stream,
+                      const SparseArgs* sp = nullptr) {
   // ---- host-side checks: nothing is launched for an invalid call
   if (!p || !q || !k_cache || !v_cache || (!out == !out_f32)) return FD_ERR_INVALID_ARGUMENT;
   const fd_status st = check_shape(p->B, p->Hq, p->Hkv, p->D, p->max_len, p->block_size);
@@ -447,6 +473,14 @@ fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
       !aligned(lse, 4) || !aligned(workspace, 16) || !aligned(seqlens, 4) ||
       !aligned(block_table, 4))
     return FD_ERR_INVALID_ARGUMENT;
+  if (sp) {
+    if (paged || fp8) return FD_ERR_UNSUPPORTED;
+    if (!sp->k8 || !sp->k8_scale || !aligned(sp->k8, 16) || !aligned(sp->k8_scale, 4) ||
+        std::isnan(sp->delta) || sp->delta < 0.f)
+      return FD_ERR_INVALID_ARGUMENT;
+    if (chunk_for(p->max_len, num_splits) > fd::kMaxSparseTiles * fd::kTile)
+      return FD_ERR_INVALID_ARGUMENT;
+  }
 
   const int B = p->B, Hq = p->Hq, Hkv = p->Hkv, D = p->D, G = Hq / Hkv;
   const int chunk = chunk_for(p->max_len, num_splits);
@@ -501,7 +535,15 @@ fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
   // L2 prefetch ahead of the wait on the previous grid (contiguous caches):
   // half the split's tiles, at most kPrefetchTiles.  Swept on B200 over
   // 0..12 tiles at 4K..64K tokens, bf16 and fp8, S = 16 and 32.
-  a.prefetch_tiles = paged ? 0 : std::min(kPrefetchTiles, std::max(1, chunk / fd::kTile / 2));
+  a.prefetch_tiles = (paged || sp) ? 0 : std::min(kPrefetchTiles, std::max(1, chunk / fd::kTile / 2));
+  a.scale = scale;
+  if (sp) {
+    a.k8 = sp->k8;
+    a.k8_scale = sp->k8_scale;
+    a.kept_out = sp->kept;
+    a.n_blocks = (p->max_len + fd::kTile - 1) / fd::kTile;
+    a.delta = sp->delta;
+  }
 
   int sms = 0;
   if (device_sms(dev, &sms) != FD_OK) return FD_ERR_CUDA;
@@ -513,11 +555,11 @@ fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
     r = paged ? dispatch_split_fp8<true>(G, tk, tv, a, n_splits, Hkv, B, s)
               : dispatch_split_fp8<false>(G, tk, tv, a, n_splits, Hkv, B, s);
   else if (D == 128)
-    r = paged ? dispatch_split<128, true>(G, tk, tv, a, n_splits, Hkv, B, deep, s)
-              : dispatch_split<128, false>(G, tk, tv, a, n_splits, Hkv, B, deep, s);
+    r = paged ? dispatch_split<128, true>(G, tk, tv, a, n_splits, Hkv, B, deep, false, s)
+              : dispatch_split<128, false>(G, tk, tv, a, n_splits, Hkv, B, deep, sp != nullptr, s);
   else
-    r = paged ? dispatch_split<64, true>(G, tk, tv, a, n_splits, Hkv, B, deep, s)
-              : dispatch_split<64, false>(G, tk, tv, a, n_splits, Hkv, B, deep, s);
+    r = paged ? dispatch_split<64, true>(G, tk, tv, a, n_splits, Hkv, B, deep, false, s)
+              : dispatch_split<64, false>(G, tk, tv, a, n_splits, Hkv, B, deep, sp != nullptr, s);
   return r;
 }
 
@@ -624,6 +666,51 @@ fd_status fd_decode_partial(const fd_problem* p, const void* q, const void* k_ca
   if (!out_f32 || !lse) return FD_ERR_INVALID_ARGUMENT;
   return decode_impl(p, q, k_cache, v_cache, seqlens, block_table, scale, num_splits, nullptr,
                      out_f32, lse, workspace, workspace_bytes, stream);
+}
+
+fd_status fd_quantize_keys(const fd_problem* p, const void* k_cache, const int32_t* seqlens,
+                           int8_t* k8, float* k8_scale, fd_stream_t stream) {
+  if (!p || !k_cache || !k8 || !k8_scale) return FD_ERR_INVALID_ARGUMENT;
+  const fd_status st = check_shape(p->B, p->Hq, p->Hkv, p->D, p->max_len, p->block_size);
+  if (st != FD_OK) return st;
+  if (p->block_size != 0 || p->kv_layout != FD_LAYOUT_HND || p->kv_dtype != FD_KV_BF16)
+    return FD_ERR_UNSUPPORTED;
+  if (!aligned(k_cache, 16) || !aligned(k8, 16) || !aligned(k8_scale, 4) || !aligned(seqlens, 4))
+    return FD_ERR_INVALID_ARGUMENT;
+  if (p->max_len == 0) return FD_OK;
+  int dev = 0;
+  if (current_device(&dev) != FD_OK) return FD_ERR_CUDA;
+  const fd_status arch = device_is_sm100(dev);
+  if (arch != FD_OK) return arch;
+  const int n_blocks = (p->max_len + fd::kTile - 1) / fd::kTile;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(n_blocks), static_cast<unsigned>(p->Hkv),
+                     static_cast<unsigned>(p->B));
+  cfg.blockDim = dim3(128);
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const __nv_bfloat16* k = static_cast<const __nv_bfloat16*>(k_cache);
+  const cudaError_t e =
+      p->D == 128 ? cudaLaunchKernelEx(&cfg, fd::fd_quantize_keys_kernel<128>, k, seqlens, p->Hkv,
+                                       p->max_len, n_blocks, k8, k8_scale)
+                  : cudaLaunchKernelEx(&cfg, fd::fd_quantize_keys_kernel<64>, k, seqlens, p->Hkv,
+                                       p->max_len, n_blocks, k8, k8_scale);
+  return e == cudaSuccess ? FD_OK : FD_ERR_CUDA;
+}
+
+fd_status fd_decode_sparse(const fd_problem* p, const void* q, const void* k_cache,
+                           const void* v_cache, const int8_t* k8, const float* k8_scale,
+                           const int32_t* seqlens, float scale, float delta, int num_splits,
+                           void* out, float* lse, uint8_t* kept, void* workspace,
+                           size_t workspace_bytes, fd_stream_t stream) {
+  if (!out) return FD_ERR_INVALID_ARGUMENT;
+  const SparseArgs sp{k8, k8_scale, kept, delta};
+  return decode_impl(p, q, k_cache, v_cache, seqlens, nullptr, scale, num_splits, out, nullptr,
+                     lse, workspace, workspace_bytes, stream, &sp);
 }
 
 fd_status fd_combine(int R, int B, int Hq, int D, const float* part_o, const float* part_lse,

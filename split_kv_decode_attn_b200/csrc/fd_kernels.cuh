@@ -69,7 +69,17 @@ struct SplitArgs {
   float v_scale;                // dequantisation scale of an fp8 V cache (1 for bf16)
   int prefetch_tiles;           // contiguous caches: tiles per CTA prefetched into L2 before
                                 // the wait on the previous grid (0 = none)
+  // Sparse decode (low-bit scan + top-delta) only:
+  const int8_t* k8;             // [B, Hkv, max_len, D] int8 key codes
+  const float* k8_scale;        // [B, Hkv, n_blocks] per 64-token block
+  uint8_t* kept_out;            // [B, Hkv, n_blocks] 1 = block kept, or null
+  int n_blocks;                 // ceil(max_len / 64)
+  float scale;                  // softmax scale (natural-log domain)
+  float delta;                  // top-delta threshold, natural-log units
 };
+
+// Longest split, in 64-token blocks, that the sparse scan handles.
+constexpr int kMaxSparseTiles = 1024;
 
 // Token of row s (0..15) of the fp8 score MMA within a warp's 16-token slice:
 // rows 2t, 2t+1 -> tokens 4t, 4t+1 and rows 8+2t, 8+2t+1 -> tokens 4t+2, 4t+3.
@@ -177,7 +187,7 @@ __device__ __forceinline__ void combine_row(const float* po, const float* pl, in
   if (lse_out && lane == 0) *lse_out = mx == -INFINITY ? -INFINITY : mx + logf(W);
 }
 
-template <int D, int NB, int STAGES, bool FP8 = false>
+template <int D, int NB, int STAGES, bool FP8 = false, bool SPARSE = false>
 struct SplitSmem {
   // Rows are stored in 128-byte swizzle rows: a bf16 row of D = 128 takes two
   // (its column halves), an fp8 row of 128 takes one.
@@ -186,7 +196,9 @@ struct SplitSmem {
   static constexpr int kTileBytes = kHalves * kHalfBytes;
   static constexpr int kStageBytes = 2 * kTileBytes;   // K tile + V tile
   static constexpr int kBarOffset = STAGES * kStageBytes;
-  static constexpr int kBytes = kBarOffset + 2 * STAGES * 8 + 16;  // + error flag
+  // + error flag; sparse: + the kept-tile list (uint16) and its length
+  static constexpr int kListOffset = kBarOffset + 2 * STAGES * 8 + 16;
+  static constexpr int kBytes = kListOffset + (SPARSE ? 2 * kMaxSparseTiles + 16 : 0);
   static constexpr int kDynamicBytes = kBytes + 1024;  // room to align to 1 KB
   // Epilogue scratch, laid over the drained pipeline buffers (floats):
   static constexpr int kNcol = NB * 8;
@@ -202,17 +214,134 @@ struct SplitSmem {
   static_assert(kScratchFloats * 4 <= kBarOffset, "epilogue scratch must fit the pipeline buffers");
 };
 
+// Sparse decode, selection step ("Faster Than Flash: Exploiting Attention
+// Sparsity for Efficient Long-Context Decoding", abstract: a low-bit scan of
+// the keys selects blocks by a top-delta rule that each unit of work applies
+// on its own, with no global synchronisation).  All threads of the CTA take
+// part, before the tile pipeline starts, using its buffers as scratch.
+//  1. q of each head of the group to int8: sq = max|q| / 127, q8 = rint(q/sq).
+//  2. For every 64-token block of the split and every head: the largest
+//     approximate logit ((scale * sq) * sk) * (q8 . k8), the dot product exact
+//     in integers (dp4a) and each product rounded to fp32 in that order.
+//  3. Per head M = the split's largest block maximum; a block is kept when
+//     some head has a block maximum >= M - delta.
+// Returns the number of kept blocks; `list` gets their indices in order.
+template <int D, int GMAX>
+__device__ __forceinline__ int sparse_select(const SplitArgs& a, uint8_t* scratch, uint16_t* list,
+                                          int* n_kept, int b, int kvh, int h0, int start,
+                                          int end, int n_tiles) {
+  static_assert(D % 128 == 0 || D == 64, "head dim");
+  int8_t* q8 = reinterpret_cast<int8_t*>(scratch);                 // [GMAX][D]
+  float* qs = reinterpret_cast<float*>(scratch + GMAX * D);        // [GMAX]: scale * sq
+  float* thr = qs + GMAX;                                          // [GMAX]
+  float* bmax = thr + GMAX;                                        // [n_tiles][GMAX]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kWarps = kThreads / 32;
+  constexpr int VPL = D / 32;                                      // q entries per lane
+
+  for (int g = warp; g < a.G; g += kWarps) {
+    const __nv_bfloat16* qrow = a.q + (static_cast<size_t>(b) * a.Hq + h0 + g) * D + lane * VPL;
+    float v[VPL];
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      v[i] = __bfloat162float(qrow[i]);
+      amax = fmaxf(amax, fabsf(v[i]));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const float sq = amax > 0.f ? __fdiv_rn(amax, 127.f) : 1.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int c = __float2int_rn(__fdiv_rn(v[i], sq));
+      q8[g * D + lane * VPL + i] = static_cast<int8_t>(max(-127, min(127, c)));
+    }
+    if (lane == 0) qs[g] = __fmul_rn(a.scale, sq);
+  }
+  __syncthreads();
+
+  // One warp per block, one token row per lane at a time.
+  const int8_t* k8 = a.k8 + (static_cast<size_t>(b) * a.Hkv + kvh) * a.max_len * D;
+  const size_t srow = (static_cast<size_t>(b) * a.Hkv + kvh) * a.n_blocks;
+  const int blk0 = start / kTile;
+  for (int i = warp; i < n_tiles; i += kWarps) {
+    const float sk = a.k8_scale[srow + blk0 + i];
+    float m[GMAX];
+#pragma unroll
+    for (int g = 0; g < GMAX; ++g) m[g] = -INFINITY;
+    for (int r = lane; r < kTile; r += 32) {
+      const int t = start + i * kTile + r;
+      if (t >= end) break;
+      const int4* row = reinterpret_cast<const int4*>(k8 + static_cast<size_t>(t) * D);
+      int4 kw[D / 16];
+#pragma unroll
+      for (int w = 0; w < D / 16; ++w) kw[w] = __ldg(row + w);
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g) {
+        if (g < a.G) {
+          const int4* qw = reinterpret_cast<const int4*>(q8 + g * D);
+          int acc = 0;
+#pragma unroll
+          for (int w = 0; w < D / 16; ++w) {
+            const int4 qv = qw[w];
+            acc = __dp4a(kw[w].x, qv.x, acc);
+            acc = __dp4a(kw[w].y, qv.y, acc);
+            acc = __dp4a(kw[w].z, qv.z, acc);
+            acc = __dp4a(kw[w].w, qv.w, acc);
+          }
+          m[g] = fmaxf(m[g], __fmul_rn(__fmul_rn(qs[g], sk), __int2float_rn(acc)));
+        }
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < GMAX; ++g) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1)
+        m[g] = fmaxf(m[g], __shfl_xor_sync(0xffffffffu, m[g], off));
+      if (lane == 0 && g < a.G) bmax[i * GMAX + g] = m[g];
+    }
+  }
+  __syncthreads();
+
+  if (threadIdx.x < a.G) {
+    float M = -INFINITY;
+    for (int i = 0; i < n_tiles; ++i) M = fmaxf(M, bmax[i * GMAX + threadIdx.x]);
+    thr[threadIdx.x] = __fsub_rn(M, a.delta);
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    int count = 0;
+    for (int i0 = 0; i0 < n_tiles; i0 += 32) {
+      const int i = i0 + lane;
+      bool keep = false;
+      if (i < n_tiles) {
+        for (int g = 0; g < a.G; ++g) keep |= bmax[i * GMAX + g] >= thr[g];
+        if (a.kept_out) a.kept_out[srow + blk0 + i] = keep ? 1 : 0;
+      }
+      const unsigned mask = __ballot_sync(0xffffffffu, keep);
+      if (keep) list[count + __popc(mask & ((1u << lane) - 1u))] = static_cast<uint16_t>(i);
+      count += __popc(mask);
+    }
+    if (lane == 0) *n_kept = count;
+  }
+  __syncthreads();
+  return *n_kept;
+}
+
 // Consumer warps of the split kernel: scores, online softmax and P.V over the
 // split's tiles, then the merge of the four warps' softmax states into this
 // split's result, which goes to `out` (the sequence has one split) or to the
 // global partials (several splits).
-template <int D, int NB, int MODE, int STAGES, bool FP8>
+template <int D, int NB, int MODE, int STAGES, bool FP8, bool SPARSE>
 __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* smem,
                                                 uint32_t smem_base, uint32_t bar_full,
                                                 uint32_t bar_empty, volatile int* cta_error,
                                                 int warp, int lane, int b, int h0, int split,
-                                                int start, int end, int n_tiles, int n_parts) {
-  using L = SplitSmem<D, NB, STAGES, FP8>;
+                                                int start, int end, int n_tiles, int n_parts,
+                                                const uint16_t* list) {
+  using L = SplitSmem<D, NB, STAGES, FP8, SPARSE>;
   constexpr int KSTEPS = D / 16;   // k-steps of the score MMA (over D)
   constexpr int DBLK = D / 16;     // m-blocks of the P.V MMA (over D)
   constexpr int NCOL = NB * 8;     // MMA columns (query heads, maybe doubled)
@@ -300,7 +429,8 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
     }
     const uint32_t kbase = smem_base + s * L::kStageBytes;
     const uint32_t vbase = kbase + L::kTileBytes;
-    const int tile_valid = min(kTile, end - (start + it * kTile));
+    const int blk = SPARSE ? static_cast<int>(list[it]) : it;   // kept blocks only, in order
+    const int tile_valid = min(kTile, end - (start + blk * kTile));
     const bool partial = tile_valid < kTile;
 
     // S^T = K Q^T for this warp's 16 tokens (two chains for ILP).
@@ -605,11 +735,12 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
 
 // Split kernel: one CTA per (split, KV head, sequence).  FP8: the cache
 // holds e4m3 values (D = 128); the contraction runs on f16 tensor cores.
-template <int D, int NB, int MODE, bool PAGED, int STAGES, bool FP8>
+template <int D, int NB, int MODE, bool PAGED, int STAGES, bool FP8, bool SPARSE = false>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     fd_split_kernel(const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const SplitArgs a) {
-  using L = SplitSmem<D, NB, STAGES, FP8>;
+  using L = SplitSmem<D, NB, STAGES, FP8, SPARSE>;
+  static_assert(!SPARSE || (!PAGED && !FP8), "sparse decode: contiguous bf16 caches");
   static_assert(MODE != kDup || NB == 1, "duplicated columns need one column block");
 
   extern __shared__ uint8_t smem_raw[];
@@ -679,6 +810,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     return;
   }
 
+  // Tiles the pipeline runs: all of the split's, or the kept ones in order.
+  int n_work = n_tiles;
+  uint16_t* list = reinterpret_cast<uint16_t*>(smem + L::kListOffset);
+  if constexpr (SPARSE)
+    n_work = sparse_select<D, NB * 8>(a, smem, list,
+                                      reinterpret_cast<int*>(smem + L::kListOffset +
+                                                             2 * kMaxSparseTiles),
+                                      b, kvh, h0, start, end, n_tiles);
+
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------- producer
     // Every lane waits (the decision is made warp-uniform); lane 0 issues.
@@ -686,12 +826,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     int issued = 0;
     bool ok = true;
     if constexpr (!PAGED) {
-      for (int it = 0; it < n_tiles; ++it) {
+      for (int it = 0; it < n_work; ++it) {
         const int s = it % STAGES, k = it / STAGES;
         if (k > 0) ok = mbar_wait(bar_empty + 8 * s, (k - 1) & 1, kWaitLimitNs);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         if (lane == 0) {
-          const int t0 = start + it * kTile;
+          const int t0 = start + (SPARSE ? static_cast<int>(list[it]) : it) * kTile;
           const uint32_t dk = smem_base + s * L::kStageBytes;
           const uint32_t dv = dk + L::kTileBytes;
           mbar_arrive_expect_tx(bar_full + 8 * s, L::kStageBytes);
@@ -711,7 +851,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       int win = start >> lbs;
       int cur = (win + lane < n_pages) ? __ldg(bt + win + lane) : 0;
       int nxt = (win + 32 + lane < n_pages) ? __ldg(bt + win + 32 + lane) : 0;
-      for (int it = 0; it < n_tiles; ++it) {
+      for (int it = 0; it < n_work; ++it) {
         const int s = it % STAGES, k = it / STAGES;
         if (k > 0) ok = mbar_wait(bar_empty + 8 * s, (k - 1) & 1, kWaitLimitNs);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
@@ -758,9 +898,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
   } else {
     // ------------------------------------------------------------- consumers
-    split_consumers<D, NB, MODE, STAGES, FP8>(a, smem, smem_base, bar_full, bar_empty, cta_error,
-                                         warp, lane, b, h0, split, start, end, n_tiles,
-                                         n_parts);
+    split_consumers<D, NB, MODE, STAGES, FP8, SPARSE>(a, smem, smem_base, bar_full, bar_empty,
+                                                      cta_error, warp, lane, b, h0, split,
+                                                      start, end, n_work, n_parts, list);
   }
 }
 
@@ -808,6 +948,69 @@ __global__ void __launch_bounds__(128) fd_merge_kernel(const float* part_o, cons
   combine_row<D>(part_o + static_cast<size_t>(row) * D, part_lse + row, R,
                  static_cast<size_t>(rows) * D, static_cast<size_t>(rows),
                  out + static_cast<size_t>(row) * D, nullptr, lse ? lse + row : nullptr, lane);
+}
+
+// Low-bit key codes for the sparse decode: one CTA of 128 threads per
+// (64-token block, KV head, sequence) of a contiguous head-major bf16 cache.
+// sk = max |K| over the block's valid rows / 127 (1 for an all-zero block) and
+// k8 = rint(K / sk), in [-127, 127]; rows at or past the sequence's length get
+// k8 = 0 and take no part in sk.
+template <int D>
+__global__ void __launch_bounds__(128)
+    fd_quantize_keys_kernel(const __nv_bfloat16* k, const int32_t* seqlens, int Hkv, int max_len,
+                            int n_blocks, int8_t* k8, float* k8_scale) {
+  grid_dependency_wait();
+  grid_dependents_launch();
+  constexpr int PER = kTile * D / 128;      // entries per thread: half a row
+  __shared__ float red[4];
+  const int blk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int n = seq_length(seqlens, b, max_len);
+  const int row = blk * kTile + threadIdx.x / 2;
+  const int col = (threadIdx.x & 1) * PER;
+  const size_t base = ((static_cast<size_t>(b) * Hkv + kvh) * max_len + row) * D + col;
+  float v[PER];
+  float amax = 0.f;
+  if (row < n) {
+#pragma unroll
+    for (int w = 0; w < PER / 8; ++w) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(k + base + 8 * w);
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(h[j]);
+        v[8 * w + 2 * j] = f.x;
+        v[8 * w + 2 * j + 1] = f.y;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  } else {
+#pragma unroll
+    for (int i = 0; i < PER; ++i) v[i] = 0.f;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  const float sk = amax > 0.f ? __fdiv_rn(amax, 127.f) : 1.f;
+  if (threadIdx.x == 0) k8_scale[(static_cast<size_t>(b) * Hkv + kvh) * n_blocks + blk] = sk;
+  if (row >= max_len) return;
+#pragma unroll
+  for (int w = 0; w < PER / 16; ++w) {
+    uint32_t word[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t x = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c = max(-127, min(127, __float2int_rn(__fdiv_rn(v[16 * w + 4 * j + e], sk))));
+        x |= (static_cast<uint32_t>(c) & 0xffu) << (8 * e);
+      }
+      word[j] = x;
+    }
+    *reinterpret_cast<uint4*>(k8 + base + 16 * w) = make_uint4(word[0], word[1], word[2], word[3]);
+  }
 }
 
 // Diagnostic: waits, with the kernels' bounded wait, on an mbarrier that

@@ -334,6 +334,32 @@ def plant_dominant_keys(w: Workload, count: int, seed: int, magnitude: float = 4
     return pos
 
 
+def plant_group_keys(w: Workload, count: int, seed: int, magnitude: float = 4.0) -> np.ndarray:
+    """Like plant_dominant_keys, but the key follows the normalised sum of all
+    query heads of the group, magnitude * u * sqrt(D) with u = sum_g q_g /
+    |sum_g q_g|, so that it stands out for every head of the group (the
+    sparse decode's peaked input).  Returns the positions."""
+    assert not w.paged and w.layout == "HND"
+    pos = distinct_positions(stream_seed(seed, STREAM_POS), count, w.max_len)
+    G = w.G
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            u = bf16_bits_to_f64(w.q[b, h * G:(h + 1) * G]).sum(axis=0)
+            key = magnitude * u / np.linalg.norm(u) * math.sqrt(w.D)
+            w.k[b, h, pos, :] = f64_to_bf16_bits(key)[None, :]
+    w.meta["dominant_positions"] = pos
+    return pos
+
+
+def peaked_group(nthreads: Optional[int] = None) -> Workload:
+    """The peaked workload's shape (B=1, Hq=32, Hkv=8, D=128, L=262144) with its
+    64 dominant keys aligned with the whole query group (plant_group_keys)."""
+    seed = CONFIG_SEED_BASE + 6
+    w = make_problem(1, 32, 8, 128, 262144, seed, name="peaked-group-L256K", nthreads=nthreads)
+    plant_group_keys(w, 64, seed)
+    return w
+
+
 # --- the five workloads -------------------------------------------------------
 
 CONFIG_SEED_BASE = 20260000

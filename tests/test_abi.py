@@ -329,3 +329,50 @@ def test_fp8_cache_checks():
     prob = P()
     prob.kv_dtype = 7
     assert decode(prob) == fd.FD_ERR_INVALID_ARGUMENT
+
+
+# fd_quantize_keys / fd_decode_sparse rejections (fake addresses, never used).
+K8, SK = 0x60000, 0x70000
+
+
+def sparse(prob, k8=K8, sk=SK, delta=4.0, S=1, **kw):
+    return fd.load_library().fd_decode_sparse(
+        ctypes.byref(prob) if prob is not None else None, kw.get("q", Q), K, V, k8, sk, None,
+        ctypes.c_float(0.125), ctypes.c_float(delta), S, kw.get("out", O), None, None, None, 0,
+        None)
+
+
+def test_sparse_decode_checks():
+    assert sparse(None) == fd.FD_ERR_INVALID_ARGUMENT
+    assert sparse(P(), k8=None) == fd.FD_ERR_INVALID_ARGUMENT
+    assert sparse(P(), sk=None) == fd.FD_ERR_INVALID_ARGUMENT
+    assert sparse(P(), k8=K8 + 8) == fd.FD_ERR_INVALID_ARGUMENT           # codes 16-byte aligned
+    assert sparse(P(), delta=float("nan")) == fd.FD_ERR_INVALID_ARGUMENT
+    assert sparse(P(), delta=-1.0) == fd.FD_ERR_INVALID_ARGUMENT
+    assert sparse(P(), out=None) == fd.FD_ERR_INVALID_ARGUMENT
+    # one split over 70,000 tokens is more than the scan's 1,024 blocks
+    assert sparse(P(L=70000)) == fd.FD_ERR_INVALID_ARGUMENT
+    assert sparse(P(L=70000), S=2) != fd.FD_ERR_INVALID_ARGUMENT
+    paged = P(L=512, bs=16, nb=32, mb=32)
+    assert fd.load_library().fd_decode_sparse(
+        ctypes.byref(paged), Q, K, V, K8, SK, None, ctypes.c_float(0.125), ctypes.c_float(4.0), 1,
+        O, None, None, None, 0, None) == fd.FD_ERR_INVALID_ARGUMENT      # no block table given
+    fp8 = fd.make_problem(1, 8, 8, 128, 512, kv_dtype=fd.FD_KV_FP8_E4M3)
+    assert sparse(fp8) == fd.FD_ERR_UNSUPPORTED
+
+
+def test_quantize_keys_checks():
+    lib = fd.load_library()
+
+    def quant(prob, k=K, k8=K8, sk=SK):
+        return lib.fd_quantize_keys(ctypes.byref(prob) if prob is not None else None, k, None, k8,
+                                    sk, None)
+    assert quant(None) == fd.FD_ERR_INVALID_ARGUMENT
+    assert quant(P(), k8=None) == fd.FD_ERR_INVALID_ARGUMENT
+    assert quant(P(), k=K + 8) == fd.FD_ERR_INVALID_ARGUMENT
+    assert quant(P(L=512, bs=16, nb=32, mb=32)) == fd.FD_ERR_UNSUPPORTED
+    assert quant(fd.make_problem(1, 8, 8, 128, 512, kv_layout=fd.FD_LAYOUT_NHD)) == \
+        fd.FD_ERR_UNSUPPORTED
+    assert quant(fd.make_problem(1, 8, 8, 128, 512, kv_dtype=fd.FD_KV_FP8_E4M3)) == \
+        fd.FD_ERR_UNSUPPORTED
+    assert quant(P(D=96)) == fd.FD_ERR_UNSUPPORTED

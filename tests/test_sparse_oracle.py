@@ -1,0 +1,123 @@
+"""Pins of the sparse-decode oracle (oracle/sparse.py): the low-bit codes, the
+scan's error bound, the top-delta rule's special cases, and the reduction to
+the dense oracle when every block is kept."""
+import numpy as np
+import pytest
+
+import oracle
+from oracle import sparse
+from split_kv_decode_attn_b200 import workloads as wl
+
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+
+def problem(B=3, Hq=8, Hkv=2, D=64, L=300, seed=1, lens=(300, 130, 1)):
+    return wl.make_problem(B, Hq, Hkv, D, L, seed=seed, seqlens=list(lens), nan_pad=True)
+
+
+def f32(bits):
+    return wl.bf16_bits_to_f64(bits).astype(np.float32)
+
+
+def test_key_codes_round_to_the_block_scale():
+    w = problem()
+    k8, sk = sparse.quantize_keys(w.k, w.seqlens)
+    B, Hkv, L, D = w.k.shape
+    assert k8.dtype == np.int8 and k8.shape == w.k.shape and sk.shape == (B, Hkv, 5)
+    assert np.abs(k8.astype(np.int32)).max() <= 127
+    for b in range(B):
+        n = int(w.seqlens[b])
+        for h in range(Hkv):
+            for blk in range(5):
+                r0, r1 = blk * 64, min(L, blk * 64 + 64)
+                rows = np.arange(r0, r1)
+                valid = rows < n
+                codes = k8[b, h, r0:r1].astype(np.float64)
+                assert np.all(codes[~valid] == 0)          # padding (NaN here) takes no part
+                if not valid.any():
+                    assert sk[b, h, blk] == 1.0
+                    continue
+                kv = f32(w.k[b, h, rows[valid]]).astype(np.float64)
+                s = float(sk[b, h, blk])
+                assert s == np.float32(np.abs(kv).max() / np.float32(127))
+                assert np.abs(codes[valid]).max() == 127    # the largest entry maps to 127
+                # half a step, plus the fp32 rounding of the scale and of the quotient
+                assert np.all(np.abs(kv - s * codes[valid]) <= s / 2 * (1 + 1e-5))
+
+
+def test_zero_block_and_query_codes():
+    k = np.zeros((1, 1, 64, 64), np.uint16)
+    k8, sk = sparse.quantize_keys(k)
+    assert np.all(k8 == 0) and sk[0, 0, 0] == 1.0
+    q8, sq = sparse.quantize_query(np.zeros((2, 64), np.uint16))
+    assert np.all(q8 == 0) and np.all(sq == 1.0)
+    w = problem()
+    q8, sq = sparse.quantize_query(w.q)
+    qf = f32(w.q).astype(np.float64)
+    assert np.all(np.abs(q8).max(axis=-1) == 127)
+    assert np.all(np.abs(qf - sq[..., None] * q8) <= sq[..., None] / 2 * (1 + 1e-5))
+
+
+def test_scan_logits_stay_within_the_quantisation_bound():
+    """|s~ - s| <= scale * sum_d (|q_d| dk/2 + |k_d| dq/2 + dq dk/4) plus fp32
+    rounding, with dq, dk the query and block scales."""
+    w = problem(B=1, Hq=4, Hkv=1, D=128, L=256, seed=3, lens=(256,))
+    k8, sk = sparse.quantize_keys(w.k)
+    q8, sq = sparse.quantize_query(w.q)
+    qf = f32(w.q[0]).astype(np.float64)
+    kf = f32(w.k[0, 0]).astype(np.float64)
+    for g in range(4):
+        for j in range(256):
+            dk = float(sk[0, 0, j // 64])
+            approx = float(np.float32(np.float32(np.float32(w.scale) * sq[0, g]) * np.float32(dk))
+                           * np.float32(int(q8[0, g].astype(np.int64) @ k8[0, 0, j].astype(np.int64))))
+            exact = w.scale * qf[g] @ kf[j]
+            bound = w.scale * (np.abs(qf[g]) @ np.full(128, dk / 2) + np.abs(kf[j]).sum() * sq[0, g] / 2
+                               + 128 * sq[0, g] * dk / 4)
+            assert abs(approx - exact) <= bound + 1e-5 * abs(exact) + 1e-6
+
+
+def test_infinite_delta_keeps_everything_and_equals_dense_attention():
+    w = problem(B=3, Hq=8, Hkv=2, D=64, L=300, lens=(300, 130, 0))
+    for S in (1, 3):
+        out, lse, kept = sparse.sparse_decode(w.q, w.k, w.v, w.scale, np.inf, S, w.seqlens)
+        ref, rl = oracle.decode(w.q, w.k, w.v, w.scale, seqlens=w.seqlens)
+        assert np.array_equal(out, ref) and np.array_equal(lse, rl)
+        for b, n in enumerate(w.seqlens):
+            nb = -(-int(n) // 64)
+            assert kept[b, :, :nb].all() and not kept[b, :, nb:].any()
+
+
+def test_one_dominant_block_is_all_that_a_zero_delta_keeps():
+    """A key aligned with every query head of the group, far above the rest:
+    with one split and delta = 0 only its block survives, and the output is
+    close to that key's value row."""
+    w = problem(B=1, Hq=4, Hkv=1, D=128, L=1024, seed=5, lens=(1024,))
+    qf = f32(w.q[0]).astype(np.float64)
+    key = qf.sum(axis=0)
+    key = 24.0 * key / np.linalg.norm(key)
+    k = w.k.copy()
+    k[0, 0, 700] = wl.f64_to_bf16_bits(key)
+    out, lse, kept = sparse.sparse_decode(w.q, k, w.v, w.scale, 0.0, 1)
+    assert kept[0, 0].tolist() == [i == 700 // 64 for i in range(16)]
+    v700 = wl.bf16_bits_to_f64(w.v[0, 0, 700])
+    assert np.abs(out[0] - v700).max() < 0.05
+
+
+def test_more_delta_keeps_more_and_each_split_keeps_its_best_block():
+    w = wl.make_problem(2, 8, 2, 128, 2048, seed=9, seqlens=[2048, 1500])
+    k8, sk = sparse.quantize_keys(w.k, w.seqlens)
+    prev = None
+    for delta in (0.0, 0.5, 1.0, 2.0, 4.0, np.inf):
+        kept = sparse.select_blocks(w.q, k8, sk, w.scale, delta, 4, w.seqlens)
+        if prev is not None:
+            assert np.all(kept >= prev)                    # monotone in delta
+        prev = kept
+    kept0 = sparse.select_blocks(w.q, k8, sk, w.scale, 0.0, 4, w.seqlens)
+    chunk = sparse.chunk_for(2048, 4) // 64
+    for b in range(2):
+        nb = -(-int(w.seqlens[b]) // 64)
+        for h in range(2):
+            for s0 in range(0, nb, chunk):
+                assert kept0[b, h, s0:min(nb, s0 + chunk)].any()
+            assert not kept0[b, h, nb:].any()
