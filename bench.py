@@ -69,6 +69,9 @@ def parse_args():
                     help="cache dimension order (heads outside tokens, or tokens outside heads)")
     ap.add_argument("--shard-sequence", action="store_true",
                     help="sequence-parallel: the ranks split one history (strong scaling)")
+    ap.add_argument("--sparse", action="store_true",
+                    help="sparse decode (low-bit scan + top-delta) on a peaked 256K workload")
+    ap.add_argument("--delta", type=float, default=8.0, help="top-delta threshold (nats)")
     ap.add_argument("--crossover", action="store_true",
                     help="planner sweep: split-count ladders over batch, length, element type")
     ap.add_argument("--no-sweep", action="store_true")
@@ -539,6 +542,96 @@ def sweep(torch, fd, device):
     return rows
 
 
+def run_sparse(args):
+    """fd_decode_sparse against fd_decode on the peaked 256K shape (B=1, Hq=32,
+    Hkv=8, D=128).  Workload "peaked" (the default workload name maps here to
+    the group-peaked keys, which dominate every head of a group) or the
+    benchmark's own peaked workload (--workload peaked: keys that dominate one
+    head per group).  The key codes are made once, outside the timed region
+    (in a decode loop they change only where tokens are appended).  Reports
+    the sparse call's time, the bytes it must read (codes of every token plus
+    K and V of the kept blocks) against the HBM peak, the dense call's time
+    and the speed-up."""
+    import numpy as np
+    import torch
+    import split_kv_decode_attn_b200 as fd
+    from split_kv_decode_attn_b200 import workloads as wl
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    fd.load_library()
+    w = wl.config(5) if args.workload == "peaked" else wl.peaked_group()
+    copies = 2
+    call = Call(torch, fd, w, device, None, copies)
+    S = call.S
+    nblk = -(-w.max_len // 64)
+    k8s, sks = [], []
+    for c in range(copies):
+        k8 = torch.empty(w.k.shape, dtype=torch.int8, device=device)
+        sk = torch.empty((w.B, w.Hkv, nblk), dtype=torch.float32, device=device)
+        assert fd.fd_quantize_keys(call.prob, call.ks[c], call.seqlens, k8, sk) == 0
+        k8s.append(k8)
+        sks.append(sk)
+    kept = torch.empty((w.B, w.Hkv, nblk), dtype=torch.uint8, device=device)
+    out_s = torch.empty_like(call.out)
+    lse_s = torch.empty_like(call.lse)
+    state = {"i": 0}
+
+    def sparse_call():
+        c = state["i"] % copies
+        state["i"] += 1
+        st = fd.fd_decode_sparse(call.prob, call.q, call.ks[c], call.vs[c], k8s[c], sks[c],
+                                 call.seqlens, w.scale, args.delta, S, out_s, lse_s, kept,
+                                 call.ws, call.wbytes, call.stream)
+        if st != 0:
+            raise RuntimeError(f"fd_decode_sparse: {fd.fd_status_string(st)}")
+
+    steps, warmup = args.steps, args.warmup
+    sampler = ClockSampler(device.index)
+    sampler.start()
+    ms_sparse = timed(torch, sparse_call, steps, warmup)
+    clocks = sampler.stop()
+    ms_dense = timed(torch, call, steps, warmup)
+    us_sparse = ms_sparse * 1e3 / steps
+    us_dense = ms_dense * 1e3 / steps
+    # one more call of each on the same copy, for the kept share and the gap
+    state["i"] = 0
+    sparse_call()
+    call.i = 0
+    call()
+    torch.cuda.synchronize()
+    assert fd.fd_check_device_error() == 0
+    kept_np = kept.cpu().numpy().astype(bool)
+    share = float(kept_np.mean())
+    gap = float((out_s.float() - call.out.float()).abs().max())
+    lse_gap = float((lse_s - call.lse).abs().max())
+    n_tok = int(w.lengths().sum())
+    read = n_tok * w.Hkv * w.D + int(kept_np.sum()) * 64 * w.D * 4   # codes + kept K, V
+    dense_bytes = w.kv_bytes()
+    peak, peak_kind = measured_peak()
+    achieved = read / (us_sparse * 1e-6) / 1e9
+    print(json.dumps({
+        "metric": "sparse decode µs/call and bytes-read GB/s (fraction of B200 HBM roofline)",
+        "value": round(achieved, 1), "unit": "GB/s", "n_gpus": 1, "steps": steps,
+        "warmup": warmup, "us_per_call": round(us_sparse, 3), "higher_is_better": True,
+        "dtype": "bf16 attention, int8 scan", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+                   "max_len": w.max_len, "num_splits": S, "delta": args.delta,
+                   "l2": f"inputs rotate over {copies} copies of K, V and the codes"},
+        "kept_block_share": round(share, 5),
+        "bytes_read_per_call": read, "dense_kv_bytes_per_call": dense_bytes,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                     "traffic": None},
+        "dense": {"us_per_call": round(us_dense, 3),
+                  "GB/s": round(dense_bytes / (us_dense * 1e-6) / 1e9, 1)},
+        "speedup_vs_dense": round(us_dense / us_sparse, 3),
+        "dense_equivalent_GB/s": round(dense_bytes / (us_sparse * 1e-6) / 1e9, 1),
+        "vs_dense_max_abs_dout": gap, "vs_dense_max_abs_dlse": lse_gap,
+        "gpu_launches": steps * call.launches_per_call,
+        "clocks": clocks,
+    }), flush=True)
+
+
 def run_sharded(args):
     """Sequence-parallel decode of the CodeLlama-34B-shaped workload: rank r
     holds tokens [r*L/N, (r+1)*L/N) of every KV head.  A step is the local
@@ -750,6 +843,8 @@ def main():
         crossover(args)
     elif args.shard_sequence:
         run_sharded(args)
+    elif args.sparse:
+        run_sparse(args)
     else:
         run_fd(args)
 

@@ -292,8 +292,11 @@ FD_API fd_status fd_quantize_keys(const fd_problem* p, const void* k_cache,
  *   kept          [B, Hkv, ceil(max_len / 64)] uint8 out (1 = kept), or NULL.
  *                 Blocks at or past a sequence's length are not written.
  * Other arguments are those of fd_decode with a contiguous head-major bf16
- * cache. The split count must make the chunk at most 65,536 tokens
- * (FD_ERR_INVALID_ARGUMENT otherwise). Results are deterministic. */
+ * cache and D = 128 (FD_ERR_UNSUPPORTED otherwise). The split count must make
+ * the chunk at most 16,384 tokens (FD_ERR_INVALID_ARGUMENT otherwise). The
+ * codes stream through the split kernel's tile pipeline (TMA, 256 tokens per
+ * stage) and the dot products run on int8 tensor cores. Results are
+ * deterministic. */
 FD_API fd_status fd_decode_sparse(const fd_problem* p, const void* q, const void* k_cache,
                                   const void* v_cache, const int8_t* k8,
                                   const float* k8_scale, const int32_t* seqlens, float scale,

@@ -304,8 +304,9 @@ constexpr int split_stages() {
 
 template <int D, int NB, int MODE, bool PAGED, bool FP8 = false, bool DEEP = false,
           bool SPARSE = false>
-fd_status launch_split(const CUtensorMap& tk, const CUtensorMap& tv, const fd::SplitArgs& a,
-                       int n_splits, int Hkv, int B, cudaStream_t stream) {
+fd_status launch_split(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tc,
+                       const fd::SplitArgs& a, int n_splits, int Hkv, int B,
+                       cudaStream_t stream) {
   constexpr int STAGES = split_stages<D, FP8, DEEP>();
   using L = fd::SplitSmem<D, NB, STAGES, FP8, SPARSE>;
   auto kern = fd::fd_split_kernel<D, NB, MODE, PAGED, STAGES, FP8, SPARSE>;
@@ -331,7 +332,7 @@ fd_status launch_split(const CUtensorMap& tk, const CUtensorMap& tv, const fd::S
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, tk, tv, a) != cudaSuccess) return FD_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, tk, tv, tc, a) != cudaSuccess) return FD_ERR_CUDA;
   return FD_OK;
 }
 
@@ -357,27 +358,27 @@ fd_status launch_combine(const fd::SplitArgs& a, int B, cudaStream_t stream) {
 // sparse: the low-bit scan and top-delta selection run first (contiguous
 // bf16 caches only).
 template <int D, int NB, int MODE, bool PAGED, bool FP8 = false>
-fd_status launch_call(const CUtensorMap& tk, const CUtensorMap& tv, const fd::SplitArgs& a,
-                      int n_splits, int Hkv, int B, bool deep, bool sparse, cudaStream_t s) {
+fd_status launch_call(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tc,
+                      const fd::SplitArgs& a, int n_splits, int Hkv, int B, bool deep,
+                      bool sparse, cudaStream_t s) {
   fd_status r = FD_ERR_UNSUPPORTED;
   if constexpr (!PAGED && !FP8) {
     if (sparse) {
-      if constexpr (D == 128)
-        r = deep ? launch_split<D, NB, MODE, PAGED, FP8, true, true>(tk, tv, a, n_splits, Hkv, B, s)
-                 : launch_split<D, NB, MODE, PAGED, FP8, false, true>(tk, tv, a, n_splits, Hkv, B, s);
-      else
-        r = launch_split<D, NB, MODE, PAGED, FP8, false, true>(tk, tv, a, n_splits, Hkv, B, s);
-      if (r == FD_OK && n_splits > 1) r = launch_combine<D>(a, B, s);
+      if constexpr (D == 128) {
+        r = deep ? launch_split<D, NB, MODE, PAGED, FP8, true, true>(tk, tv, tc, a, n_splits, Hkv, B, s)
+                 : launch_split<D, NB, MODE, PAGED, FP8, false, true>(tk, tv, tc, a, n_splits, Hkv, B, s);
+        if (r == FD_OK && n_splits > 1) r = launch_combine<D>(a, B, s);
+      }
       return r;
     }
   }
   if (sparse) return FD_ERR_UNSUPPORTED;
   if constexpr (D == 128 && !FP8) {
-    r = deep ? launch_split<D, NB, MODE, PAGED, FP8, true>(tk, tv, a, n_splits, Hkv, B, s)
-             : launch_split<D, NB, MODE, PAGED, FP8, false>(tk, tv, a, n_splits, Hkv, B, s);
+    r = deep ? launch_split<D, NB, MODE, PAGED, FP8, true>(tk, tv, tc, a, n_splits, Hkv, B, s)
+             : launch_split<D, NB, MODE, PAGED, FP8, false>(tk, tv, tc, a, n_splits, Hkv, B, s);
   } else {
     (void)deep;
-    r = launch_split<D, NB, MODE, PAGED, FP8, false>(tk, tv, a, n_splits, Hkv, B, s);
+    r = launch_split<D, NB, MODE, PAGED, FP8, false>(tk, tv, tc, a, n_splits, Hkv, B, s);
   }
   if (r == FD_OK && n_splits > 1) r = launch_combine<D>(a, B, s);
   return r;
@@ -389,19 +390,21 @@ fd_status dispatch_split_fp8(int G, const CUtensorMap& tk, const CUtensorMap& tv
                              const fd::SplitArgs& a, int n_splits, int Hkv, int B,
                              cudaStream_t s) {
   if (G <= 8)
-    return launch_call<128, 1, fd::kHi, PAGED, true>(tk, tv, a, n_splits, Hkv, B, false, false, s);
-  return launch_call<128, 2, fd::kHi, PAGED, true>(tk, tv, a, n_splits, Hkv, B, false, false, s);
+    return launch_call<128, 1, fd::kHi, PAGED, true>(tk, tv, tk, a, n_splits, Hkv, B, false,
+                                                     false, s);
+  return launch_call<128, 2, fd::kHi, PAGED, true>(tk, tv, tk, a, n_splits, Hkv, B, false, false,
+                                                   s);
 }
 
 template <int D, bool PAGED>
 fd_status dispatch_split(int G, const CUtensorMap& tk, const CUtensorMap& tv,
-                         const fd::SplitArgs& a, int n_splits, int Hkv, int B, bool deep,
-                         bool sparse, cudaStream_t s) {
+                         const CUtensorMap& tc, const fd::SplitArgs& a, int n_splits, int Hkv,
+                         int B, bool deep, bool sparse, cudaStream_t s) {
   if (G <= 4)
-    return launch_call<D, 1, fd::kDup, PAGED>(tk, tv, a, n_splits, Hkv, B, deep, sparse, s);
+    return launch_call<D, 1, fd::kDup, PAGED>(tk, tv, tc, a, n_splits, Hkv, B, deep, sparse, s);
   if (G == 8)
-    return launch_call<D, 1, fd::kHiLo, PAGED>(tk, tv, a, n_splits, Hkv, B, deep, sparse, s);
-  return launch_call<D, 2, fd::kHiLo, PAGED>(tk, tv, a, n_splits, Hkv, B, deep, sparse, s);
+    return launch_call<D, 1, fd::kHiLo, PAGED>(tk, tv, tc, a, n_splits, Hkv, B, deep, sparse, s);
+  return launch_call<D, 2, fd::kHiLo, PAGED>(tk, tv, tc, a, n_splits, Hkv, B, deep, sparse, s);
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -474,7 +477,7 @@ fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
       !aligned(block_table, 4))
     return FD_ERR_INVALID_ARGUMENT;
   if (sp) {
-    if (paged || fp8) return FD_ERR_UNSUPPORTED;
+    if (paged || fp8 || p->D != 128 || p->kv_layout != FD_LAYOUT_HND) return FD_ERR_UNSUPPORTED;
     if (!sp->k8 || !sp->k8_scale || !aligned(sp->k8, 16) || !aligned(sp->k8_scale, 4) ||
         std::isnan(sp->delta) || sp->delta < 0.f)
       return FD_ERR_INVALID_ARGUMENT;
@@ -509,6 +512,12 @@ fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
   const int box_rows = paged ? std::min(p->block_size, fd::kTile) : fd::kTile;
   if (cached_cache_map(&tk, MapKey{k_cache, rows, planes, D, Hkv, layout, box_rows, dev, fp8}) != FD_OK ||
       cached_cache_map(&tv, MapKey{v_cache, rows, planes, D, Hkv, layout, box_rows, dev, fp8}) != FD_OK)
+    return FD_ERR_CUDA;
+  // Sparse: the int8 key codes, read kScanTilesPerStage blocks per box (one
+  // 128-byte row per token, as an fp8 cache).
+  CUtensorMap tc{};
+  if (sp && cached_cache_map(&tc, MapKey{sp->k8, rows, planes, D, Hkv, layout,
+                                         fd::kScanTilesPerStage * fd::kTile, dev, true}) != FD_OK)
     return FD_ERR_CUDA;
 
   fd::SplitArgs a{};
@@ -555,11 +564,12 @@ fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
     r = paged ? dispatch_split_fp8<true>(G, tk, tv, a, n_splits, Hkv, B, s)
               : dispatch_split_fp8<false>(G, tk, tv, a, n_splits, Hkv, B, s);
   else if (D == 128)
-    r = paged ? dispatch_split<128, true>(G, tk, tv, a, n_splits, Hkv, B, deep, false, s)
-              : dispatch_split<128, false>(G, tk, tv, a, n_splits, Hkv, B, deep, sp != nullptr, s);
+    r = paged ? dispatch_split<128, true>(G, tk, tv, tk, a, n_splits, Hkv, B, deep, false, s)
+              : dispatch_split<128, false>(G, tk, tv, sp ? tc : tk, a, n_splits, Hkv, B, deep,
+                                           sp != nullptr, s);
   else
-    r = paged ? dispatch_split<64, true>(G, tk, tv, a, n_splits, Hkv, B, deep, false, s)
-              : dispatch_split<64, false>(G, tk, tv, a, n_splits, Hkv, B, deep, sp != nullptr, s);
+    r = paged ? dispatch_split<64, true>(G, tk, tv, tk, a, n_splits, Hkv, B, deep, false, s)
+              : dispatch_split<64, false>(G, tk, tv, tk, a, n_splits, Hkv, B, deep, false, s);
   return r;
 }
 

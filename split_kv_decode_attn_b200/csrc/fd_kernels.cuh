@@ -78,8 +78,10 @@ struct SplitArgs {
   float delta;                  // top-delta threshold, natural-log units
 };
 
-// Longest split, in 64-token blocks, that the sparse scan handles.
-constexpr int kMaxSparseTiles = 1024;
+// Longest split, in 64-token blocks, that the sparse scan handles, and the
+// blocks one scan stage carries (one TMA box of 256 code rows).
+constexpr int kMaxSparseTiles = 256;
+constexpr int kScanTilesPerStage = 4;
 
 // Token of row s (0..15) of the fp8 score MMA within a warp's 16-token slice:
 // rows 2t, 2t+1 -> tokens 4t, 4t+1 and rows 8+2t, 8+2t+1 -> tokens 4t+2, 4t+3.
@@ -196,9 +198,14 @@ struct SplitSmem {
   static constexpr int kTileBytes = kHalves * kHalfBytes;
   static constexpr int kStageBytes = 2 * kTileBytes;   // K tile + V tile
   static constexpr int kBarOffset = STAGES * kStageBytes;
-  // + error flag; sparse: + the kept-tile list (uint16) and its length
+  // + error flag; sparse: + the kept-tile list (uint16) and its length, the
+  // per-head thresholds and the block maxima [kMaxSparseTiles][NB * 8]
   static constexpr int kListOffset = kBarOffset + 2 * STAGES * 8 + 16;
-  static constexpr int kBytes = kListOffset + (SPARSE ? 2 * kMaxSparseTiles + 16 : 0);
+  static constexpr int kCountOffset = kListOffset + 2 * kMaxSparseTiles;
+  static constexpr int kThrOffset = kCountOffset + 16;
+  static constexpr int kBmaxOffset = kThrOffset + 4 * NB * 8;
+  static constexpr int kBytes =
+      SPARSE ? kBmaxOffset + 4 * kMaxSparseTiles * NB * 8 : kListOffset;
   static constexpr int kDynamicBytes = kBytes + 1024;  // room to align to 1 KB
   // Epilogue scratch, laid over the drained pipeline buffers (floats):
   static constexpr int kNcol = NB * 8;
@@ -214,120 +221,124 @@ struct SplitSmem {
   static_assert(kScratchFloats * 4 <= kBarOffset, "epilogue scratch must fit the pipeline buffers");
 };
 
-// Sparse decode, selection step ("Faster Than Flash: Exploiting Attention
-// Sparsity for Efficient Long-Context Decoding", abstract: a low-bit scan of
-// the keys selects blocks by a top-delta rule that each unit of work applies
-// on its own, with no global synchronisation).  All threads of the CTA take
-// part, before the tile pipeline starts, using its buffers as scratch.
-//  1. q of each head of the group to int8: sq = max|q| / 127, q8 = rint(q/sq).
-//  2. For every 64-token block of the split and every head: the largest
-//     approximate logit ((scale * sq) * sk) * (q8 . k8), the dot product exact
-//     in integers (dp4a) and each product rounded to fp32 in that order.
-//  3. Per head M = the split's largest block maximum; a block is kept when
-//     some head has a block maximum >= M - delta.
-// Returns the number of kept blocks; `list` gets their indices in order.
-template <int D, int GMAX>
-__device__ __forceinline__ int sparse_select(const SplitArgs& a, uint8_t* scratch, uint16_t* list,
-                                          int* n_kept, int b, int kvh, int h0, int start,
-                                          int end, int n_tiles) {
-  static_assert(D % 128 == 0 || D == 64, "head dim");
-  int8_t* q8 = reinterpret_cast<int8_t*>(scratch);                 // [GMAX][D]
-  float* qs = reinterpret_cast<float*>(scratch + GMAX * D);        // [GMAX]: scale * sq
-  float* thr = qs + GMAX;                                          // [GMAX]
-  float* bmax = thr + GMAX;                                        // [n_tiles][GMAX]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int kWarps = kThreads / 32;
-  constexpr int VPL = D / 32;                                      // q entries per lane
-
-  for (int g = warp; g < a.G; g += kWarps) {
-    const __nv_bfloat16* qrow = a.q + (static_cast<size_t>(b) * a.Hq + h0 + g) * D + lane * VPL;
-    float v[VPL];
+// Sparse decode, selection ("Faster Than Flash: Exploiting Attention
+// Sparsity for Efficient Long-Context Decoding", abstract: a scan of low-bit
+// keys selects blocks by a top-delta rule that each unit of work applies on
+// its own, with no global synchronisation).  The consumer warps' part of the
+// scan: the int8 key codes of the split stream through the same mbarrier ring
+// as the K/V tiles, kScanTilesPerStage blocks per stage, and warp w takes
+// block w of each stage.  Per block and head the largest approximate logit
+// ((scale * sq) * sk) * (q8 . k8) goes to bmax: the dot products are exact
+// (int8 tensor cores, int32 accumulation), each product is rounded to fp32
+// in that order, and q8 = rint(q / sq) with sq = max |q| / 127.
+template <int D, int NB, int STAGES, int STAGE_BYTES>
+__device__ __forceinline__ bool sparse_scan_consumer(const SplitArgs& a, uint32_t smem_base,
+                                                     uint32_t bar_full, uint32_t bar_empty,
+                                                     float* bmax, int warp, int lane, int b,
+                                                     int h0, int start, int end, int n_tiles,
+                                                     int n_scan) {
+  static_assert(D == 128, "the scan reads 128-byte code rows");
+  constexpr int KSTEPS = D / 32;
+  static_assert(STAGE_BYTES >= kScanTilesPerStage * kTile * D, "a scan stage fits a ring stage");
+  // B fragments of q8 (k = head dim, n = head): lane (g, t) holds entries
+  // 32c + 4t .. +3 and 32c + 16 + 4t .. +3 of head nb*8 + g.
+  uint32_t qb[NB][KSTEPS][2];
+  float qsc[NB][2];     // scale * sq of this lane's two score columns
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) {
+    const int head = nb * 8 + (lane >> 2);
+    const bool live = head < a.G;
+    const __nv_bfloat16* qrow = a.q + (static_cast<size_t>(b) * a.Hq + h0 + (live ? head : 0)) * D;
+    float v[KSTEPS][2][4];
     float amax = 0.f;
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      v[i] = __bfloat162float(qrow[i]);
-      amax = fmaxf(amax, fabsf(v[i]));
-    }
+    for (int c = 0; c < KSTEPS; ++c)
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      for (int h = 0; h < 2; ++h) {
+        const uint2 raw = live ? *reinterpret_cast<const uint2*>(qrow + 32 * c + 16 * h + 4 * (lane & 3))
+                               : make_uint2(0u, 0u);
+        const float2 f01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+        const float2 f23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+        v[c][h][0] = f01.x;
+        v[c][h][1] = f01.y;
+        v[c][h][2] = f23.x;
+        v[c][h][3] = f23.y;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) amax = fmaxf(amax, fabsf(v[c][h][i]));
+      }
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
     const float sq = amax > 0.f ? __fdiv_rn(amax, 127.f) : 1.f;
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const int c = __float2int_rn(__fdiv_rn(v[i], sq));
-      q8[g * D + lane * VPL + i] = static_cast<int8_t>(max(-127, min(127, c)));
-    }
-    if (lane == 0) qs[g] = __fmul_rn(a.scale, sq);
-  }
-  __syncthreads();
-
-  // One warp per block, one token row per lane at a time.
-  const int8_t* k8 = a.k8 + (static_cast<size_t>(b) * a.Hkv + kvh) * a.max_len * D;
-  const size_t srow = (static_cast<size_t>(b) * a.Hkv + kvh) * a.n_blocks;
-  const int blk0 = start / kTile;
-  for (int i = warp; i < n_tiles; i += kWarps) {
-    const float sk = a.k8_scale[srow + blk0 + i];
-    float m[GMAX];
+    for (int c = 0; c < KSTEPS; ++c)
 #pragma unroll
-    for (int g = 0; g < GMAX; ++g) m[g] = -INFINITY;
-    for (int r = lane; r < kTile; r += 32) {
-      const int t = start + i * kTile + r;
-      if (t >= end) break;
-      const int4* row = reinterpret_cast<const int4*>(k8 + static_cast<size_t>(t) * D);
-      int4 kw[D / 16];
+      for (int h = 0; h < 2; ++h) {
+        uint32_t word = 0;
 #pragma unroll
-      for (int w = 0; w < D / 16; ++w) kw[w] = __ldg(row + w);
-#pragma unroll
-      for (int g = 0; g < GMAX; ++g) {
-        if (g < a.G) {
-          const int4* qw = reinterpret_cast<const int4*>(q8 + g * D);
-          int acc = 0;
-#pragma unroll
-          for (int w = 0; w < D / 16; ++w) {
-            const int4 qv = qw[w];
-            acc = __dp4a(kw[w].x, qv.x, acc);
-            acc = __dp4a(kw[w].y, qv.y, acc);
-            acc = __dp4a(kw[w].z, qv.z, acc);
-            acc = __dp4a(kw[w].w, qv.w, acc);
-          }
-          m[g] = fmaxf(m[g], __fmul_rn(__fmul_rn(qs[g], sk), __int2float_rn(acc)));
+        for (int i = 0; i < 4; ++i) {
+          const int code = max(-127, min(127, __float2int_rn(__fdiv_rn(v[c][h][i], sq))));
+          word |= (static_cast<uint32_t>(code) & 0xffu) << (8 * i);
         }
+        qb[nb][c][h] = word;
       }
-    }
-#pragma unroll
-    for (int g = 0; g < GMAX; ++g) {
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1)
-        m[g] = fmaxf(m[g], __shfl_xor_sync(0xffffffffu, m[g], off));
-      if (lane == 0 && g < a.G) bmax[i * GMAX + g] = m[g];
-    }
+    const float qs = __fmul_rn(a.scale, sq);
+    qsc[nb][0] = __shfl_sync(0xffffffffu, qs, 8 * (lane & 3));
+    qsc[nb][1] = __shfl_sync(0xffffffffu, qs, 8 * (lane & 3) + 4);
   }
-  __syncthreads();
 
-  if (threadIdx.x < a.G) {
-    float M = -INFINITY;
-    for (int i = 0; i < n_tiles; ++i) M = fmaxf(M, bmax[i * GMAX + threadIdx.x]);
-    thr[threadIdx.x] = __fsub_rn(M, a.delta);
-  }
-  __syncthreads();
-
-  if (warp == 0) {
-    int count = 0;
-    for (int i0 = 0; i0 < n_tiles; i0 += 32) {
-      const int i = i0 + lane;
-      bool keep = false;
-      if (i < n_tiles) {
-        for (int g = 0; g < a.G; ++g) keep |= bmax[i * GMAX + g] >= thr[g];
-        if (a.kept_out) a.kept_out[srow + blk0 + i] = keep ? 1 : 0;
+  const size_t srow = (static_cast<size_t>(b) * a.Hkv + (h0 / a.G)) * a.n_blocks + start / kTile;
+  const int g = lane >> 2, t = lane & 3;
+  for (int j = 0; j < n_scan; ++j) {
+    const int s = j % STAGES, k = j / STAGES;
+    const bool ok = mbar_wait(bar_full + 8 * s, k & 1, kWaitLimitNs);
+    if (!__all_sync(0xffffffffu, ok)) return false;
+    const int blk = kScanTilesPerStage * j + warp;
+    if (blk < n_tiles) {
+      const float sk = a.k8_scale[srow + blk];
+      const uint32_t sb = smem_base + s * STAGE_BYTES;
+      float mcol[NB][2];
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) mcol[nb][0] = mcol[nb][1] = -INFINITY;
+#pragma unroll
+      for (int mg = 0; mg < kTile / 16; ++mg) {
+        int acc[NB][4];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[nb][i] = 0;
+        const uint32_t row = warp * kTile + mg * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+#pragma unroll
+        for (int kp = 0; kp < KSTEPS; ++kp) {
+          const uint32_t chunk16 = 2 * kp + (lane >> 4);
+          uint32_t r[4];
+          ldmatrix_x4(sb + row * 128 + ((chunk16 ^ (row & 7)) << 4), r[0], r[1], r[2], r[3]);
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) mma_s8_16832(acc[nb], r, qb[nb][kp][0], qb[nb][kp][1]);
+        }
+        const int tok = start + blk * kTile + mg * 16 + g;   // C rows g and g + 8
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const bool valid = (i < 2 ? tok : tok + 8) < end;
+            const float x = __fmul_rn(__fmul_rn(qsc[nb][i & 1], sk), __int2float_rn(acc[nb][i]));
+            mcol[nb][i & 1] = fmaxf(mcol[nb][i & 1], valid ? x : -INFINITY);
+          }
       }
-      const unsigned mask = __ballot_sync(0xffffffffu, keep);
-      if (keep) list[count + __popc(mask & ((1u << lane) - 1u))] = static_cast<uint16_t>(i);
-      count += __popc(mask);
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+#pragma unroll
+          for (int off = 4; off < 32; off <<= 1)
+            mcol[nb][c] = fmaxf(mcol[nb][c], __shfl_xor_sync(0xffffffffu, mcol[nb][c], off));
+          if (g == 0) bmax[blk * NB * 8 + nb * 8 + 2 * t + c] = mcol[nb][c];
+        }
     }
-    if (lane == 0) *n_kept = count;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_empty + 8 * s);
   }
-  __syncthreads();
-  return *n_kept;
+  return true;
 }
 
 // Consumer warps of the split kernel: scores, online softmax and P.V over the
@@ -340,7 +351,7 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
                                                 uint32_t bar_empty, volatile int* cta_error,
                                                 int warp, int lane, int b, int h0, int split,
                                                 int start, int end, int n_tiles, int n_parts,
-                                                const uint16_t* list) {
+                                                const uint16_t* list, int it_base) {
   using L = SplitSmem<D, NB, STAGES, FP8, SPARSE>;
   constexpr int KSTEPS = D / 16;   // k-steps of the score MMA (over D)
   constexpr int DBLK = D / 16;     // m-blocks of the P.V MMA (over D)
@@ -421,7 +432,8 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
   bool failed = false;
 
   for (int it = 0; it < n_tiles; ++it) {
-    const int s = it % STAGES, k = it / STAGES;
+    const int ig = it_base + it;                 // ring use, after any scan stages
+    const int s = ig % STAGES, k = ig / STAGES;
     const bool ok = mbar_wait(bar_full + 8 * s, k & 1, kWaitLimitNs);
     if (!__all_sync(0xffffffffu, ok)) {
       failed = true;
@@ -738,7 +750,9 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
 template <int D, int NB, int MODE, bool PAGED, int STAGES, bool FP8, bool SPARSE = false>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     fd_split_kernel(const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const SplitArgs a) {
+                    const __grid_constant__ CUtensorMap tmV,
+                    const __grid_constant__ CUtensorMap tmC,   // sparse: int8 key codes
+                    const SplitArgs a) {
   using L = SplitSmem<D, NB, STAGES, FP8, SPARSE>;
   static_assert(!SPARSE || (!PAGED && !FP8), "sparse decode: contiguous bf16 caches");
   static_assert(MODE != kDup || NB == 1, "duplicated columns need one column block");
@@ -810,24 +824,86 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     return;
   }
 
-  // Tiles the pipeline runs: all of the split's, or the kept ones in order.
+  // Tiles the pipeline runs: all of the split's, or the kept ones in order,
+  // after it_base ring uses by the sparse scan.
   int n_work = n_tiles;
+  int it_base = 0;
   uint16_t* list = reinterpret_cast<uint16_t*>(smem + L::kListOffset);
-  if constexpr (SPARSE)
-    n_work = sparse_select<D, NB * 8>(a, smem, list,
-                                      reinterpret_cast<int*>(smem + L::kListOffset +
-                                                             2 * kMaxSparseTiles),
-                                      b, kvh, h0, start, end, n_tiles);
+  if constexpr (SPARSE) {
+    const int n_scan = (n_tiles + kScanTilesPerStage - 1) / kScanTilesPerStage;
+    float* bmax = reinterpret_cast<float*>(smem + L::kBmaxOffset);
+    float* thr = reinterpret_cast<float*>(smem + L::kThrOffset);
+    int* count = reinterpret_cast<int*>(smem + L::kCountOffset);
+    bool ok = true;
+    if (warp == kConsumerWarps) {
+      // Producer: one TMA box of kScanTilesPerStage blocks of codes per stage.
+      const uint64_t policy = policy_evict_first();
+      for (int j = 0; j < n_scan; ++j) {
+        const int s = j % STAGES, k = j / STAGES;
+        if (k > 0) ok = mbar_wait(bar_empty + 8 * s, (k - 1) & 1, kWaitLimitNs);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar_full + 8 * s, kScanTilesPerStage * kTile * D);
+          tma_load_5d(smem_base + s * L::kStageBytes, &tmC, bar_full + 8 * s, 0, kvh,
+                      start + j * kScanTilesPerStage * kTile, 0, b, policy);
+        }
+        __syncwarp();
+      }
+      if (!ok && lane == 0) {  // no code copy may still be landing when the CTA retires
+        for (int j = n_scan > STAGES ? n_scan - STAGES : 0; j < n_scan; ++j)
+          if (!mbar_wait(bar_full + 8 * (j % STAGES), (j / STAGES) & 1, kWaitLimitNs))
+            raise_device_error(2u);
+      }
+    } else {
+      ok = sparse_scan_consumer<D, NB, STAGES, L::kStageBytes>(a, smem_base, bar_full, bar_empty,
+                                                             bmax, warp, lane, b, h0, start, end,
+                                                             n_tiles, n_scan);
+    }
+    if (!ok && lane == 0) {
+      raise_device_error(1u);
+      *cta_error = 1;
+    }
+    __syncthreads();
+    if (*cta_error) return;
+    // Per head: M = the split's largest block maximum; the threshold M - delta.
+    if (threadIdx.x < a.G) {
+      float M = -INFINITY;
+      for (int i = 0; i < n_tiles; ++i) M = fmaxf(M, bmax[i * NB * 8 + threadIdx.x]);
+      thr[threadIdx.x] = __fsub_rn(M, a.delta);
+    }
+    __syncthreads();
+    // Kept blocks in order: some head's block maximum reaches its threshold.
+    if (warp == 0) {
+      const size_t srow = (static_cast<size_t>(b) * a.Hkv + kvh) * a.n_blocks + start / kTile;
+      int kept = 0;
+      for (int i0 = 0; i0 < n_tiles; i0 += 32) {
+        const int i = i0 + lane;
+        bool keep = false;
+        if (i < n_tiles) {
+          for (int g = 0; g < a.G; ++g) keep |= bmax[i * NB * 8 + g] >= thr[g];
+          if (a.kept_out) a.kept_out[srow + i] = keep ? 1 : 0;
+        }
+        const unsigned mask = __ballot_sync(0xffffffffu, keep);
+        if (keep) list[kept + __popc(mask & ((1u << lane) - 1u))] = static_cast<uint16_t>(i);
+        kept += __popc(mask);
+      }
+      if (lane == 0) *count = kept;
+    }
+    __syncthreads();
+    n_work = *count;
+    it_base = n_scan;
+  }
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------- producer
     // Every lane waits (the decision is made warp-uniform); lane 0 issues.
     const uint64_t policy = policy_evict_first();
-    int issued = 0;
+    int issued = it_base;   // ring uses so far (the sparse scan's stages)
     bool ok = true;
     if constexpr (!PAGED) {
       for (int it = 0; it < n_work; ++it) {
-        const int s = it % STAGES, k = it / STAGES;
+        const int ig = it_base + it;
+        const int s = ig % STAGES, k = ig / STAGES;
         if (k > 0) ok = mbar_wait(bar_empty + 8 * s, (k - 1) & 1, kWaitLimitNs);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         if (lane == 0) {
@@ -900,7 +976,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     // ------------------------------------------------------------- consumers
     split_consumers<D, NB, MODE, STAGES, FP8, SPARSE>(a, smem, smem_base, bar_full, bar_empty,
                                                       cta_error, warp, lane, b, h0, split,
-                                                      start, end, n_work, n_parts, list);
+                                                      start, end, n_work, n_parts, list,
+                                                      it_base);
   }
 }
 

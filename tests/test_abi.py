@@ -350,9 +350,12 @@ def test_sparse_decode_checks():
     assert sparse(P(), delta=float("nan")) == fd.FD_ERR_INVALID_ARGUMENT
     assert sparse(P(), delta=-1.0) == fd.FD_ERR_INVALID_ARGUMENT
     assert sparse(P(), out=None) == fd.FD_ERR_INVALID_ARGUMENT
-    # one split over 70,000 tokens is more than the scan's 1,024 blocks
-    assert sparse(P(L=70000)) == fd.FD_ERR_INVALID_ARGUMENT
-    assert sparse(P(L=70000), S=2) != fd.FD_ERR_INVALID_ARGUMENT
+    # one split over 20,000 tokens is more than the scan's 256 blocks
+    assert sparse(P(L=20000)) == fd.FD_ERR_INVALID_ARGUMENT
+    assert sparse(P(L=20000), S=2) != fd.FD_ERR_INVALID_ARGUMENT
+    assert sparse(P(D=64)) == fd.FD_ERR_UNSUPPORTED
+    assert sparse(fd.make_problem(1, 8, 8, 128, 512, kv_layout=fd.FD_LAYOUT_NHD)) == \
+        fd.FD_ERR_UNSUPPORTED
     paged = P(L=512, bs=16, nb=32, mb=32)
     assert fd.load_library().fd_decode_sparse(
         ctypes.byref(paged), Q, K, V, K8, SK, None, ctypes.c_float(0.125), ctypes.c_float(4.0), 1,

@@ -73,12 +73,12 @@ def test_quantize_keys_bit_exact(D):
     assert np.array_equal(k8.cpu().numpy(), ref8)
 
 
-@pytest.mark.parametrize("D", [64, 128])
-@pytest.mark.parametrize("G", [1, 4, 8, 16])
-def test_sparse_decode_matches_oracle(G, D):
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
+def test_sparse_decode_matches_oracle(G):
+    D = 128
     Hkv = 2
     lens = [0, 1, 65, 700, 2000, 3333]
-    w = wl.make_problem(len(lens), G * Hkv, Hkv, D, 3333, seed=410 + G * D, seqlens=lens,
+    w = wl.make_problem(len(lens), G * Hkv, Hkv, D, 3333, seed=410 + G, seqlens=lens,
                         nan_pad=True)
     d = OnDevice(w)
     k8, sk = quantize_on_gpu(d)
@@ -89,7 +89,7 @@ def test_sparse_decode_matches_oracle(G, D):
             ref, rl, kref = sparse.sparse_decode(w.q, w.k, w.v, w.scale, delta, S, w.seqlens,
                                                  k8=ref8, sk=refs)
             check_kept(w, kept, kref)
-            assert_close(got, gl, ref, rl, f"sparse G={G} D={D} S={S} delta={delta}")
+            assert_close(got, gl, ref, rl, f"sparse G={G} S={S} delta={delta}")
 
 
 def test_infinite_delta_is_dense_decode_bit_for_bit():
