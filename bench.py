@@ -621,7 +621,8 @@ def run_sparse(args):
         "bytes_read_per_call": read, "dense_kv_bytes_per_call": dense_bytes,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-                     "traffic": None},
+                     "traffic": ncu_traffic(w.name, S) if args.delta == 8.0 else None,
+                     "traffic_kernel": "fd_split_kernel (sparse)"},
         "dense": {"us_per_call": round(us_dense, 3),
                   "GB/s": round(dense_bytes / (us_dense * 1e-6) / 1e9, 1)},
         "speedup_vs_dense": round(us_dense / us_sparse, 3),
