@@ -152,3 +152,29 @@ def check_peaked(w, delta, share_lo, share_hi):
     print(f"{w.name} sparse S={S} delta={delta} kept {100 * share:.2f} % of blocks, "
           f"errors {e}, sparse-vs-dense max|dO| {gap:.3e}")
     assert share_lo <= share <= share_hi
+
+
+def test_sparse_decode_replays_from_a_cuda_graph():
+    t = torch()
+    w = wl.make_problem(2, 32, 8, 128, 4096, seed=450, seqlens=[4096, 3000])
+    d = OnDevice(w)
+    k8, sk = quantize_on_gpu(d)
+    eager, el, ek = run_sparse(d, k8, sk, 2.0, 3)
+    out = t.empty((w.B, w.Hq, w.D), dtype=t.bfloat16, device="cuda")
+    lse = t.empty((w.B, w.Hq), dtype=t.float32, device="cuda")
+    kept = t.full((w.B, w.Hkv, n_blocks(w)), 255, dtype=t.uint8, device="cuda")
+    nbytes = fd.fd_workspace_bytes(w.B, w.Hq, w.D, 3)
+    ws = t.empty(nbytes // 4, dtype=t.float32, device="cuda")
+    s = t.cuda.Stream()
+    g = t.cuda.CUDAGraph()
+    with t.cuda.graph(g, stream=s):
+        st = fd.fd_decode_sparse(d.problem(), d.q, d.k, d.v, k8, sk, d.seqlens, w.scale, 2.0, 3,
+                                 out, lse, kept, ws, nbytes, s.cuda_stream)
+    assert st == fd.FD_OK
+    for _ in range(3):
+        g.replay()
+    t.cuda.synchronize()
+    assert fd.fd_check_device_error() == fd.FD_OK
+    assert np.array_equal(host_bf16(out), eager)
+    assert np.array_equal(lse.cpu().numpy().astype(np.float64), el)
+    assert np.array_equal(kept.cpu().numpy(), ek)
