@@ -115,9 +115,10 @@ __device__ __forceinline__ void raise_device_error(unsigned int code) {
 // Merge the n_parts partials of one (sequence, query head) row; one warp,
 // lanes cover D.  Partial s of the row sits at po + s * o_stride (D floats)
 // and pl[s * l_stride].  Partials written by other CTAs are read through L2
-// (ld.global.cg).  The first 16 partials are requested together with the
-// lse values, so a row with up to 16 of them costs one round trip.  They are
-// summed in index order, so the result is deterministic.  A row whose
+// (ld.global.cg).  The first 32 partials are requested together with the
+// lse values, so a row with up to 32 of them (every fp8 call at S = 32
+// included) costs one round trip.  They are summed in index order, so the
+// result is deterministic and does not depend on the batch size.  A row whose
 // partials are all empty (lse = -inf) gives 0 and -inf.  The result goes to
 // orow (bf16) or, when orow_f32 is set, to orow_f32 (fp32).
 template <int D>
@@ -126,7 +127,7 @@ __device__ __forceinline__ void combine_row(const float* po, const float* pl, in
                                             __nv_bfloat16* orow, float* orow_f32,
                                             float* lse_out, int lane) {
   constexpr int VPL = D / 32;  // 4 or 2 values per lane
-  constexpr int BATCH = 16;
+  constexpr int BATCH = 32;
   constexpr float kLog2e = 1.4426950408889634074f;
   const float* col = po + lane * VPL;
   float lb[BATCH], ob[BATCH][VPL];
