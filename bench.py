@@ -74,6 +74,8 @@ def parse_args():
     ap.add_argument("--delta", type=float, default=8.0, help="top-delta threshold (nats)")
     ap.add_argument("--crossover", action="store_true",
                     help="planner sweep: split-count ladders over batch, length, element type")
+    ap.add_argument("--crossover-filter", default=None,
+                    help="with --crossover: only the shapes whose tag contains this text")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -728,9 +730,9 @@ def crossover(args):
     call over a ladder of split counts, timed from CUDA-graph replays (the
     call's own cost; eager calls below ~2K tokens are bound by the host's
     launch work), with cache copies rotated past L2.  Shapes: the CodeLlama-34B
-    head shape (Hq=64, Hkv=8, D=128) at B=1 over L = 512..128K and at B = 2..40
-    over L = 2K..64K, bf16 and fp8 caches; G=4; the varlen, paged and peaked
-    workloads.  One JSON line per shape on stdout, with the planner's pick
+    head shape (Hq=64, Hkv=8, D=128) at B=1 over L = 512..128K, at B = 2..40
+    over L = 2K..64K, and at B = 64 and 256 over L = 512..8K, bf16 and fp8
+    caches; G=4; the varlen, paged and peaked workloads.  One JSON line per shape on stdout, with the planner's pick
     (fd_plan_problem) and its regret against the fastest measured count."""
     import torch
     import split_kv_decode_attn_b200 as fd
@@ -740,7 +742,11 @@ def crossover(args):
     fd.load_library()
     ladder = (1, 2, 3, 4, 6, 8, 12, 16, 20, 24, 28, 32, 40, 48, 64)
 
-    def run(w, Ss, tag):
+    def run(make, Ss, tag):
+        """make: builds the workload (only for the shapes that are run)."""
+        if args.crossover_filter and args.crossover_filter not in tag:
+            return
+        w = make()
         copies, _ = copies_for(torch, w.k.nbytes + w.v.nbytes, device)
         prob = fd.make_problem(w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size, w.num_blocks,
                                w.max_blocks_per_seq, w.kv_layout, w.kv_dtype_code, w.k_scale,
@@ -763,24 +769,32 @@ def crossover(args):
 
     for L in (512, 1024, 2048, 4096, 8192, 16384, 32768, 65536, 131072):
         for kvd in ("bf16", "fp8"):
-            w = make_workload("codellama34b", L, 0, kv_dtype=kvd)
-            run(w, [s for s in ladder if s <= L // 64], f"B1-L{L}-{kvd}")
+            run(lambda L=L, kvd=kvd: make_workload("codellama34b", L, 0, kv_dtype=kvd),
+                [s for s in ladder if s <= L // 64], f"B1-L{L}-{kvd}")
     for L in (16384, 65536):
-        run(wl.make_problem(1, 32, 8, 128, L, wl.CONFIG_SEED_BASE + 300, name="g4"),
+        run(lambda L=L: wl.make_problem(1, 32, 8, 128, L, wl.CONFIG_SEED_BASE + 300, name="g4"),
             [s for s in ladder if s <= L // 64], f"G4-B1-L{L}")
     for B in (2, 4, 8, 16, 32, 40):
         for L in (2048, 8192, 16384, 65536):
             if B * 8 * L * 128 * 4 > 4.5e9:
                 continue
             for kvd in (("bf16", "fp8") if B in (4, 16) else ("bf16",)):
-                w = wl.make_problem(B, 64, 8, 128, L, wl.CONFIG_SEED_BASE + 200 + B,
-                                    name=f"B{B}-L{L}", kv_dtype=kvd)
-                run(w, [s for s in (1, 2, 3, 4, 6, 8, 12, 16, 24, 32) if s <= L // 64],
+                run(lambda B=B, L=L, kvd=kvd: wl.make_problem(
+                        B, 64, 8, 128, L, wl.CONFIG_SEED_BASE + 200 + B, name=f"B{B}-L{L}",
+                        kv_dtype=kvd),
+                    [s for s in (1, 2, 3, 4, 6, 8, 12, 16, 24, 32) if s <= L // 64],
                     f"B{B}-L{L}-{kvd}")
+    # Large batches: B * Hkv = 512 and 2048 CTAs at S = 1 already fill the device.
+    for B, Ls in ((64, (512, 2048, 8192)), (256, (512, 2048, 4096))):
+        for L in Ls:
+            run(lambda B=B, L=L: wl.make_problem(B, 64, 8, 128, L, wl.CONFIG_SEED_BASE + 200 + B,
+                                                 name=f"B{B}-L{L}"),
+                [1, 2, 3, 4], f"bigbatch-B{B}-L{L}-bf16")
     for kvd in ("bf16", "fp8"):
-        run(make_workload("varlen", None, 0, kv_dtype=kvd), [1, 2, 3, 4, 6, 8], f"varlen-{kvd}")
-    run(make_workload("paged", None, 0), [1, 2, 3, 4, 6, 8], "paged-bf16")
-    run(make_workload("peaked", None, 0), [8, 12, 16, 20, 24, 32, 48, 64], "peaked-bf16")
+        run(lambda kvd=kvd: make_workload("varlen", None, 0, kv_dtype=kvd), [1, 2, 3, 4, 6, 8],
+            f"varlen-{kvd}")
+    run(lambda: make_workload("paged", None, 0), [1, 2, 3, 4, 6, 8], "paged-bf16")
+    run(lambda: make_workload("peaked", None, 0), [8, 12, 16, 20, 24, 32, 48, 64], "peaked-bf16")
     assert fd.fd_check_device_error() == 0
 
 
