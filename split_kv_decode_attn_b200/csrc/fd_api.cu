@@ -150,7 +150,7 @@ int ilog2(int x) {
 }
 
 fd_status check_shape(int B, int Hq, int Hkv, int D, int max_len, int block_size) {
-  if (B < 1 || B > 65535 || Hq < 1 || Hkv < 1 || Hkv > 65535 || max_len < 0)
+  if (B < 1 || B > 65535 || Hq < 1 || Hkv < 1 || Hkv > 65535 || max_len < 0 || block_size < 0)
     return FD_ERR_INVALID_ARGUMENT;
   if (Hq % Hkv != 0) return FD_ERR_INVALID_ARGUMENT;
   if (D != 64 && D != 128) return FD_ERR_UNSUPPORTED;
@@ -158,7 +158,6 @@ fd_status check_shape(int B, int Hq, int Hkv, int D, int max_len, int block_size
   if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return FD_ERR_UNSUPPORTED;
   if (block_size != 0 && (!is_pow2(block_size) || block_size < 8 || block_size > 256))
     return FD_ERR_UNSUPPORTED;
-  if (block_size < 0) return FD_ERR_INVALID_ARGUMENT;
   return FD_OK;
 }
 

@@ -196,6 +196,7 @@ def test_plan_invalid_and_unsupported():
     assert fd.fd_plan_sm(B200_SMS, 1, 24, 1, 128, 100, 0) == fd.FD_ERR_UNSUPPORTED  # G = 24
     assert fd.fd_plan_sm(B200_SMS, 1, 8, 8, 128, 100, 24) == fd.FD_ERR_UNSUPPORTED
     assert fd.fd_plan_sm(B200_SMS, 1, 8, 8, 128, 100, 4) == fd.FD_ERR_UNSUPPORTED
+    assert fd.fd_plan_sm(B200_SMS, 1, 8, 8, 128, 100, -16) == fd.FD_ERR_INVALID_ARGUMENT
     assert fd.fd_plan_sm(0, 1, 8, 8, 128, 100, 0) == fd.FD_ERR_INVALID_ARGUMENT
 
 
