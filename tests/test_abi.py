@@ -110,6 +110,12 @@ def test_plan_long_history_fills_the_device():
     ((16, 64, 8, 128, 16384, 0), {1, 2, 4, 6, 8, 12}),
     ((32, 64, 8, 128, 2048, 0), {1}),
     ((40, 64, 8, 128, 8192, 0), {2, 3, 4, 6, 8, 12}),  # just above one wave: split
+    ((64, 64, 8, 128, 512, 0), {1}),            # 512 and 2048 units: one split fastest
+    ((64, 64, 8, 128, 2048, 0), {1}),
+    ((64, 64, 8, 128, 8192, 0), {1}),
+    ((256, 64, 8, 128, 512, 0), {1}),
+    ((256, 64, 8, 128, 2048, 0), {1}),
+    ((256, 64, 8, 128, 4096, 0), {1}),
     ((8, 32, 8, 128, 131072, 16), {3, 4, 8}),
     ((1, 32, 8, 128, 262144, 0), {16, 17, 20, 24, 32, 64}),
 ])
