@@ -251,6 +251,24 @@ class Call:
             raise RuntimeError(f"fd_decode: {self.fd.fd_status_string(st)}")
 
 
+def planner_cost(fd, prob, seqlens, num_sms=0, calls=2000):
+    """Host microseconds per fd_plan_problem call through the Python binding,
+    with the lengths when the workload has them (the planner runs outside the
+    timed region; this is its cost).  None if the planner fails."""
+    try:
+        first = fd.fd_plan_problem(num_sms, prob, seqlens)
+        if first < 1:
+            return None
+        t0 = time.perf_counter()
+        for _ in range(calls):
+            fd.fd_plan_problem(num_sms, prob, seqlens)
+        dt = time.perf_counter() - t0
+        return {"us_per_call": round(dt / calls * 1e6, 3), "calls": calls, "num_splits": first,
+                "with_lengths": seqlens is not None}
+    except Exception:
+        return None
+
+
 def max_over_ranks(torch, ms, world, device=None):
     """The slowest rank's time: the job is done when every rank is done."""
     if world <= 1:
@@ -471,6 +489,7 @@ def run_fd(args):
                      "algorithmic_bytes": kvb},
         "gpu_launches": args.steps * call.launches_per_call,
         "clocks": clocks,
+        "planner": planner_cost(fd, call.prob, w.seqlens),
     }
 
     if not args.no_e2e:

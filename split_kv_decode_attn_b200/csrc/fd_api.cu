@@ -420,15 +420,21 @@ int pick_splits(int max_len, Model model) {
   int best = 1;
   double best_t = model(1);
   int last_eff = 1;
-  for (int S = 2; S <= s_max; ++S) {
+  for (int S = 2; S <= s_max;) {
+    // Split S has c = ceil(tiles / S) tiles; every S up to `last` has the
+    // same chunking (and effective count), so only the first is evaluated.
+    const long long c = (tiles + S - 1) / S;
+    const long long last = c > 1 ? (tiles - 1) / (c - 1) : s_max;
     const int eff = effective_splits(max_len, chunk_for(max_len, S));
-    if (eff == last_eff) continue;  // same chunking as a smaller S
-    last_eff = eff;
-    const double t = model(S);
-    if (t < best_t * 0.98) {
-      best_t = t;
-      best = S;
+    if (eff != last_eff) {  // otherwise the same chunking as a smaller S
+      last_eff = eff;
+      const double t = model(S);
+      if (t < best_t * 0.98) {
+        best_t = t;
+        best = S;
+      }
     }
+    S = static_cast<int>(std::min<long long>(last, s_max)) + 1;
   }
   return best;
 }
