@@ -240,6 +240,65 @@ def make_problem(B, Hq, Hkv, D, max_len, block_size=0, num_blocks=0, max_blocks_
                       kv_layout, kv_dtype, k_scale, v_scale)
 
 
+def _check(t, name, dtypes, shape=None):
+    """Checks a tensor argument of decode() before its address is passed on:
+    the kernels read and write dense row-major buffers of the stated shapes."""
+    if dtypes is not None and t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {' or '.join(map(str, dtypes))}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (row-major)")
+
+
+def _check_decode_args(q, k_cache, v_cache, seqlens, block_table, kv_layout, max_len, out, lse,
+                       workspace):
+    """Shape, dtype, layout and device checks of decode(); raises ValueError.
+    The device checks come last."""
+    import torch
+    cache_types = [torch.bfloat16, torch.uint8]
+    if hasattr(torch, "float8_e4m3fn"):
+        cache_types.append(torch.float8_e4m3fn)
+    if q.dim() != 3:
+        raise ValueError(f"q: expected [B, Hq, D], got shape {tuple(q.shape)}")
+    B, Hq, D = q.shape
+    _check(q, "q", [torch.bfloat16])
+    if kv_layout not in (FD_LAYOUT_HND, FD_LAYOUT_NHD):
+        raise ValueError(f"kv_layout: {kv_layout}, expected FD_LAYOUT_HND or FD_LAYOUT_NHD")
+    if k_cache.dim() != 4:
+        raise ValueError(f"k_cache: expected 4 dimensions, got shape {tuple(k_cache.shape)}")
+    _check(k_cache, "k_cache", cache_types)
+    _check(v_cache, "v_cache", [k_cache.dtype], k_cache.shape)
+    if k_cache.shape[3] != D:
+        raise ValueError(f"k_cache: head dim {k_cache.shape[3]}, q has {D}")
+    if block_table is None:
+        if k_cache.shape[0] != B:
+            raise ValueError(f"k_cache: {k_cache.shape[0]} sequences, q has {B}")
+        rows = k_cache.shape[2] if kv_layout == FD_LAYOUT_HND else k_cache.shape[1]
+        if max_len is not None and max_len != rows:
+            raise ValueError(f"max_len {max_len}: a contiguous cache holds {rows} rows per "
+                             "sequence and KV head, and max_len must equal it")
+    else:
+        if block_table.dim() != 2 or block_table.shape[0] != B:
+            raise ValueError(f"block_table: expected [B={B}, max_blocks], got "
+                             f"{tuple(block_table.shape)}")
+        _check(block_table, "block_table", [torch.int32])
+    if seqlens is not None:
+        _check(seqlens, "seqlens", [torch.int32], (B,))
+    if out is not None:
+        _check(out, "out", [torch.bfloat16], (B, Hq, D))
+    if lse is not None:
+        _check(lse, "lse", [torch.float32], (B, Hq))
+    if workspace is not None:
+        _check(workspace, "workspace", None)
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("seqlens", seqlens),
+                    ("block_table", block_table), ("out", out), ("lse", lse),
+                    ("workspace", workspace)):
+        if t is not None and (not t.is_cuda or t.device != q.device):
+            raise ValueError(f"{name} is on {t.device}; every tensor must be on q's CUDA device "
+                             f"({q.device})")
+
+
 def decode(q, k_cache, v_cache, seqlens=None, block_table=None, *, max_len: Optional[int] = None,
            kv_layout: int = FD_LAYOUT_HND, scale: Optional[float] = None,
            num_splits: Optional[int] = None, out=None, lse=None, workspace=None, stream=None,
@@ -253,8 +312,12 @@ def decode(q, k_cache, v_cache, seqlens=None, block_table=None, *, max_len: Opti
     [B, max_len, Hkv, D] or paged [num_blocks, block_size, Hkv, D].  Paged
     caches come with block_table [B, max_blocks] int32.  seqlens [B] int32
     or None.  Returns (out [B, Hq, D] bf16, lse [B, Hq] fp32).  num_splits
-    defaults to fd_plan_problem's choice."""
+    defaults to fd_plan_problem's choice.  Raises ValueError for tensors of
+    the wrong dtype, shape or device, or not contiguous, before anything is
+    launched, and FdError for a failing status."""
     import torch
+    _check_decode_args(q, k_cache, v_cache, seqlens, block_table, kv_layout, max_len, out, lse,
+                       workspace)
     B, Hq, D = q.shape
     block_size = 0
     fp8 = k_cache.element_size() == 1
