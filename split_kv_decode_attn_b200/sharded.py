@@ -38,6 +38,8 @@ def local_partial(q, k_shard, v_shard, seqlens_shard=None, *, block_table=None, 
     import torch
 
     import split_kv_decode_attn_b200 as fd
+    fd._check_decode_args(q, k_shard, v_shard, seqlens_shard, block_table, kv_layout, None,
+                          None, None, None)
     B, Hq, D = q.shape
     if block_table is None:
         if kv_layout == fd.FD_LAYOUT_HND:
@@ -73,6 +75,12 @@ def combine(o_all, lse_all, stream=None):
 
     import split_kv_decode_attn_b200 as fd
     R, B, Hq, D = o_all.shape
+    if o_all.dtype != torch.float32 or lse_all.dtype != torch.float32:
+        raise ValueError("combine: o_all and lse_all must be float32")
+    if tuple(lse_all.shape) != (R, B, Hq):
+        raise ValueError(f"combine: lse_all shape {tuple(lse_all.shape)}, expected {(R, B, Hq)}")
+    if not (o_all.is_cuda and lse_all.device == o_all.device):
+        raise ValueError("combine: o_all and lse_all must be on one CUDA device")
     out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=o_all.device)
     lse = torch.empty((B, Hq), dtype=torch.float32, device=o_all.device)
     st = fd.fd_combine(R, B, Hq, D, o_all.contiguous(), lse_all.contiguous(), out, lse, stream)

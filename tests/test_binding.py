@@ -65,3 +65,18 @@ def test_views_that_are_not_contiguous():
     raises("k_cache must be contiguous", q, kt, kt)
     wide = torch.zeros(2, 2, 512, 128, dtype=torch.bfloat16)[:, :, :256]
     raises("k_cache must be contiguous", q, wide, wide)
+
+
+def test_sharded_helpers_check_their_tensors():
+    from split_kv_decode_attn_b200 import sharded
+    q, k, v = args()
+    with pytest.raises(ValueError, match="CUDA device"):
+        sharded.local_partial(q, k, v, torch.zeros(2, dtype=torch.int32))
+    with pytest.raises(ValueError, match="seqlens: dtype"):
+        sharded.local_partial(q, k, v, torch.zeros(2, dtype=torch.int64))
+    with pytest.raises(ValueError, match="float32"):
+        sharded.combine(torch.zeros(2, 2, 16, 128, dtype=torch.float64), torch.zeros(2, 2, 16))
+    with pytest.raises(ValueError, match="lse_all shape"):
+        sharded.combine(torch.zeros(2, 2, 16, 128), torch.zeros(2, 16))
+    with pytest.raises(ValueError, match="CUDA device"):
+        sharded.combine(torch.zeros(2, 2, 16, 128), torch.zeros(2, 2, 16))
