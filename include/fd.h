@@ -308,8 +308,8 @@ FD_API fd_status fd_decode_sparse(const fd_problem* p, const void* q, const void
 #define FD_STATIC_WORKSPACE_BYTES (8u << 20)
 
 /* fd_decode for callers that cannot allocate device memory.
- * The paper has no counterpart to this entry point; it is an addition of this
- * library. Some callers cannot call cudaMalloc at all. Examples: a plain C
+ * The Flash-Decoding pages have no counterpart to this entry point; it is an
+ * addition of this library. Some callers cannot call cudaMalloc at all. Examples: a plain C
  * host program that links only this library and has no device allocator of
  * its own; code inside a framework whose memory pool owns all device memory
  * and forbids raw allocations; a decode loop that must not call cudaMalloc
