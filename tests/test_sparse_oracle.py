@@ -121,3 +121,23 @@ def test_more_delta_keeps_more_and_each_split_keeps_its_best_block():
             for s0 in range(0, nb, chunk):
                 assert kept0[b, h, s0:min(nb, s0 + chunk)].any()
             assert not kept0[b, h, nb:].any()
+
+
+def test_kept_blocks_are_the_union_over_the_heads_of_a_group():
+    """Two query heads of one group, each with its own dominant key in a
+    different block: with one split and delta = 0 exactly those two blocks
+    survive, one chosen by each head (a rule that looked at one head only, or
+    at the sum over heads, would keep one)."""
+    w = problem(B=1, Hq=2, Hkv=1, D=128, L=1024, seed=21, lens=(1024,))
+    qf = f32(w.q[0]).astype(np.float64)
+    k = w.k.copy()
+    for g, pos in ((0, 130), (1, 900)):
+        key = 24.0 * qf[g] / np.linalg.norm(qf[g])
+        k[0, 0, pos] = wl.f64_to_bf16_bits(key)
+    k8, sk = sparse.quantize_keys(k)
+    kept = sparse.select_blocks(w.q, k8, sk, w.scale, 0.0, 1)
+    assert kept[0, 0].tolist() == [i in (130 // 64, 900 // 64) for i in range(16)]
+    # each head alone keeps only its own block
+    for g, pos in ((0, 130), (1, 900)):
+        one = sparse.select_blocks(w.q[:, g:g + 1], k8, sk, w.scale, 0.0, 1)
+        assert one[0, 0].tolist() == [i == pos // 64 for i in range(16)]
