@@ -1,8 +1,8 @@
 """Sequence-parallel decode on one GPU: the history is cut into R contiguous
 slices; fd_decode_partial runs on each slice, the R results are stacked (as
-an all-gather would lay them out) and fd_combine merges them.  The pool these
-tests run on gives one GPU, so the slices run one after another on the same
-device; nothing waits on anything else."""
+an all-gather would lay them out) and fd_combine merges them.  The slices run
+one after another on one device, so nothing waits on anything else; with one
+GPU per rank the same partials would be all-gathered instead of stacked."""
 import numpy as np
 import pytest
 
