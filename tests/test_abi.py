@@ -386,3 +386,28 @@ def test_quantize_keys_checks():
     assert quant(fd.make_problem(1, 8, 8, 128, 512, kv_dtype=fd.FD_KV_FP8_E4M3)) == \
         fd.FD_ERR_UNSUPPORTED
     assert quant(P(D=96)) == fd.FD_ERR_UNSUPPORTED
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/fd.h is a C header: a C99 program (pedantic, all warnings as
+    errors) includes it, links libfd.so and calls the planner, with no
+    device needed when the SM count is given."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_fd.c"
+    src.write_text(
+        '#include "fd.h"\n'
+        "int main(void) {\n"
+        "  fd_problem p = {0};\n"
+        "  p.B = 1; p.Hq = 64; p.Hkv = 8; p.D = 128; p.max_len = 65536;\n"
+        "  return fd_plan_problem(148, &p, 0) == 16 ? 0 : 1;\n"
+        "}\n")
+    libdir = os.path.dirname(fd.LIB_PATH)
+    exe = tmp_path / "use_fd"
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-L", libdir, "-lfd",
+                    f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    assert subprocess.run([str(exe)]).returncode == 0
