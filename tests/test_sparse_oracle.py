@@ -1,12 +1,30 @@
 """Pins of the sparse-decode oracle (oracle/sparse.py): the low-bit codes, the
 scan's error bound, the top-delta rule's special cases, and the reduction to
 the dense oracle when every block is kept."""
+import importlib.util
+import os
+
 import numpy as np
 import pytest
 
 import oracle
-from oracle import sparse
 from split_kv_decode_attn_b200 import workloads as wl
+
+
+def _sparse_oracle():
+    """oracle.sparse, or the copy named by FD_SPARSE_ORACLE (the mutant tests
+    run these pins against copies with one planted slip)."""
+    path = os.environ.get("FD_SPARSE_ORACLE")
+    if not path:
+        from oracle import sparse as module
+        return module
+    spec = importlib.util.spec_from_file_location("sparse_under_test", path)
+    module = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(module)
+    return module
+
+
+sparse = _sparse_oracle()
 
 pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
 
@@ -141,3 +159,12 @@ def test_kept_blocks_are_the_union_over_the_heads_of_a_group():
     for g, pos in ((0, 130), (1, 900)):
         one = sparse.select_blocks(w.q[:, g:g + 1], k8, sk, w.scale, 0.0, 1)
         assert one[0, 0].tolist() == [i == pos // 64 for i in range(16)]
+
+
+def test_split_chunks_follow_the_dense_chunking():
+    """ceil(max_len / S) rounded up to the 64-token tile, at least one tile."""
+    assert sparse.chunk_for(2048, 4) == 512
+    assert sparse.chunk_for(1000, 3) == 384     # ceil(1000 / 3) = 334 -> 384
+    assert sparse.chunk_for(65, 2) == 64        # 33 -> 64
+    assert sparse.chunk_for(10, 16) == 64
+    assert sparse.chunk_for(262144, 16) == 16384
