@@ -31,6 +31,13 @@ MUTANTS = {
     "combine lse drops max": ("*lse = M + std::log(W);", "*lse = std::log(W);"),
     "max is first element": ("for (long j = 0; j < n; ++j) m = s[j] > m ? s[j] : m;",
                              "m = s[0];"),
+    "lengths not clamped to max_len": ("    if (n > max_len) n = max_len;\n", ""),
+    "batch base counts query heads": ("const long base = (b * Hkv + kv) * max_len * D;",
+                                      "const long base = (b * Hq + kv) * max_len * D;"),
+    "every head reads the first query": ("attend_one_head(n, D, q + i * D, k + base",
+                                         "attend_one_head(n, D, q + b * Hq * D, k + base"),
+    "empty split lse zero": ("part_lse[s] = s < S ? l_s[s] : ninf;",
+                             "part_lse[s] = s < S ? l_s[s] : 0.0;"),
     "empty sequence lse zero": ("    *lse = ninf;\n    return;\n  }\n  std::vector<double> s(",
                                 "    *lse = 0.0;\n    return;\n  }\n  std::vector<double> s("),
 }
