@@ -1,7 +1,7 @@
 // fd_ptx.cuh — inline-PTX building blocks for the sm_100a decode kernels:
-// mbarriers with bounded waits, TMA tensor loads (no multicast), ldmatrix,
-// bf16 mma.sync, movmatrix, programmatic dependent launch and the global
-// timer.  Every wrapper is a single instruction or a short fixed sequence.
+// mbarriers with bounded waits, TMA tensor loads into the CTA's own shared
+// memory, ldmatrix, bf16 mma.sync, movmatrix, programmatic dependent launch
+// and the global timer.  Every wrapper is a single instruction or a short fixed sequence.
 #pragma once
 
 #include <cstdint>
@@ -67,7 +67,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
   return true;
 }
 
-// ---- TMA (tensor-map bulk copies, CTA-local destination, no multicast) ------
+// ---- TMA (tensor-map bulk copies into this CTA's own shared memory) ---------
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* tm) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
