@@ -1,7 +1,8 @@
 // fd_ptx.cuh — inline-PTX building blocks for the sm_100a decode kernels:
 // mbarriers with bounded waits, TMA tensor loads into the CTA's own shared
 // memory, ldmatrix, bf16 mma.sync, movmatrix, programmatic dependent launch
-// and the global timer.  Every wrapper is a single instruction or a short fixed sequence.
+// and the global timer.  Every wrapper is a single instruction or a short
+// fixed sequence.
 #pragma once
 
 #include <cstdint>
