@@ -16,6 +16,8 @@ Reported (one JSON line from rank 0):
                host<->device copies inside the timed region
   cpu_baseline the fp64 oracle on this host's cores, on a bounded sample
   sweep        the same call at cache lengths 512 .. 64K
+  planner      host microseconds per fd_plan_problem call (outside the timed
+               region)
 
 Multi-GPU (torchrun, one rank per GPU): every rank decodes its own batch
 (independent sequences; the path needs no collective), weak scaling.
