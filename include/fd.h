@@ -158,17 +158,25 @@ FD_API int fd_plan_seqlens(int num_sms, int B, int Hq, int Hkv, int D, int max_l
  * cache with D != 128. Host only and deterministic. */
 FD_API int fd_plan_problem(int num_sms, const fd_problem* p, const int32_t* seqlens);
 
-/* Tokens per split for a given split count. This is ceil(max_len /
- * num_splits) rounded up to the 64-token tile. Split s covers tokens
- * [s*chunk, (s+1)*chunk) of every sequence, and splits past a sequence's end
- * are empty. Returns a negative fd_status for invalid arguments. */
+/* How a call cuts the history. With T = ceil(max_len / 64) tiles of 64
+ * tokens, the effective split count is S = min(num_splits, T) (1 when
+ * max_len is 0), and split s covers the tiles [floor(s*T/S),
+ * floor((s+1)*T/S)) of every sequence: tokens [64*floor(s*T/S),
+ * 64*floor((s+1)*T/S)), cut at the sequence's length. The splits differ by
+ * at most one tile, so any split count up to T gives CTAs of balanced size.
+ * Splits past a sequence's end are empty.
+ * fd_split_chunk returns the largest split's tokens, 64*ceil(T/S) (64 when
+ * max_len is 0); fd_effective_splits returns S. Both return a negative
+ * fd_status for invalid arguments. */
 FD_API int fd_split_chunk(int max_len, int num_splits);
+FD_API int fd_effective_splits(int max_len, int num_splits);
 
 /* Workspace bytes that fd_decode needs for num_splits splits. This is 0
  * when num_splits == 1. Otherwise it is the fp32 partial outputs
  * [B, Hq, S, D] followed by the fp32 partial log-sum-exps [B, Hq, S], each
  * part rounded up to 256 bytes, with S = num_splits. The effective split
- * count never exceeds num_splits, so this size is always enough for the call.
+ * count (fd_effective_splits) never exceeds num_splits, so this size is
+ * always enough for the call.
  * Returns 0 for invalid arguments. */
 FD_API size_t fd_workspace_bytes(int B, int Hq, int D, int num_splits);
 
@@ -193,7 +201,8 @@ FD_API size_t fd_workspace_bytes(int B, int Hq, int D, int num_splits);
  *                NULL selects the contiguous layout and needs block_size == 0.
  *   scale        softmax scale (finite, > 0), typically 1/sqrt(D)
  *   num_splits   requested split count in [1, 1024], normally fd_plan's
- *                result. The effective count is ceil(max_len / chunk).
+ *                result. The effective count is min(num_splits,
+ *                ceil(max_len / 64)); see fd_split_chunk for the cut.
  *   out          [B, Hq, D] bf16, round-to-nearest-even, 16-byte aligned
  *   lse          [B, Hq] fp32 natural-log log-sum-exp of the scaled logits,
  *                or NULL to skip it
@@ -250,6 +259,21 @@ FD_API fd_status fd_decode_partial(const fd_problem* p, const void* q, const voi
 FD_API fd_status fd_combine(int R, int B, int Hq, int D, const float* part_o,
                             const float* part_lse, void* out, float* lse, fd_stream_t stream);
 
+/* fd_combine over parts placed at any stride, so that a gathered buffer is
+ * merged where it lies, with no copy. Part r of row i (i = b * Hq + h) is the
+ * D floats at part_o + r * o_stride + i * D and the lse at
+ * part_lse[r * lse_stride + i]; fd_combine is the case o_stride = B*Hq*D,
+ * lse_stride = B*Hq. One packed buffer per part, for example
+ *   [O: B*Hq*D floats][lse: B*Hq floats][padding]
+ * all-gathered into R consecutive buffers of P floats, is merged with
+ *   part_o = buf, part_lse = buf + B*Hq*D, o_stride = lse_stride = P.
+ * Strides count floats. o_stride must be a multiple of 4 and at least
+ * B*Hq*D; lse_stride at least B*Hq; otherwise FD_ERR_INVALID_ARGUMENT. The
+ * rest is as fd_combine. */
+FD_API fd_status fd_combine_strided(int R, int B, int Hq, int D, const float* part_o,
+                                    size_t o_stride, const float* part_lse, size_t lse_stride,
+                                    void* out, float* lse, fd_stream_t stream);
+
 /* Low-bit key codes for fd_decode_sparse ("Faster Than Flash: Exploiting
  * Attention Sparsity for Efficient Long-Context Decoding", abstract: a scan
  * over low-bit keys replaces metadata indices). Call it when the cache
@@ -293,7 +317,8 @@ FD_API fd_status fd_quantize_keys(const fd_problem* p, const void* k_cache,
  *                 Blocks at or past a sequence's length are not written.
  * Other arguments are those of fd_decode with a contiguous head-major bf16
  * cache and D = 128 (FD_ERR_UNSUPPORTED otherwise). The split count must make
- * the chunk at most 16,384 tokens (FD_ERR_INVALID_ARGUMENT otherwise). The
+ * the largest split (fd_split_chunk) at most 16,384 tokens
+ * (FD_ERR_INVALID_ARGUMENT otherwise). The
  * codes stream through the split kernel's tile pipeline (TMA, 256 tokens per
  * stage) and the dot products run on int8 tensor cores. Results are
  * deterministic. */
@@ -321,8 +346,12 @@ FD_API fd_status fd_decode_sparse(const fd_problem* p, const void* q, const void
  * loads this library holds until the process exits. This entry point calls
  * no cudaMalloc, cudaFree or other allocating routine.
  *  - Set-up: the first call on a device looks up the array's device address
- *    with the device current (cudaGetSymbolAddress) and caches it. Make that
- *    first call before any stream capture on that device.
+ *    with the device current (cudaGetSymbolAddress) and caches it with the
+ *    id of the device's context. Make that first call before any stream
+ *    capture on that device. After a device reset (cudaDeviceReset) the
+ *    device has a new context, in which the array may sit elsewhere: the
+ *    next call sees the new context id and looks the address up again, so
+ *    make that call, too, outside a capture.
  *  - Size limit: when the effective split count needs more than
  *    FD_STATIC_WORKSPACE_BYTES (see fd_workspace_bytes), the call returns
  *    FD_ERR_WORKSPACE and launches nothing. Pass a smaller num_splits, or use

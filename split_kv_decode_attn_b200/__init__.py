@@ -27,12 +27,14 @@ FD_ERR_CUDA = -4
 FD_ERR_DEVICE_TIMEOUT = -5
 
 # Entry points declared in include/fd.h.
-EXPORTS = ("fd_plan", "fd_plan_sm", "fd_plan_seqlens", "fd_plan_problem", "fd_split_chunk", "fd_workspace_bytes", "fd_decode",
-           "fd_decode_partial", "fd_combine", "fd_quantize_keys", "fd_decode_sparse",
+EXPORTS = ("fd_plan", "fd_plan_sm", "fd_plan_seqlens", "fd_plan_problem", "fd_split_chunk",
+           "fd_effective_splits", "fd_workspace_bytes", "fd_decode",
+           "fd_decode_partial", "fd_combine", "fd_combine_strided", "fd_quantize_keys",
+           "fd_decode_sparse",
            "fd_decode_static_workspace", "fd_check_device_error",
            "fd_selftest_device_timeout", "fd_status_string")
 
-# Mirrors FD_STATIC_WORKSPACE_BYTES in include/fd.h.
+# Mirrors FD_STATIC_WORKSPACE_BYTES in include/fd.h (a CPU test compares the two).
 FD_STATIC_WORKSPACE_BYTES = 8 << 20
 
 
@@ -79,6 +81,8 @@ def load_library(path: str = LIB_PATH):
         lib.fd_plan_problem.restype = I
         lib.fd_split_chunk.argtypes = [I, I]
         lib.fd_split_chunk.restype = I
+        lib.fd_effective_splits.argtypes = [I, I]
+        lib.fd_effective_splits.restype = I
         lib.fd_workspace_bytes.argtypes = [I, I, I, I]
         lib.fd_workspace_bytes.restype = sz
         lib.fd_decode.argtypes = [ctypes.POINTER(fd_problem), vp, vp, vp, vp, vp, F, I, vp, vp,
@@ -94,6 +98,8 @@ def load_library(path: str = LIB_PATH):
         lib.fd_decode_sparse.restype = I
         lib.fd_combine.argtypes = [I, I, I, I, vp, vp, vp, vp, vp]
         lib.fd_combine.restype = I
+        lib.fd_combine_strided.argtypes = [I, I, I, I, vp, sz, vp, sz, vp, vp, vp]
+        lib.fd_combine_strided.restype = I
         lib.fd_decode_static_workspace.argtypes = [ctypes.POINTER(fd_problem), vp, vp, vp, vp,
                                                    vp, F, I, vp, vp, vp]
         lib.fd_decode_static_workspace.restype = I
@@ -161,6 +167,10 @@ def fd_split_chunk(max_len: int, num_splits: int) -> int:
     return int(load_library().fd_split_chunk(max_len, num_splits))
 
 
+def fd_effective_splits(max_len: int, num_splits: int) -> int:
+    return int(load_library().fd_effective_splits(max_len, num_splits))
+
+
 def fd_workspace_bytes(B: int, Hq: int, D: int, num_splits: int) -> int:
     return int(load_library().fd_workspace_bytes(B, Hq, D, num_splits))
 
@@ -213,11 +223,32 @@ def fd_combine(R: int, B: int, Hq: int, D: int, part_o, part_lse, out, lse, stre
                                          _ptr(lse), _stream(stream)))
 
 
+def fd_combine_strided(R: int, B: int, Hq: int, D: int, part_o, o_stride: int, part_lse,
+                       lse_stride: int, out, lse, stream=None) -> int:
+    """Call the C fd_combine_strided: merge R partials placed at strides
+    (counted in floats), e.g. R packed per-rank buffers gathered end to end.
+    Returns the status."""
+    return int(load_library().fd_combine_strided(R, B, Hq, D, _ptr(part_o), o_stride,
+                                                 _ptr(part_lse), lse_stride, _ptr(out),
+                                                 _ptr(lse), _stream(stream)))
+
+
 def fd_decode_static_workspace(problem: fd_problem, q, k_cache, v_cache, seqlens, block_table,
                                scale: float, num_splits: int, out, lse, stream=None) -> int:
     """Call the C fd_decode_static_workspace: fd_decode for callers that cannot
     allocate device memory; its scratch is the library's static device array
-    of FD_STATIC_WORKSPACE_BYTES.  Returns the status code."""
+    of FD_STATIC_WORKSPACE_BYTES.  Returns the status code.
+
+    When q is a torch tensor, the tensors are checked as decode() checks them
+    (dtype, shape, contiguity, device, and a contiguous cache's row count
+    against problem.max_len) and against the problem's sizes, and a mismatch
+    raises ValueError before anything is launched: the C ABI sees only
+    addresses, and a strided or padded view would be read as dense memory."""
+    if q is not None and q.__class__ is not int:
+        if q.dim() == 3 and k_cache.dim() == 4:
+            _check_problem_sizes(problem, q, k_cache)
+        _check_decode_args(q, k_cache, v_cache, seqlens, block_table, problem.kv_layout,
+                           problem.max_len if problem.block_size == 0 else None, out, lse, None)
     return int(load_library().fd_decode_static_workspace(
         ctypes.byref(problem), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens),
         _ptr(block_table), ctypes.c_float(scale), int(num_splits), _ptr(out), _ptr(lse),
@@ -297,6 +328,23 @@ def _check_decode_args(q, k_cache, v_cache, seqlens, block_table, kv_layout, max
         if t is not None and (not t.is_cuda or t.device != q.device):
             raise ValueError(f"{name} is on {t.device}; every tensor must be on q's CUDA device "
                              f"({q.device})")
+
+
+def _check_problem_sizes(problem: fd_problem, q, k_cache):
+    """The problem's B, Hq, D, Hkv (and page size) must describe the tensors."""
+    B, Hq, D = q.shape
+    if (problem.B, problem.Hq, problem.D) != (B, Hq, D):
+        raise ValueError(f"problem (B, Hq, D) = {(problem.B, problem.Hq, problem.D)}, q has "
+                         f"{(B, Hq, D)}")
+    hnd = problem.kv_layout == FD_LAYOUT_HND
+    Hkv = k_cache.shape[1] if hnd else k_cache.shape[2]
+    if problem.Hkv != Hkv:
+        raise ValueError(f"problem Hkv = {problem.Hkv}, the cache holds {Hkv} KV heads")
+    if problem.block_size:
+        bs = k_cache.shape[2] if hnd else k_cache.shape[1]
+        if (problem.block_size, problem.num_blocks) != (bs, k_cache.shape[0]):
+            raise ValueError(f"problem pages {(problem.num_blocks, problem.block_size)}, the "
+                             f"cache holds {(k_cache.shape[0], bs)}")
 
 
 def decode(q, k_cache, v_cache, seqlens=None, block_table=None, *, max_len: Optional[int] = None,

@@ -60,19 +60,30 @@ struct PlanModel {
   static constexpr double kCombinePer16Us = 2.0;
 };
 
-int tile_round_up(long long x) {
-  return static_cast<int>((x + fd::kTile - 1) / fd::kTile * fd::kTile);
+// How a call cuts the history: T = ceil(max_len / 64) tiles into S = min(S
+// requested, T) splits (1 when T = 0); split s covers the tiles
+// [floor(s T / S), floor((s + 1) T / S)) of every sequence, so the splits
+// differ by at most one tile and the largest has ceil(T / S).
+struct Chunking {
+  int tiles;      // T
+  int splits;     // S, the effective split count
+  int max_tiles;  // ceil(T / S)
+};
+
+Chunking chunking(int max_len, int num_splits) {
+  const int T = max_len > 0 ? static_cast<int>((static_cast<long long>(max_len) + fd::kTile - 1) /
+                                                fd::kTile)
+                            : 0;
+  const int S = T == 0 ? 1 : std::min(num_splits, T);
+  return Chunking{T, S, T == 0 ? 0 : (T + S - 1) / S};
 }
 
-int chunk_for(int max_len, int num_splits) {
-  const long long per = (static_cast<long long>(max_len) + num_splits - 1) / num_splits;
-  const int c = tile_round_up(per);
-  return c < fd::kTile ? fd::kTile : c;
-}
-
-int effective_splits(int max_len, int chunk) {
-  if (max_len <= 0) return 1;
-  return static_cast<int>((static_cast<long long>(max_len) + chunk - 1) / chunk);
+// Splits that hold tokens of a sequence of n tokens (the kernels' rule).
+int split_parts(const Chunking& c, long long n) {
+  const long long m = (n + fd::kTile - 1) / fd::kTile;
+  if (m <= 0) return 0;
+  const long long p = (m * c.splits + c.tiles - 1) / c.tiles;
+  return static_cast<int>(std::min<long long>(p, c.splits));
 }
 
 // What the model needs to know of a problem besides its lengths.
@@ -121,24 +132,25 @@ double model_time_us(const PlanShape& ps, double n_ctas, double tokens, double m
 
 // The model for a batch whose sequences all hold max_len tokens.
 double model_time_uniform(const PlanShape& ps, int B, int max_len, int S) {
-  const int chunk = chunk_for(max_len, S);
-  const int s_eff = effective_splits(max_len, chunk);
+  const Chunking c = chunking(max_len, S);
   const double units = static_cast<double>(B) * ps.Hkv;
-  return model_time_us(ps, units * s_eff, units * max_len, std::min(chunk, max_len), s_eff);
+  return model_time_us(ps, units * c.splits, units * max_len,
+                       std::min<double>(static_cast<double>(c.max_tiles) * fd::kTile, max_len),
+                       c.splits);
 }
 
 // The model for given per-sequence lengths (clamped to [0, max_len]).
 double model_time_lengths(const PlanShape& ps, int B, int max_len, const int32_t* lens, int S) {
-  const int chunk = chunk_for(max_len, S);
-  const int s_eff = effective_splits(max_len, chunk);
+  const Chunking c = chunking(max_len, S);
+  const double largest = static_cast<double>(c.max_tiles) * fd::kTile;
   double n_ctas = 0.0, tokens = 0.0, max_tok = 0.0;
   for (int b = 0; b < B; ++b) {
     const double n = std::min<double>(std::max<int32_t>(lens[b], 0), max_len);
-    n_ctas += std::ceil(n / chunk);
+    n_ctas += split_parts(c, static_cast<long long>(n));
     tokens += n;
-    max_tok = std::max(max_tok, std::min<double>(n, chunk));
+    max_tok = std::max(max_tok, std::min(n, largest));
   }
-  return model_time_us(ps, n_ctas * ps.Hkv, tokens * ps.Hkv, max_tok, s_eff);
+  return model_time_us(ps, n_ctas * ps.Hkv, tokens * ps.Hkv, max_tok, c.splits);
 }
 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
@@ -197,6 +209,33 @@ fd_status device_is_sm100(int dev) {
     g_dev[dev].sm100.store(v);
   }
   return v ? FD_OK : FD_ERR_UNSUPPORTED;
+}
+
+// Unique id of the calling thread's current CUDA context, or 0 when it cannot
+// be read.  A device reset destroys the primary context; the next runtime
+// call creates a new one, with a new id, in which the module is loaded again:
+// device symbols may then sit at other addresses and function attributes are
+// back at their defaults.  Per-device set-up is therefore keyed by this id.
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 4000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  unsigned long long id = 0;
+  return get_id(ctx, &id) == CUDA_SUCCESS ? id : 0;
 }
 
 // ------------------------------------------------------------ tensor maps
@@ -294,11 +333,18 @@ fd_status cached_cache_map(CUtensorMap* tm, const MapKey& key) {
 
 // --------------------------------------------------------------- launches
 
-// Stages of the split kernel's ring: about 96 KB, two CTAs per SM; DEEP
-// (bf16, D = 128, a grid of at most one CTA per SM): 4 stages, 128 KB.
-template <int D, bool FP8, bool DEEP>
+// Stages of the split kernel's ring: about 96 KB, two CTAs per SM.  DEEP
+// (bf16, D = 128, a grid of at most one CTA per SM): the CTA has its SM to
+// itself and runs eight consumer warps over a 6-stage ring (192 KB; the
+// sparse decode, whose scan stages hold 32 KB of codes, 4 stages).
+template <int D, bool FP8, bool DEEP, bool SPARSE>
 constexpr int split_stages() {
-  return (D == 128 && !FP8) ? (DEEP ? 4 : 3) : 6;
+  return (D == 128 && !FP8) ? (DEEP ? (SPARSE ? 4 : 6) : 3) : 6;
+}
+
+template <bool DEEP, bool SPARSE>
+constexpr int split_consumer_warps() {
+  return DEEP ? fd::kWideConsumerWarps : fd::kConsumerWarps;
 }
 
 template <int D, int NB, int MODE, bool PAGED, bool FP8 = false, bool DEEP = false,
@@ -306,24 +352,26 @@ template <int D, int NB, int MODE, bool PAGED, bool FP8 = false, bool DEEP = fal
 fd_status launch_split(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tc,
                        const fd::SplitArgs& a, int n_splits, int Hkv, int B,
                        cudaStream_t stream) {
-  constexpr int STAGES = split_stages<D, FP8, DEEP>();
-  using L = fd::SplitSmem<D, NB, STAGES, FP8, SPARSE>;
-  auto kern = fd::fd_split_kernel<D, NB, MODE, PAGED, STAGES, FP8, SPARSE>;
-  // The shared-memory opt-in is per device; remember which devices have it.
-  static std::atomic<unsigned long long> attr_done{0};
+  constexpr int STAGES = split_stages<D, FP8, DEEP, SPARSE>();
+  constexpr int CW = split_consumer_warps<DEEP, SPARSE>();
+  using L = fd::SplitSmem<D, NB, STAGES, FP8, SPARSE, CW>;
+  auto kern = fd::fd_split_kernel<D, NB, MODE, PAGED, STAGES, FP8, SPARSE, CW>;
+  // The shared-memory opt-in belongs to the device's context; remember the
+  // context in which each device got it (0: not yet, or the id is unknown).
+  static std::atomic<unsigned long long> attr_ctx[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FD_ERR_CUDA;
-  const unsigned long long bit = 1ull << dev;
-  if (!(attr_done.load() & bit)) {
+  const unsigned long long ctx = current_context_id();
+  if (ctx == 0 || attr_ctx[dev].load() != ctx) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              L::kDynamicBytes) != cudaSuccess)
       return FD_ERR_CUDA;
-    attr_done.fetch_or(bit);
+    attr_ctx[dev].store(ctx);
   }
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(n_splits), static_cast<unsigned>(Hkv),
                      static_cast<unsigned>(B));
-  cfg.blockDim = dim3(fd::kThreads);
+  cfg.blockDim = dim3(fd::split_threads<CW>());
   cfg.dynamicSmemBytes = L::kDynamicBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -411,30 +459,24 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // The split count with the lowest modelled time; a larger count must win by
-// more than 2 % (fewer splits mean fewer partials to merge).
+// more than 2 % (fewer splits mean fewer partials to merge).  Counts beyond
+// two CTAs per SM slot, from the batch's units alone, only add waves, so the
+// search stops there.
 template <class Model>
-int pick_splits(int max_len, Model model) {
+int pick_splits(int max_len, long long units, int slots, Model model) {
   const long long tiles = (static_cast<long long>(max_len) + fd::kTile - 1) / fd::kTile;
   if (tiles <= 1) return 1;
-  const int s_max = static_cast<int>(std::min<long long>(tiles, kMaxSplits));
+  const long long fill = (2LL * slots + units - 1) / std::max(units, 1LL);
+  const int s_max = static_cast<int>(std::min<long long>(std::min<long long>(tiles, kMaxSplits),
+                                                         std::max(fill, 1LL)));
   int best = 1;
   double best_t = model(1);
-  int last_eff = 1;
-  for (int S = 2; S <= s_max;) {
-    // Split S has c = ceil(tiles / S) tiles; every S up to `last` has the
-    // same chunking (and effective count), so only the first is evaluated.
-    const long long c = (tiles + S - 1) / S;
-    const long long last = c > 1 ? (tiles - 1) / (c - 1) : s_max;
-    const int eff = effective_splits(max_len, chunk_for(max_len, S));
-    if (eff != last_eff) {  // otherwise the same chunking as a smaller S
-      last_eff = eff;
-      const double t = model(S);
-      if (t < best_t * 0.98) {
-        best_t = t;
-        best = S;
-      }
+  for (int S = 2; S <= s_max; ++S) {
+    const double t = model(S);
+    if (t < best_t * 0.98) {
+      best_t = t;
+      best = S;
     }
-    S = static_cast<int>(std::min<long long>(last, s_max)) + 1;
   }
   return best;
 }
@@ -486,13 +528,13 @@ fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
     if (!sp->k8 || !sp->k8_scale || !aligned(sp->k8, 16) || !aligned(sp->k8_scale, 4) ||
         std::isnan(sp->delta) || sp->delta < 0.f)
       return FD_ERR_INVALID_ARGUMENT;
-    if (chunk_for(p->max_len, num_splits) > fd::kMaxSparseTiles * fd::kTile)
+    if (chunking(p->max_len, num_splits).max_tiles > fd::kMaxSparseTiles)
       return FD_ERR_INVALID_ARGUMENT;
   }
 
   const int B = p->B, Hq = p->Hq, Hkv = p->Hkv, D = p->D, G = Hq / Hkv;
-  const int chunk = chunk_for(p->max_len, num_splits);
-  const int n_splits = effective_splits(p->max_len, chunk);
+  const Chunking chunks = chunking(p->max_len, num_splits);
+  const int n_splits = chunks.splits;
   float* part_o = nullptr;
   float* part_lse = nullptr;
   if (n_splits > 1) {
@@ -542,14 +584,17 @@ fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
   a.log2_block_size = paged ? ilog2(p->block_size) : 0;
   a.log2_box_rows = ilog2(box_rows);
   a.max_blocks_per_seq = paged ? p->max_blocks_per_seq : 0;
-  a.chunk = chunk;
+  a.tiles = chunks.tiles;
   a.n_splits = n_splits;
+  a.tile_q = chunks.tiles / n_splits;
+  a.tile_r = chunks.tiles % n_splits;
   a.scale_log2 = scale * (fp8 ? p->k_scale : 1.f) * 1.4426950408889634074f;
   a.v_scale = fp8 ? p->v_scale : 1.f;
   // L2 prefetch ahead of the wait on the previous grid (contiguous caches):
   // half the split's tiles, at most kPrefetchTiles.  Swept on B200 over
   // 0..12 tiles at 4K..64K tokens, bf16 and fp8, S = 16 and 32.
-  a.prefetch_tiles = (paged || sp) ? 0 : std::min(kPrefetchTiles, std::max(1, chunk / fd::kTile / 2));
+  a.prefetch_tiles =
+      (paged || sp) ? 0 : std::min(kPrefetchTiles, std::max(1, chunks.max_tiles / 2));
   a.scale = scale;
   if (sp) {
     a.k8 = sp->k8;
@@ -588,11 +633,14 @@ int plan_impl(int num_sms, int B, int Hkv, int D, int max_len, int block_size, i
   const PlanShape ps{num_sms, B, Hkv, 2.0 * D * elem_bytes,
                      block_size > 0 && block_size < fd::kTile, elem_bytes == 2 && D == 128,
                      elem_bytes == 1};
+  const long long units = static_cast<long long>(B) * Hkv;
+  const int slots = num_sms * fd::kCtasPerSm;
   if (seqlens)
-    return pick_splits(max_len, [&](int S) {
+    return pick_splits(max_len, units, slots, [&](int S) {
       return model_time_lengths(ps, B, max_len, seqlens, S);
     });
-  return pick_splits(max_len, [&](int S) { return model_time_uniform(ps, B, max_len, S); });
+  return pick_splits(max_len, units, slots,
+                     [&](int S) { return model_time_uniform(ps, B, max_len, S); });
 }
 
 }  // namespace
@@ -613,7 +661,12 @@ const char* fd_status_string(fd_status status) {
 
 int fd_split_chunk(int max_len, int num_splits) {
   if (max_len < 0 || num_splits < 1 || num_splits > kMaxSplits) return FD_ERR_INVALID_ARGUMENT;
-  return chunk_for(max_len, num_splits);
+  return std::max(1, chunking(max_len, num_splits).max_tiles) * fd::kTile;
+}
+
+int fd_effective_splits(int max_len, int num_splits) {
+  if (max_len < 0 || num_splits < 1 || num_splits > kMaxSplits) return FD_ERR_INVALID_ARGUMENT;
+  return chunking(max_len, num_splits).splits;
 }
 
 int fd_plan_sm(int num_sms, int B, int Hq, int Hkv, int D, int max_len, int block_size) {
@@ -730,6 +783,14 @@ fd_status fd_decode_sparse(const fd_problem* p, const void* q, const void* k_cac
 
 fd_status fd_combine(int R, int B, int Hq, int D, const float* part_o, const float* part_lse,
                      void* out, float* lse, fd_stream_t stream) {
+  const size_t rows = static_cast<size_t>(B > 0 ? B : 0) * static_cast<size_t>(Hq > 0 ? Hq : 0);
+  return fd_combine_strided(R, B, Hq, D, part_o, rows * static_cast<size_t>(D > 0 ? D : 0),
+                            part_lse, rows, out, lse, stream);
+}
+
+fd_status fd_combine_strided(int R, int B, int Hq, int D, const float* part_o, size_t o_stride,
+                             const float* part_lse, size_t lse_stride, void* out, float* lse,
+                             fd_stream_t stream) {
   if (R < 1 || R > kMaxSplits || B < 1 || Hq < 1 || !part_o || !part_lse || !out)
     return FD_ERR_INVALID_ARGUMENT;
   if (D != 64 && D != 128) return FD_ERR_UNSUPPORTED;
@@ -737,6 +798,11 @@ fd_status fd_combine(int R, int B, int Hq, int D, const float* part_o, const flo
     return FD_ERR_INVALID_ARGUMENT;
   const long long rows = static_cast<long long>(B) * Hq;
   if (rows > (1ll << 30)) return FD_ERR_INVALID_ARGUMENT;
+  // Every part starts 16 bytes aligned and holds its rows; lse entries of a
+  // part do not overlap the next part's.
+  if (o_stride % 4 != 0 || o_stride < static_cast<size_t>(rows) * D ||
+      lse_stride < static_cast<size_t>(rows))
+    return FD_ERR_INVALID_ARGUMENT;
   int dev = 0;
   if (current_device(&dev) != FD_OK) return FD_ERR_CUDA;
   const fd_status arch = device_is_sm100(dev);
@@ -753,8 +819,10 @@ fd_status fd_combine(int R, int B, int Hq, int D, const float* part_o, const flo
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
   const int r = static_cast<int>(rows);
   const cudaError_t e = D == 128
-      ? cudaLaunchKernelEx(&cfg, fd::fd_merge_kernel<128>, part_o, part_lse, R, r, o, lse)
-      : cudaLaunchKernelEx(&cfg, fd::fd_merge_kernel<64>, part_o, part_lse, R, r, o, lse);
+      ? cudaLaunchKernelEx(&cfg, fd::fd_merge_kernel<128>, part_o, part_lse, R, r, o_stride,
+                           lse_stride, o, lse)
+      : cudaLaunchKernelEx(&cfg, fd::fd_merge_kernel<64>, part_o, part_lse, R, r, o_stride,
+                           lse_stride, o, lse);
   return e == cudaSuccess ? FD_OK : FD_ERR_CUDA;
 }
 
@@ -770,19 +838,34 @@ fd_status fd_decode_static_workspace(const fd_problem* p, const void* q, const v
   if (!p || num_splits < 1 || num_splits > kMaxSplits) return FD_ERR_INVALID_ARGUMENT;
   const fd_status st = check_shape(p->B, p->Hq, p->Hkv, p->D, p->max_len, p->block_size);
   if (st != FD_OK) return st;
-  const int n_splits = effective_splits(p->max_len, chunk_for(p->max_len, num_splits));
+  const int n_splits = chunking(p->max_len, num_splits).splits;
   const size_t need = n_splits > 1 ? fd_workspace_bytes(p->B, p->Hq, p->D, n_splits) : 0;
   if (need > FD_STATIC_WORKSPACE_BYTES) return FD_ERR_WORKSPACE;
 
-  // Set-up, once per device, with that device current: the host-side name of
+  // Set-up, once per device (and again after a device reset, which gives the
+  // device a new context), with that device current: the host-side name of
   // the array is not a device address; ask the runtime for the real one.
-  static std::atomic<void*> ws_ptr[kMaxDevices];
+  struct StaticSlot {
+    std::mutex m;
+    unsigned long long ctx = 0;
+    void* ptr = nullptr;
+  };
+  static StaticSlot slots[kMaxDevices];
   int dev = 0;
   if (current_device(&dev) != FD_OK) return FD_ERR_CUDA;
-  void* ws = ws_ptr[dev].load();
-  if (!ws) {
-    if (cudaGetSymbolAddress(&ws, g_static_workspace) != cudaSuccess || !ws) return FD_ERR_CUDA;
-    ws_ptr[dev].store(ws);
+  void* ws = nullptr;
+  {
+    StaticSlot& sl = slots[dev];
+    std::lock_guard<std::mutex> lock(sl.m);
+    const unsigned long long ctx = current_context_id();
+    if (ctx != 0 && sl.ptr && sl.ctx == ctx) {
+      ws = sl.ptr;
+    } else {
+      if (cudaGetSymbolAddress(&ws, g_static_workspace) != cudaSuccess || !ws)
+        return FD_ERR_CUDA;
+      sl.ptr = ws;
+      sl.ctx = current_context_id();  // the lookup makes the context current if it was not
+    }
   }
   return fd_decode(p, q, k_cache, v_cache, seqlens, block_table, scale, num_splits, out, lse, ws,
                    FD_STATIC_WORKSPACE_BYTES, stream);

@@ -31,9 +31,16 @@
 namespace fd {
 
 constexpr int kTile = 64;           // tokens per pipeline stage
-constexpr int kConsumerWarps = 4;   // each takes 16 tokens of every tile
+constexpr int kTileWarps = 4;       // consumer warps per tile, 16 tokens each
+constexpr int kConsumerWarps = 4;   // consumer warps of a CTA sized for two CTAs per SM
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kCtasPerSm = 2;       // occupancy the split kernel is sized for
+// A CTA alone on its SM runs two sets of four consumer warps, which take the
+// even and the odd tiles: one warp per SM sub-partition is bound by the
+// latency of its tile loop, two hide it.
+constexpr int kWideConsumerWarps = 8;
+template <int CW>
+constexpr int split_threads() { return (CW + 1) * 32; }
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
 
 // How the softmax weights P enter the bf16 P.V contraction.
@@ -63,8 +70,9 @@ struct SplitArgs {
   int block_size, log2_block_size;
   int log2_box_rows;            // rows per TMA box: 64, or the page size when smaller
   int max_blocks_per_seq;
-  int chunk;                    // tokens per split, a multiple of kTile
-  int n_splits;                 // effective split count = gridDim.x
+  int tiles;                    // 64-token tiles of max_len, T = ceil(max_len / 64)
+  int n_splits;                 // effective split count S = gridDim.x, 1 <= S <= max(T, 1)
+  int tile_q, tile_r;           // T = tile_q * S + tile_r, 0 <= tile_r < S
   float scale_log2;             // scale * k_scale * log2(e)
   float v_scale;                // dequantisation scale of an fp8 V cache (1 for bf16)
   int prefetch_tiles;           // contiguous caches: tiles per CTA prefetched into L2 before
@@ -101,6 +109,24 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 
 __device__ __forceinline__ float round_to_bf16(float x) {
   return __bfloat162float(__float2bfloat16_rn(x));
+}
+
+// Split s of S covers the tiles [floor(s T / S), floor((s + 1) T / S)) of
+// every sequence: the splits differ by at most one tile, so any S up to T
+// gives CTAs of balanced size.  With T = q S + r, floor(s T / S) =
+// s q + floor(s r / S), and s r < S^2 <= 2^20 stays in 32 bits.
+__device__ __forceinline__ int split_first_tile(const SplitArgs& a, int s) {
+  return s * a.tile_q + static_cast<int>(static_cast<unsigned>(s * a.tile_r) /
+                                         static_cast<unsigned>(a.n_splits));
+}
+
+// Splits that hold tokens of a sequence of n tokens: those whose first tile
+// is below m = ceil(n / 64), i.e. ceil(m S / T) of them.
+__device__ __forceinline__ int split_parts(const SplitArgs& a, int n) {
+  const long long m = (n + kTile - 1) / kTile;
+  if (m == 0) return 0;
+  const long long p = (m * a.n_splits + a.tiles - 1) / a.tiles;
+  return static_cast<int>(p < a.n_splits ? p : a.n_splits);
 }
 
 __device__ __forceinline__ int seq_length(const int32_t* seqlens, int b, int max_len) {
@@ -190,7 +216,8 @@ __device__ __forceinline__ void combine_row(const float* po, const float* pl, in
   if (lse_out && lane == 0) *lse_out = mx == -INFINITY ? -INFINITY : mx + logf(W);
 }
 
-template <int D, int NB, int STAGES, bool FP8 = false, bool SPARSE = false>
+template <int D, int NB, int STAGES, bool FP8 = false, bool SPARSE = false,
+          int CW = kConsumerWarps>
 struct SplitSmem {
   // Rows are stored in 128-byte swizzle rows: a bf16 row of D = 128 takes two
   // (its column halves), an fp8 row of 128 takes one.
@@ -216,9 +243,9 @@ struct SplitSmem {
   // arithmetic spilled, so those rows stay unpadded.)
   static constexpr int kAccStride = NB == 1 ? D + 4 : D;
   static constexpr int kRedAcc = 0;                                   // [warp][col][kAccStride]
-  static constexpr int kRedM = kRedAcc + kConsumerWarps * kNcol * kAccStride;  // [warp][col]
-  static constexpr int kRedL = kRedM + kConsumerWarps * kNcol;        // [warp][col]
-  static constexpr int kScratchFloats = kRedL + kConsumerWarps * kNcol;
+  static constexpr int kRedM = kRedAcc + CW * kNcol * kAccStride;     // [warp][col]
+  static constexpr int kRedL = kRedM + CW * kNcol;                    // [warp][col]
+  static constexpr int kScratchFloats = kRedL + CW * kNcol;
   static_assert(kScratchFloats * 4 <= kBarOffset, "epilogue scratch must fit the pipeline buffers");
 };
 
@@ -227,12 +254,13 @@ struct SplitSmem {
 // keys selects blocks by a top-delta rule that each unit of work applies on
 // its own, with no global synchronisation).  The consumer warps' part of the
 // scan: the int8 key codes of the split stream through the same mbarrier ring
-// as the K/V tiles, kScanTilesPerStage blocks per stage, and warp w takes
-// block w of each stage.  Per block and head the largest approximate logit
+// as the K/V tiles, kScanTilesPerStage blocks per stage; with CW consumer
+// warps, warp w takes block w mod 4 of every (CW / 4)-th stage, starting at
+// stage w / 4.  Per block and head the largest approximate logit
 // ((scale * sq) * sk) * (q8 . k8) goes to bmax: the dot products are exact
 // (int8 tensor cores, int32 accumulation), each product is rounded to fp32
 // in that order, and q8 = rint(q / sq) with sq = max |q| / 127.
-template <int D, int NB, int STAGES, int STAGE_BYTES>
+template <int D, int NB, int STAGES, int STAGE_BYTES, int CW>
 __device__ __forceinline__ bool sparse_scan_consumer(const SplitArgs& a, uint32_t smem_base,
                                                      uint32_t bar_full, uint32_t bar_empty,
                                                      float* bmax, int warp, int lane, int b,
@@ -241,6 +269,8 @@ __device__ __forceinline__ bool sparse_scan_consumer(const SplitArgs& a, uint32_
   static_assert(D == 128, "the scan reads 128-byte code rows");
   constexpr int KSTEPS = D / 32;
   static_assert(STAGE_BYTES >= kScanTilesPerStage * kTile * D, "a scan stage fits a ring stage");
+  static_assert(kScanTilesPerStage == kTileWarps, "one block per warp of a set");
+  constexpr int kSets = CW / kTileWarps;
   // B fragments of q8 (k = head dim, n = head): lane (g, t) holds entries
   // 32c + 4t .. +3 and 32c + 16 + 4t .. +3 of head nb*8 + g.
   uint32_t qb[NB][KSTEPS][2];
@@ -289,11 +319,11 @@ __device__ __forceinline__ bool sparse_scan_consumer(const SplitArgs& a, uint32_
 
   const size_t srow = (static_cast<size_t>(b) * a.Hkv + (h0 / a.G)) * a.n_blocks + start / kTile;
   const int g = lane >> 2, t = lane & 3;
-  for (int j = 0; j < n_scan; ++j) {
+  for (int j = warp / kTileWarps; j < n_scan; j += kSets) {
     const int s = j % STAGES, k = j / STAGES;
     const bool ok = mbar_wait(bar_full + 8 * s, k & 1, kWaitLimitNs);
     if (!__all_sync(0xffffffffu, ok)) return false;
-    const int blk = kScanTilesPerStage * j + warp;
+    const int blk = kScanTilesPerStage * j + warp % kTileWarps;
     if (blk < n_tiles) {
       const float sk = a.k8_scale[srow + blk];
       const uint32_t sb = smem_base + s * STAGE_BYTES;
@@ -307,7 +337,8 @@ __device__ __forceinline__ bool sparse_scan_consumer(const SplitArgs& a, uint32_
         for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
           for (int i = 0; i < 4; ++i) acc[nb][i] = 0;
-        const uint32_t row = warp * kTile + mg * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+        const uint32_t row = (warp % kTileWarps) * kTile + mg * 16 + ((lane >> 3) & 1) * 8 +
+                             (lane & 7);
 #pragma unroll
         for (int kp = 0; kp < KSTEPS; ++kp) {
           const uint32_t chunk16 = 2 * kp + (lane >> 4);
@@ -343,17 +374,31 @@ __device__ __forceinline__ bool sparse_scan_consumer(const SplitArgs& a, uint32_
 }
 
 // Consumer warps of the split kernel: scores, online softmax and P.V over the
-// split's tiles, then the merge of the four warps' softmax states into this
+// split's tiles, then the merge of the CW warps' softmax states into this
 // split's result, which goes to `out` (the sequence has one split) or to the
-// global partials (several splits).
-template <int D, int NB, int MODE, int STAGES, bool FP8, bool SPARSE>
+// global partials (several splits).  Warp w takes tokens 16 (w mod 4) ..
+// +15 of every (CW / 4)-th tile, starting at tile w / 4.
+template <int D, int NB, int MODE, int STAGES, bool FP8, bool SPARSE, int CW = kConsumerWarps>
 __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* smem,
                                                 uint32_t smem_base, uint32_t bar_full,
                                                 uint32_t bar_empty, volatile int* cta_error,
                                                 int warp, int lane, int b, int h0, int split,
                                                 int start, int end, int n_tiles, int n_parts,
                                                 const uint16_t* list, int it_base) {
-  using L = SplitSmem<D, NB, STAGES, FP8, SPARSE>;
+  using L = SplitSmem<D, NB, STAGES, FP8, SPARSE, CW>;
+  static_assert(CW % kTileWarps == 0, "whole sets of tile warps");
+  constexpr int kSets = CW / kTileWarps;   // tiles in flight among the consumers
+  // A set must see every phase of the stages it reads (a parity wait cannot
+  // tell phase k from phase k - 2).  STAGES is a multiple of kSets, so the
+  // tiles that share a stage (indices congruent modulo STAGES) belong to one
+  // set.  Before the tiles, the sparse scan's stages (sets by stage index)
+  // all complete ahead of a CTA-wide barrier, so a stage's first tile use
+  // never waits behind another set's scan use.  Tiles go to sets by tile
+  // index, which keeps the warp that sums each tile the same with or
+  // without a scan in front.
+  static_assert(STAGES % kSets == 0, "every stage belongs to one set of warps");
+  const int wr = warp % kTileWarps;        // this warp's 16-token slice of a tile
+  const int set = warp / kTileWarps;       // first tile of this warp
   constexpr int KSTEPS = D / 16;   // k-steps of the score MMA (over D)
   constexpr int DBLK = D / 16;     // m-blocks of the P.V MMA (over D)
   constexpr int NCOL = NB * 8;     // MMA columns (query heads, maybe doubled)
@@ -417,8 +462,8 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
   // 4t, 4t+1 and 4t+2, 4t+3: the order in which the byte-transposing
   // ldmatrix delivers V (see ldmatrix_x2_trans_b8).
   const uint32_t r16 = ((lane >> 3) & 1) * 8 + (lane & 7);
-  const uint32_t rowK = warp * 16 + (FP8 ? perm16(r16) : r16);
-  const uint32_t rowV = warp * 16 + (FP8 ? (lane & 15) : (lane >> 4) * 8 + (lane & 7));
+  const uint32_t rowK = wr * 16 + (FP8 ? perm16(r16) : r16);
+  const uint32_t rowV = wr * 16 + (FP8 ? (lane & 15) : (lane >> 4) * 8 + (lane & 7));
   const uint32_t x7 = lane & 7;              // swizzle phase of rowV (and of rowK if not FP8)
   const uint32_t xk = rowK & 7;
   const uint32_t lgr = a.log2_box_rows;
@@ -427,12 +472,12 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
   const uint32_t offK = (rowK >> lgr) * box_bytes + (rowK & ((1u << lgr) - 1)) * 128;
   const uint32_t offV = (rowV >> lgr) * box_bytes + (rowV & ((1u << lgr) - 1)) * 128;
   // Token rows of the C fragment held by this lane.
-  const int r_lo = warp * 16 + (FP8 ? perm16(lane >> 2) : (lane >> 2));
-  const int r_hi = warp * 16 + (FP8 ? perm16((lane >> 2) + 8) : (lane >> 2) + 8);
+  const int r_lo = wr * 16 + (FP8 ? perm16(lane >> 2) : (lane >> 2));
+  const int r_hi = wr * 16 + (FP8 ? perm16((lane >> 2) + 8) : (lane >> 2) + 8);
   const float sl2 = a.scale_log2;
   bool failed = false;
 
-  for (int it = 0; it < n_tiles; ++it) {
+  for (int it = set; it < n_tiles; it += kSets) {
     const int ig = it_base + it;                 // ring use, after any scan stages
     const int s = ig % STAGES, k = ig / STAGES;
     const bool ok = mbar_wait(bar_full + 8 * s, k & 1, kWaitLimitNs);
@@ -557,11 +602,11 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
     uint32_t vmask_lo = 0xffffffffu, vmask_hi = 0xffffffffu;
     if (partial) {
       if constexpr (FP8) {  // bytes i of a register: token 4t + i
-        const int tk = warp * 16 + 4 * (lane & 3);
+        const int tk = wr * 16 + 4 * (lane & 3);
         vmask_lo = (tk < tile_valid ? 0xffu : 0u) | (tk + 1 < tile_valid ? 0xff00u : 0u) |
                    (tk + 2 < tile_valid ? 0xff0000u : 0u) | (tk + 3 < tile_valid ? 0xff000000u : 0u);
       } else {
-        const int tk = warp * 16 + 2 * (lane & 3);
+        const int tk = wr * 16 + 2 * (lane & 3);
         vmask_lo = (tk < tile_valid ? 0x0000ffffu : 0u) | (tk + 1 < tile_valid ? 0xffff0000u : 0u);
         vmask_hi = (tk + 8 < tile_valid ? 0x0000ffffu : 0u) | (tk + 9 < tile_valid ? 0xffff0000u : 0u);
       }
@@ -640,7 +685,7 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
   // Every consumer warp is past its last shared-memory read of the pipeline,
   // so the drained buffers hold the epilogue scratch: each warp's
   // accumulator [warp][col][D] and its running max and sum per column.
-  named_barrier_sync(1, kConsumerWarps * 32);
+  named_barrier_sync(1, CW * 32);
   float* f = reinterpret_cast<float*>(smem);
   const bool live = !*cta_error;
   if (live) {
@@ -666,46 +711,46 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
       }
     }
   }
-  named_barrier_sync(1, kConsumerWarps * 32);
+  named_barrier_sync(1, CW * 32);
   if (!live) return;
 
-  // One pass with no further barrier.  Each thread merges the four warp
+  // One pass with no further barrier.  Each thread merges the CW warp
   // states for 8 head-dim entries of one head (4 at d0 and 4 at d0 + D/2, so
   // that a warp's 16-byte reads and writes are contiguous) and computes that
   // head's weights itself from a few broadcast reads.  (A separate per-head
   // pass behind two more barriers took about 1.5 us per CTA.)
   constexpr int kChunks = D / 8;  // chunks of 8 entries per head
   const bool direct = n_parts == 1;
-  for (int c = threadIdx.x; c < a.G * kChunks; c += kConsumerWarps * 32) {
+  for (int c = threadIdx.x; c < a.G * kChunks; c += CW * 32) {
     const int g = c / kChunks;
     const int d0 = (c - g * kChunks) * 4;
-    float mw[kConsumerWarps];
+    float mw[CW];
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) {
+    for (int w = 0; w < CW; ++w) {
       mw[w] = f[L::kRedM + w * NCOL + g];
       M = fmaxf(M, mw[w]);
     }
-    float wt[kConsumerWarps];
+    float wt[CW];
     float lse_s = -INFINITY;
     if (M == -INFINITY) {  // no token in this split
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) wt[w] = 0.f;
+      for (int w = 0; w < CW; ++w) wt[w] = 0.f;
     } else {
       float Ls = 0.f;
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
+      for (int w = 0; w < CW; ++w) {
         wt[w] = ex2(mw[w] - M);
         Ls += wt[w] * f[L::kRedL + w * NCOL + g];
       }
       const float inv = a.v_scale / Ls;  // an fp8 V cache is dequantised here
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) wt[w] *= inv;
+      for (int w = 0; w < CW; ++w) wt[w] *= inv;
       lse_s = (M + log2f(Ls)) * 0.69314718055994530942f;
     }
     float4 o[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) {
+    for (int w = 0; w < CW; ++w) {
       const float* src = f + L::kRedAcc + (w * NCOL + g) * L::kAccStride + d0;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -748,13 +793,16 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
 
 // Split kernel: one CTA per (split, KV head, sequence).  FP8: the cache
 // holds e4m3 values (D = 128); the contraction runs on f16 tensor cores.
-template <int D, int NB, int MODE, bool PAGED, int STAGES, bool FP8, bool SPARSE = false>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+// CW consumer warps and one producer warp; kWideConsumerWarps for a CTA
+// that has its SM to itself.
+template <int D, int NB, int MODE, bool PAGED, int STAGES, bool FP8, bool SPARSE = false,
+          int CW = kConsumerWarps>
+__global__ void __launch_bounds__(split_threads<CW>(), CW == kConsumerWarps ? kCtasPerSm : 1)
     fd_split_kernel(const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ CUtensorMap tmC,   // sparse: int8 key codes
                     const SplitArgs a) {
-  using L = SplitSmem<D, NB, STAGES, FP8, SPARSE>;
+  using L = SplitSmem<D, NB, STAGES, FP8, SPARSE, CW>;
   static_assert(!SPARSE || (!PAGED && !FP8), "sparse decode: contiguous bf16 caches");
   static_assert(MODE != kDup || NB == 1, "duplicated columns need one column block");
 
@@ -775,12 +823,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_empty + 8 * s, kConsumerWarps);
+      mbar_init(bar_empty + 8 * s, kTileWarps);   // the four warps that read a tile
     }
     *cta_error = 0;
     fence_mbar_init();
   }
-  if (warp == kConsumerWarps && lane == 0) {
+  if (warp == CW && lane == 0) {
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
   }
@@ -788,9 +836,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     // While the previous grid finishes, pull the first tiles of this split
     // into L2, one tile per lane.  Only kernel arguments are used (the
     // lengths may still be in flight), so the range stops at max_len.
-    if (warp == kConsumerWarps && lane < a.prefetch_tiles) {
-      const int t0 = split * a.chunk + lane * kTile;
-      if (lane * kTile < a.chunk && t0 < a.max_len) {
+    if (warp == CW && lane < a.prefetch_tiles) {
+      const int tile0 = split_first_tile(a, split);
+      const int t0 = (tile0 + lane) * kTile;
+      if (tile0 + lane < split_first_tile(a, split + 1) && t0 < a.max_len) {
         tma_prefetch_l2_5d(&tmK, 0, kvh, t0, 0, b);
         tma_prefetch_l2_5d(&tmV, 0, kvh, t0, 0, b);
       }
@@ -802,19 +851,22 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   grid_dependency_wait();
 
   const int n = seq_length(a.seqlens, b, a.max_len);
-  const int start = split * a.chunk;
-  const int end = min(start + a.chunk, n);
+  const int start = split_first_tile(a, split) * kTile;
+  const int end = min(split_first_tile(a, split + 1) * kTile, n);
   const int h0 = kvh * a.G;
   const int n_tiles = start < end ? (end - start + kTile - 1) / kTile : 0;
   // Splits of this sequence that hold tokens.
-  const int n_parts = min((n + a.chunk - 1) / a.chunk, a.n_splits);
+  // Whether the sequence has tokens in other splits than split 0 (then this
+  // split's result is a partial for the combine kernel): 1 = only split 0,
+  // 2 = several.  Split 0 holds tiles [0, tile_q).
+  const int n_parts = (a.n_splits == 1 || (n + kTile - 1) / kTile <= a.tile_q) ? 1 : 2;
 
   if (n_tiles == 0) {
     // Empty split.  Split 0 is empty only for an empty sequence, whose
     // result is out = 0, lse = -inf; other empty splits take no part.
     if (split == 0) {
       const size_t base = (static_cast<size_t>(b) * a.Hq + h0) * D;
-      for (int i = threadIdx.x; i < a.G * D; i += kThreads) {
+      for (int i = threadIdx.x; i < a.G * D; i += split_threads<CW>()) {
         if (a.out_f32)
           a.out_f32[base + i] = 0.f;
         else
@@ -836,7 +888,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     float* thr = reinterpret_cast<float*>(smem + L::kThrOffset);
     int* count = reinterpret_cast<int*>(smem + L::kCountOffset);
     bool ok = true;
-    if (warp == kConsumerWarps) {
+    if (warp == CW) {
       // Producer: one TMA box of kScanTilesPerStage blocks of codes per stage.
       const uint64_t policy = policy_evict_first();
       for (int j = 0; j < n_scan; ++j) {
@@ -856,7 +908,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             raise_device_error(2u);
       }
     } else {
-      ok = sparse_scan_consumer<D, NB, STAGES, L::kStageBytes>(a, smem_base, bar_full, bar_empty,
+      ok = sparse_scan_consumer<D, NB, STAGES, L::kStageBytes, CW>(a, smem_base, bar_full, bar_empty,
                                                              bmax, warp, lane, b, h0, start, end,
                                                              n_tiles, n_scan);
     }
@@ -895,7 +947,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     it_base = n_scan;
   }
 
-  if (warp == kConsumerWarps) {
+  if (warp == CW) {
     // ------------------------------------------------------------- producer
     // Every lane waits (the decision is made warp-uniform); lane 0 issues.
     const uint64_t policy = policy_evict_first();
@@ -975,7 +1027,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
   } else {
     // ------------------------------------------------------------- consumers
-    split_consumers<D, NB, MODE, STAGES, FP8, SPARSE>(a, smem, smem_base, bar_full, bar_empty,
+    split_consumers<D, NB, MODE, STAGES, FP8, SPARSE, CW>(a, smem, smem_base, bar_full, bar_empty,
                                                       cta_error, warp, lane, b, h0, split,
                                                       start, end, n_work, n_parts, list,
                                                       it_base);
@@ -990,10 +1042,11 @@ __global__ void __launch_bounds__(128) fd_combine_kernel(const SplitArgs a, int 
   // one depends on, does not write them, and this grid launches only after
   // every split CTA passed its own wait, i.e. after all earlier writes to
   // them completed.  Read through L2 (coherent), not L1.
-  int n = 0;
+  int n_parts = 0;
   if (row < B * a.Hq) {
-    n = a.seqlens ? __ldcg(a.seqlens + row / a.Hq) : a.max_len;
+    int n = a.seqlens ? __ldcg(a.seqlens + row / a.Hq) : a.max_len;
     n = n < 0 ? 0 : (n > a.max_len ? a.max_len : n);
+    n_parts = split_parts(a, n);
   }
   grid_dependency_wait();     // partials come from the split kernel
   // The next call's split kernel may now start its prologue, which pulls its
@@ -1003,7 +1056,6 @@ __global__ void __launch_bounds__(128) fd_combine_kernel(const SplitArgs a, int 
   // be evicted and read twice at 16K tokens.)
   grid_dependents_launch();
   if (row >= B * a.Hq) return;
-  const int n_parts = min((n + a.chunk - 1) / a.chunk, a.n_splits);
   if (n_parts <= 1) return;
   combine_row<D>(a.part_o + static_cast<size_t>(row) * a.n_splits * D,
                  a.part_lse + static_cast<size_t>(row) * a.n_splits, n_parts, D, 1,
@@ -1012,19 +1064,22 @@ __global__ void __launch_bounds__(128) fd_combine_kernel(const SplitArgs a, int 
                  a.lse ? a.lse + row : nullptr, lane);
 }
 
-// Merge of R partial results laid out [R][rows][D] (fp32) and [R][rows]
-// (lse): one warp per row, partial r at stride rows * D.
+// Merge of R partial results: partial r of row i is the D floats at
+// part_o + r * o_stride + i * D and the lse at part_lse[r * l_stride + i]
+// ([R][rows][D] and [R][rows] when the strides are rows * D and rows; one
+// packed buffer per part when both strides are the part's size).  One warp
+// per row.
 template <int D>
 __global__ void __launch_bounds__(128) fd_merge_kernel(const float* part_o, const float* part_lse,
-                                                       int R, int rows, __nv_bfloat16* out,
+                                                       int R, int rows, size_t o_stride,
+                                                       size_t l_stride, __nv_bfloat16* out,
                                                        float* lse) {
   grid_dependency_wait();
   grid_dependents_launch();
   const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
-  combine_row<D>(part_o + static_cast<size_t>(row) * D, part_lse + row, R,
-                 static_cast<size_t>(rows) * D, static_cast<size_t>(rows),
+  combine_row<D>(part_o + static_cast<size_t>(row) * D, part_lse + row, R, o_stride, l_stride,
                  out + static_cast<size_t>(row) * D, nullptr, lse ? lse + row : nullptr, lane);
 }
 

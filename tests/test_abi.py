@@ -47,10 +47,25 @@ def test_split_chunk(L, S, chunk):
     assert chunk % 64 == 0
 
 
+@pytest.mark.parametrize("L,S,chunk,s_eff", [
+    (16384, 18, 960, 18),    # 256 tiles: 14 or 15 per split
+    (1000, 3, 384, 3),       # 16 tiles: 5, 5, 6
+    (1000, 7, 192, 7),       # 16 tiles: 2 or 3 per split
+    (65, 2, 64, 2), (10, 16, 64, 1), (0, 4, 64, 1), (64 * 1024 + 1, 1024, 128, 1024),
+])
+def test_split_cut_is_balanced(L, S, chunk, s_eff):
+    """T = ceil(L / 64) tiles into min(S, T) splits: the largest split has
+    ceil(T / S_eff) tiles and no split is empty."""
+    assert fd.fd_split_chunk(L, S) == chunk
+    assert fd.fd_effective_splits(L, S) == s_eff
+
+
 def test_split_chunk_invalid():
     assert fd.fd_split_chunk(-1, 2) == fd.FD_ERR_INVALID_ARGUMENT
     assert fd.fd_split_chunk(100, 0) == fd.FD_ERR_INVALID_ARGUMENT
     assert fd.fd_split_chunk(100, 1025) == fd.FD_ERR_INVALID_ARGUMENT
+    assert fd.fd_effective_splits(-1, 2) == fd.FD_ERR_INVALID_ARGUMENT
+    assert fd.fd_effective_splits(100, 0) == fd.FD_ERR_INVALID_ARGUMENT
 
 
 def test_workspace_bytes():
@@ -82,8 +97,8 @@ def test_plan_short_history_does_not_split():
 def test_plan_long_history_fills_the_device():
     for L in (16384, 32768, 65536, 262144):
         S = fd.fd_plan_sm(B200_SMS, 1, 64, 8, 128, L, 0)
-        chunk = fd.fd_split_chunk(L, S)
-        s_eff = -(-L // chunk)
+        s_eff = fd.fd_effective_splits(L, S)
+        assert s_eff == min(S, -(-L // 64))
         ctas = 8 * s_eff
         assert ctas >= 0.75 * B200_SMS, (L, S, ctas)
         assert ctas <= 4 * 2 * B200_SMS, (L, S, ctas)
@@ -411,3 +426,15 @@ def test_header_is_plain_c_and_links(tmp_path):
                     "-I", os.path.join(ROOT, "include"), str(src), "-L", libdir, "-lfd",
                     f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
     assert subprocess.run([str(exe)]).returncode == 0
+
+
+def test_static_workspace_size_matches_header():
+    """The binding's FD_STATIC_WORKSPACE_BYTES is the header's #define, as the
+    C preprocessor evaluates it."""
+    import re
+    with open(os.path.join(ROOT, "include", "fd.h")) as f:
+        m = re.search(r"#define\s+FD_STATIC_WORKSPACE_BYTES\s+(.+)", f.read())
+    assert m, "FD_STATIC_WORKSPACE_BYTES is not defined in fd.h"
+    expr = m.group(1).strip()
+    value = eval(re.sub(r"(\d+)[uUlL]+", r"\1", expr), {"__builtins__": {}})
+    assert value == fd.FD_STATIC_WORKSPACE_BYTES

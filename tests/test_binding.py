@@ -76,7 +76,41 @@ def test_sharded_helpers_check_their_tensors():
         sharded.local_partial(q, k, v, torch.zeros(2, dtype=torch.int64))
     with pytest.raises(ValueError, match="float32"):
         sharded.combine(torch.zeros(2, 2, 16, 128, dtype=torch.float64), torch.zeros(2, 2, 16))
+    P = sharded.packed_floats(2, 16, 128)
+    with pytest.raises(ValueError, match="float32"):
+        sharded.combine_packed(torch.zeros(2, P, dtype=torch.float64), 2, 16, 128)
+    with pytest.raises(ValueError, match="parts shape"):
+        sharded.combine_packed(torch.zeros(2, P - 64), 2, 16, 128)
+    with pytest.raises(ValueError, match="contiguous"):
+        sharded.combine_packed(torch.zeros(P, 2).t(), 2, 16, 128)
+    with pytest.raises(ValueError, match="CUDA device"):
+        sharded.combine_packed(torch.zeros(2, P), 2, 16, 128)
     with pytest.raises(ValueError, match="lse_all shape"):
         sharded.combine(torch.zeros(2, 2, 16, 128), torch.zeros(2, 16))
     with pytest.raises(ValueError, match="CUDA device"):
         sharded.combine(torch.zeros(2, 2, 16, 128), torch.zeros(2, 2, 16))
+
+
+def test_static_workspace_wrapper_checks_its_tensors():
+    """fd_decode_static_workspace takes the problem struct and raw tensors; a
+    strided or padded cache, or a problem that does not describe the tensors,
+    is rejected before the C call (which sees only addresses)."""
+    q, k, v = args()
+    prob = fd.make_problem(2, 16, 2, 128, 256)
+    out = torch.zeros(2, 16, 128, dtype=torch.bfloat16)
+    lse = torch.zeros(2, 16)
+
+    def call(*a, prob=prob):
+        with pytest.raises(ValueError) as e:
+            fd.fd_decode_static_workspace(prob, *a, None, None, 0.125, 4, out, lse)
+        return str(e.value)
+
+    kt = torch.zeros(2, 256, 2, 128, dtype=torch.bfloat16).transpose(1, 2)
+    assert "k_cache must be contiguous" in call(q, kt, kt)
+    wide = torch.zeros(2, 2, 512, 128, dtype=torch.bfloat16)[:, :, :256]
+    assert "k_cache must be contiguous" in call(q, wide, wide)
+    padded = torch.zeros(2, 2, 512, 128, dtype=torch.bfloat16)
+    assert "max_len" in call(q, padded, padded)
+    assert "Hkv" in call(q, k, v, prob=fd.make_problem(2, 16, 4, 128, 256))
+    assert "(B, Hq, D)" in call(q, k, v, prob=fd.make_problem(2, 32, 2, 128, 256))
+    assert "CUDA device" in call(q, k, v)

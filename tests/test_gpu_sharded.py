@@ -1,8 +1,9 @@
 """Sequence-parallel decode on one GPU: the history is cut into R contiguous
-slices; fd_decode_partial runs on each slice, the R results are stacked (as
-an all-gather would lay them out) and fd_combine merges them.  The slices run
-one after another on one device, so nothing waits on anything else; with one
-GPU per rank the same partials would be all-gathered instead of stacked."""
+slices; fd_decode_partial runs on each slice, the R results are laid out as an
+all-gather would lay them out (stacked, or packed buffers end to end) and
+fd_combine / fd_combine_strided merge them.  The slices run one after another
+on one device, so nothing waits on anything else; with one GPU per rank the
+same partials would be all-gathered instead."""
 import numpy as np
 import pytest
 
@@ -103,3 +104,36 @@ def test_paged_slices_merge(cuda_device):
     torch.cuda.synchronize()
     ref, rl = reference(w)
     assert_close(host_bf16(out), lse.cpu().numpy().astype(np.float64), ref, rl, "paged slices")
+
+
+@pytest.mark.parametrize("R", [1, 2, 3])
+def test_packed_parts_merge_where_they_lie(cuda_device, R):
+    """The sequence-parallel exchange format: each slice's partial is written
+    by sharded.local_partial straight into its row of one [R, P] buffer (the
+    layout an all-gather of the packed buffers produces), and
+    fd_combine_strided merges the rows in place.  The result equals the
+    merge of the same partials stacked into [R, B, Hq, D] / [R, B, Hq] bit
+    for bit, and the fp64 oracle over the whole history."""
+    import torch
+    B, Hq, Hkv, D, L = 2, 32, 8, 128, 4096
+    w = wl.make_problem(B, Hq, Hkv, D, L, seed=96 + R, seqlens=[4096, 1500])
+    P = sharded.packed_floats(B, Hq, D)
+    parts = torch.full((R, P), float("nan"), dtype=torch.float32, device="cuda")
+    for r in range(R):
+        lo, hi = sharded.shard_bounds(L, R, r)
+        d = OnDevice(slice_workload(w, lo, hi))
+        sharded.local_partial(d.q, d.k, d.v, d.seqlens, packed=parts[r])
+    out, lse = sharded.combine_packed(parts, B, Hq, D)
+    o_all, l_all = sharded.unpack(parts, B, Hq, D)
+    out2, lse2 = sharded.combine(o_all.contiguous(), l_all.contiguous())
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2) and torch.equal(lse, lse2)
+    ref, rl = reference(w)
+    assert_close(host_bf16(out), lse.cpu().numpy().astype(np.float64), ref, rl, f"packed R={R}")
+    # strides that would put a part's rows out of line are refused
+    base = parts.data_ptr()
+    assert fd.fd_combine_strided(R, B, Hq, D, base, P - 2, base + 4 * B * Hq * D, P, out,
+                                 lse) == fd.FD_ERR_INVALID_ARGUMENT
+    assert fd.fd_combine_strided(R, B, Hq, D, base, B * Hq * D - 4, base, P, out,
+                                 lse) == fd.FD_ERR_INVALID_ARGUMENT
+    assert fd.fd_check_device_error() == fd.FD_OK

@@ -1,9 +1,14 @@
 """GPU parity of the sparse decode: fd_quantize_keys and fd_decode_sparse
 (through the C ABI) against the oracle in oracle/sparse.py.
 
-The block selection is exact integer and fp32 arithmetic on both sides, so the
-kept-block masks must match bit for bit. The outputs are compared with the
-fp64 attention over the kept blocks at the usual tolerances."""
+The kept-block masks are checked twice:
+- against the scan's definition in fp64 (select_blocks_exact), on every block
+  whose decision lies outside the fp32 rounding margin; the blocks inside it
+  are counted and reported;
+- bit for bit against the oracle's fp32 form of the rule, which takes the
+  library's product order.
+The outputs are compared with the fp64 attention over the kept blocks at the
+usual tolerances."""
 import numpy as np
 import pytest
 
@@ -63,6 +68,22 @@ def check_kept(w, kept_gpu, kept_ref):
         assert np.all(kept_gpu[b, :, nb:] == 255)     # past the length: not written
 
 
+def check_kept_exact(w, kept_gpu, k8, sk, delta, S, what=""):
+    """The GPU's kept blocks equal the fp64 definition's on every block whose
+    decision no fp32 rounding can flip; returns (inside the margin, total)."""
+    kept64, certain = sparse.select_blocks_exact(w.q, k8, sk, w.scale, delta, S, w.seqlens)
+    inside = total = 0
+    for b in range(w.B):
+        nb = -(-int(w.lengths()[b]) // 64)
+        c = certain[b, :, :nb]
+        got = kept_gpu[b, :, :nb].astype(bool)
+        assert np.array_equal(got[c], kept64[b, :, :nb][c]), f"{what} sequence {b}"
+        inside += int((~c).sum())
+        total += c.size
+    print(f"{what}: {inside} of {total} block decisions inside the fp32 rounding margin")
+    return inside, total
+
+
 @pytest.mark.parametrize("D", [64, 128])
 def test_quantize_keys_bit_exact(D):
     w = wl.make_problem(3, 8, 4, D, 1000, seed=400 + D, seqlens=[1000, 130, 0], nan_pad=True)
@@ -83,13 +104,18 @@ def test_sparse_decode_matches_oracle(G):
     d = OnDevice(w)
     k8, sk = quantize_on_gpu(d)
     ref8, refs = sparse.quantize_keys(w.k, w.seqlens)
+    inside = total = 0
     for S in (1, 3, 7):
         for delta in (0.0, 2.0, 6.0):
             got, gl, kept = run_sparse(d, k8, sk, delta, S)
             ref, rl, kref = sparse.sparse_decode(w.q, w.k, w.v, w.scale, delta, S, w.seqlens,
                                                  k8=ref8, sk=refs)
+            i, t = check_kept_exact(w, kept, ref8, refs, delta, S, f"G={G} S={S} delta={delta}")
+            inside += i
+            total += t
             check_kept(w, kept, kref)
             assert_close(got, gl, ref, rl, f"sparse G={G} S={S} delta={delta}")
+    assert inside <= max(2, total // 1000)
 
 
 def test_infinite_delta_is_dense_decode_bit_for_bit():
@@ -141,6 +167,8 @@ def check_peaked(w, delta, share_lo, share_hi):
     ref8 = np.concatenate([p[0] for p in parts], axis=1)
     refs = np.concatenate([p[1] for p in parts], axis=1)
     assert np.array_equal(k8.cpu().numpy(), ref8) and np.array_equal(sk.cpu().numpy(), refs)
+    inside, total = check_kept_exact(w, kept, ref8, refs, delta, S, f"{w.name} S={S}")
+    assert inside <= max(2, total // 1000)
     kref = sparse.select_blocks(w.q, ref8, refs, w.scale, delta, S)
     check_kept(w, kept, kref)
     ref, rl, _ = sparse.sparse_decode(w.q, w.k, w.v, w.scale, delta, S, groups=[(0, 0), (0, 5)],

@@ -72,7 +72,8 @@ def test_single_rank_needs_no_process_group():
 def _sharded_worker(rank, world, port, q_out):
     """One rank of a sequence-parallel decode on CPU: the partial over this
     rank's slice comes from the fp64 oracle, the merge is the log-sum-exp
-    formula written out in numpy; the gather is the package's own code."""
+    formula written out in numpy; the packing, the one all-gather and the
+    unpacking of the gathered parts are the package's own code."""
     sys.path.insert(0, ROOT)
     import numpy as np
     import torch
@@ -92,9 +93,16 @@ def _sharded_worker(rank, world, port, q_out):
 
         def partial(q, k, v, seqlens):
             o, lse = oracle.decode(q, k, v, w.scale, seqlens=seqlens, nthreads=1)
-            return torch.from_numpy(o), torch.from_numpy(lse)
+            buf = torch.full((sharded.packed_floats(w.B, w.Hq, w.D),), float("nan"),
+                             dtype=torch.float64)
+            po, pl = sharded.unpack(buf, w.B, w.Hq, w.D)
+            po.copy_(torch.from_numpy(o))
+            pl.copy_(torch.from_numpy(lse))
+            return buf
 
-        def merge(o_all, lse_all):
+        def merge(parts, B, Hq, D):
+            assert tuple(parts.shape) == (world, sharded.packed_floats(B, Hq, D))
+            o_all, lse_all = sharded.unpack(parts, B, Hq, D)
             o_all, lse_all = o_all.numpy(), lse_all.numpy()
             m = lse_all.max(axis=0)
             with np.errstate(invalid="ignore"):
@@ -129,6 +137,26 @@ def test_sequence_sharded_decode_orchestration(world):
     res = [q.get(timeout=10) for _ in range(world)]
     for rank, err, empty_ok, lse_err in res:
         assert err < 1e-12 and lse_err < 1e-12 and empty_ok, (rank, err, lse_err)
+
+
+def test_packed_partial_layout():
+    """One part is O rows then lse values, padded to 64 floats; unpack gives
+    views of one part or of R gathered parts."""
+    sys.path.insert(0, ROOT)
+    import torch
+
+    from split_kv_decode_attn_b200 import sharded
+    for B, Hq, D in ((1, 1, 64), (3, 8, 64), (1, 64, 128), (2, 6, 128)):
+        P = sharded.packed_floats(B, Hq, D)
+        rows = B * Hq
+        assert P % 64 == 0 and rows * (D + 1) <= P < rows * (D + 1) + 64
+        parts = torch.arange(3 * P, dtype=torch.float32).reshape(3, P)
+        o, lse = sharded.unpack(parts, B, Hq, D)
+        assert o.shape == (3, B, Hq, D) and lse.shape == (3, B, Hq)
+        assert o[2, B - 1, Hq - 1, D - 1] == 2 * P + rows * D - 1
+        assert lse[1, 0, 0] == P + rows * D and lse[1, B - 1, Hq - 1] == P + rows * D + rows - 1
+        o1, l1 = sharded.unpack(parts[1], B, Hq, D)
+        assert o1.data_ptr() == parts[1].data_ptr() and torch.equal(l1, lse[1])
 
 
 def test_shard_bounds_cover_the_history_once():

@@ -27,8 +27,25 @@ MUTANTS = {
     "first head of the group only": ("(bmax[s0:s1] >= thr[None, :]).any(axis=1)",
                                      "(bmax[s0:s1] >= thr[None, :])[:, 0]"),
     "delta added, not subtracted": ("thr = (M - delta32)", "thr = (M + delta32)"),
-    "chunk not rounded to the tile": ("c = -(-per // BLOCK) * BLOCK", "c = per"),
+    "equal chunks of ceil(T / S) blocks": (
+        "return [(s * T // S, (s + 1) * T // S) for s in range(S)]",
+        "return [(s * -(-T // S), min(T, (s + 1) * -(-T // S))) for s in range(S)]"),
     "kept blocks ignored in attention": ("tok = tok[kept[b, h, tok // BLOCK]]", "pass"),
+    # the fp64 form of the selection (select_blocks_exact / block_maxima_exact)
+    "exact: query scale dropped": (
+        "factor = sc * sq[b, h * G:(h + 1) * G].astype(np.float64)",
+        "factor = sc * np.ones(G)"),
+    "exact: first block's scale for every block": (
+        "logit = factor[None, :] * sk[b, h, blk].astype(np.float64)[:, None] * dots",
+        "logit = factor[None, :] * float(sk[b, h, 0]) * dots"),
+    "exact: whole history as one split": (
+        "        for s0, s1 in split_blocks(L, num_splits):\n            if s0 >= nb:\n"
+        "                break\n            s1 = min(nb, s1)\n            part = bm[s0:s1]",
+        "        for s0, s1 in [(0, nb)]:\n            if s0 >= nb:\n"
+        "                break\n            s1 = min(nb, s1)\n            part = bm[s0:s1]"),
+    "exact: certainty against the split maximum": (
+        "other = np.where(np.arange(n_blk)[:, None] == top[None, :], second[None, :],",
+        "other = np.where(np.arange(n_blk)[:, None] == top[None, :], m1[None, :],"),
 }
 
 

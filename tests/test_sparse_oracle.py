@@ -29,6 +29,15 @@ sparse = _sparse_oracle()
 pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
 
 
+def exact_kept(q, k8, sk, scale, delta, num_splits, seqlens=None):
+    return sparse.select_blocks_exact(q, k8, sk, scale, delta, num_splits, seqlens)[0]
+
+
+# The rule's pins run on both forms of the selection: the fp32 product order
+# the library uses, and the fp64 definition.
+SELECTORS = {"fp32": lambda *a, **kw: sparse.select_blocks(*a, **kw), "fp64": exact_kept}
+
+
 def problem(B=3, Hq=8, Hkv=2, D=64, L=300, seed=1, lens=(300, 130, 1)):
     return wl.make_problem(B, Hq, Hkv, D, L, seed=seed, seqlens=list(lens), nan_pad=True)
 
@@ -106,6 +115,21 @@ def test_infinite_delta_keeps_everything_and_equals_dense_attention():
             assert kept[b, :, :nb].all() and not kept[b, :, nb:].any()
 
 
+@pytest.mark.parametrize("form", sorted(SELECTORS))
+def test_one_dominant_block_selects_alone(form):
+    """The selection alone, in both forms: a key aligned with every query
+    head of the group, far above the rest, is the only block kept at
+    delta = 0 with one split."""
+    w = problem(B=1, Hq=4, Hkv=1, D=128, L=1024, seed=5, lens=(1024,))
+    qf = f32(w.q[0]).astype(np.float64)
+    key = qf.sum(axis=0)
+    k = w.k.copy()
+    k[0, 0, 700] = wl.f64_to_bf16_bits(24.0 * key / np.linalg.norm(key))
+    k8, sk = sparse.quantize_keys(k)
+    kept = SELECTORS[form](w.q, k8, sk, w.scale, 0.0, 1)
+    assert kept[0, 0].tolist() == [i == 700 // 64 for i in range(16)]
+
+
 def test_one_dominant_block_is_all_that_a_zero_delta_keeps():
     """A key aligned with every query head of the group, far above the rest:
     with one split and delta = 0 only its block survives, and the output is
@@ -122,26 +146,29 @@ def test_one_dominant_block_is_all_that_a_zero_delta_keeps():
     assert np.abs(out[0] - v700).max() < 0.05
 
 
-def test_more_delta_keeps_more_and_each_split_keeps_its_best_block():
+@pytest.mark.parametrize("form", sorted(SELECTORS))
+def test_more_delta_keeps_more_and_each_split_keeps_its_best_block(form):
+    select = SELECTORS[form]
     w = wl.make_problem(2, 8, 2, 128, 2048, seed=9, seqlens=[2048, 1500])
     k8, sk = sparse.quantize_keys(w.k, w.seqlens)
     prev = None
     for delta in (0.0, 0.5, 1.0, 2.0, 4.0, np.inf):
-        kept = sparse.select_blocks(w.q, k8, sk, w.scale, delta, 4, w.seqlens)
+        kept = select(w.q, k8, sk, w.scale, delta, 4, w.seqlens)
         if prev is not None:
             assert np.all(kept >= prev)                    # monotone in delta
         prev = kept
-    kept0 = sparse.select_blocks(w.q, k8, sk, w.scale, 0.0, 4, w.seqlens)
-    chunk = sparse.chunk_for(2048, 4) // 64
+    kept0 = select(w.q, k8, sk, w.scale, 0.0, 4, w.seqlens)
     for b in range(2):
         nb = -(-int(w.seqlens[b]) // 64)
         for h in range(2):
-            for s0 in range(0, nb, chunk):
-                assert kept0[b, h, s0:min(nb, s0 + chunk)].any()
+            for s0, s1 in sparse.split_blocks(2048, 4):
+                if s0 < nb:
+                    assert kept0[b, h, s0:min(nb, s1)].any()
             assert not kept0[b, h, nb:].any()
 
 
-def test_kept_blocks_are_the_union_over_the_heads_of_a_group():
+@pytest.mark.parametrize("form", sorted(SELECTORS))
+def test_kept_blocks_are_the_union_over_the_heads_of_a_group(form):
     """Two query heads of one group, each with its own dominant key in a
     different block: with one split and delta = 0 exactly those two blocks
     survive, one chosen by each head (a rule that looked at one head only, or
@@ -153,18 +180,93 @@ def test_kept_blocks_are_the_union_over_the_heads_of_a_group():
         key = 24.0 * qf[g] / np.linalg.norm(qf[g])
         k[0, 0, pos] = wl.f64_to_bf16_bits(key)
     k8, sk = sparse.quantize_keys(k)
-    kept = sparse.select_blocks(w.q, k8, sk, w.scale, 0.0, 1)
+    kept = SELECTORS[form](w.q, k8, sk, w.scale, 0.0, 1)
     assert kept[0, 0].tolist() == [i in (130 // 64, 900 // 64) for i in range(16)]
     # each head alone keeps only its own block
     for g, pos in ((0, 130), (1, 900)):
-        one = sparse.select_blocks(w.q[:, g:g + 1], k8, sk, w.scale, 0.0, 1)
+        one = SELECTORS[form](w.q[:, g:g + 1], k8, sk, w.scale, 0.0, 1)
         assert one[0, 0].tolist() == [i == pos // 64 for i in range(16)]
 
 
-def test_split_chunks_follow_the_dense_chunking():
-    """ceil(max_len / S) rounded up to the 64-token tile, at least one tile."""
-    assert sparse.chunk_for(2048, 4) == 512
-    assert sparse.chunk_for(1000, 3) == 384     # ceil(1000 / 3) = 334 -> 384
-    assert sparse.chunk_for(65, 2) == 64        # 33 -> 64
-    assert sparse.chunk_for(10, 16) == 64
-    assert sparse.chunk_for(262144, 16) == 16384
+def test_split_blocks_follow_the_dense_cut():
+    """T = ceil(max_len / 64) blocks into min(S, T) splits of floor(s T / S)
+    boundaries: sizes differ by at most one block."""
+    assert sparse.split_blocks(2048, 4) == [(0, 8), (8, 16), (16, 24), (24, 32)]
+    assert sparse.split_blocks(1000, 3) == [(0, 5), (5, 10), (10, 16)]   # T = 16
+    assert sparse.split_blocks(65, 2) == [(0, 1), (1, 2)]
+    assert sparse.split_blocks(10, 16) == [(0, 1)]
+    assert sparse.split_blocks(0, 4) == [(0, 0)]
+    assert sparse.split_blocks(262144, 16) == [(256 * s, 256 * (s + 1)) for s in range(16)]
+    # 256 blocks in 18 splits: floor(8 * 256 / 18) = 113, floor(9 * 256 / 18) = 128
+    sizes = [b - a for a, b in sparse.split_blocks(16384, 18)]
+    assert sum(sizes) == 256 and set(sizes) == {14, 15}
+    assert [i for i, n in enumerate(sizes) if n == 15] == [4, 8, 13, 17]
+
+
+@pytest.mark.parametrize("form", sorted(SELECTORS))
+def test_top_delta_applies_per_split_of_the_balanced_cut(form):
+    """Block maxima that fall with the block index and delta = 0: each split
+    keeps exactly its first block, so the kept blocks are the splits' first
+    blocks, 0, 5 and 10 for 16 blocks in 3 splits (equal chunks of
+    ceil(16 / 3) = 6 blocks would keep 0, 6 and 12)."""
+    w = problem(B=1, Hq=1, Hkv=1, D=128, L=1024, seed=23, lens=(1024,))
+    qf = f32(w.q[0, 0]).astype(np.float64)
+    k = w.k.copy()
+    for blk in range(16):
+        key = (20.0 - blk) * np.sqrt(128.0) * qf / np.linalg.norm(qf)
+        k[0, 0, 64 * blk + 3] = wl.f64_to_bf16_bits(key)
+    k8, sk = sparse.quantize_keys(k)
+    select = SELECTORS[form]
+    kept = select(w.q, k8, sk, w.scale, 0.0, 3)
+    assert np.flatnonzero(kept[0, 0]).tolist() == [0, 5, 10]
+    kept = select(w.q, k8, sk, w.scale, 0.0, 16)
+    assert kept[0, 0].all()                       # one block per split
+    kept = select(w.q, k8, sk, w.scale, 0.0, 1)
+    assert np.flatnonzero(kept[0, 0]).tolist() == [0]
+
+
+def test_exact_block_maxima_by_brute_force():
+    """block_maxima_exact against the logits written out token by token with
+    Python integers and fractions-free fp64 products, on a tiny ragged case."""
+    w = problem(B=2, Hq=4, Hkv=2, D=64, L=150, seed=31, lens=(150, 70))
+    k8, sk = sparse.quantize_keys(w.k, w.seqlens)
+    q8, sq = sparse.quantize_query(w.q)
+    maxima = sparse.block_maxima_exact(w.q, k8, sk, w.scale, w.seqlens)
+    for b, n in enumerate((150, 70)):
+        for h in range(2):
+            bm = maxima[(b, h)]
+            assert bm.shape == (-(-n // 64), 2)
+            for blk in range(bm.shape[0]):
+                for g in range(2):
+                    best = -np.inf
+                    for j in range(blk * 64, min(n, blk * 64 + 64)):
+                        dot = sum(int(x) * int(y) for x, y in zip(q8[b, 2 * h + g], k8[b, h, j]))
+                        best = max(best, float(np.float32(w.scale)) * float(sq[b, 2 * h + g])
+                                   * float(sk[b, h, blk]) * dot)
+                    assert bm[blk, g] == pytest.approx(best, rel=1e-15, abs=0)
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
+def test_fp32_rule_agrees_with_the_exact_scan_outside_the_rounding_margin(G):
+    """The fp32 product order the library follows and the fp64 definition of
+    the scan keep the same blocks wherever the decision lies farther from its
+    threshold than fp32 rounding can move it (select_blocks_exact's
+    'certain'); the blocks inside that margin are counted and must be rare."""
+    lens = [0, 1, 65, 700, 2000, 3333]
+    w = wl.make_problem(len(lens), 2 * G, 2, 128, 3333, seed=410 + G, seqlens=lens,
+                        nan_pad=True)
+    k8, sk = sparse.quantize_keys(w.k, w.seqlens)
+    inside = total = 0
+    for S in (1, 3, 7):
+        for delta in (0.0, 2.0, 6.0):
+            kept32 = sparse.select_blocks(w.q, k8, sk, w.scale, delta, S, w.seqlens)
+            kept64, certain = sparse.select_blocks_exact(w.q, k8, sk, w.scale, delta, S,
+                                                         w.seqlens)
+            for b, n in enumerate(lens):
+                nb = -(-n // 64)
+                c = certain[b, :, :nb]
+                assert np.array_equal(kept32[b, :, :nb][c], kept64[b, :, :nb][c])
+                inside += int((~c).sum())
+                total += c.size
+    print(f"G={G}: {inside} of {total} block decisions inside the fp32 rounding margin")
+    assert inside <= max(2, total // 1000)

@@ -7,11 +7,12 @@ whose memory pool owns all device memory; a decode loop that must not block or
 fail on an allocation mid-step. This entry point takes the same inputs and
 outputs as fd_decode. Its scratch is the library's static device array
 (FD_STATIC_WORKSPACE_BYTES), so the caller allocates nothing. The test calls
-it twice in a row through the C ABI and checks each result against fd_decode
-with a caller-allocated workspace, using the same tolerances as the other
-parity tests. This file sorts last so that a run stopping at the first
-failure has already run every other test. It must also pass on its own, in
-a fresh process.
+it twice in a row through the C ABI. Each result must equal fd_decode's with a
+caller-allocated workspace bit for bit (same split count, same kernels, no
+atomics in the data path), and must match the fp64 oracle within the
+tolerances of the other parity tests. This file sorts last so that a run
+stopping at the first failure has already run every other test. It must also
+pass on its own, in a fresh process.
 """
 import numpy as np
 import pytest
@@ -19,7 +20,7 @@ import pytest
 import split_kv_decode_attn_b200 as fd
 from split_kv_decode_attn_b200 import workloads as wl
 
-from fdtest import LSE_TOL, OUT_TOL, OnDevice, host_bf16
+from fdtest import OnDevice, assert_close, host_bf16, reference
 
 pytestmark = pytest.mark.gpu
 
@@ -46,22 +47,18 @@ def test_static_workspace_matches_fd_decode(cuda_device, name):
     assert fd.fd_workspace_bytes(w.B, w.Hq, w.D, S) <= fd.FD_STATIC_WORKSPACE_BYTES
     ref_out, ref_lse, _ = d.run(S)  # fd_decode with a torch-allocated workspace
     torch.cuda.synchronize()
-    ref = host_bf16(ref_out)
-    rl = ref_lse.cpu().numpy().astype(np.float64)
-    for _ in range(2):
+    oracle_out, oracle_lse = reference(w)
+    for i in range(2):
         out = torch.full_like(ref_out, float("nan"))
         lse = torch.full_like(ref_lse, float("nan"))
         st = fd.fd_decode_static_workspace(d.problem(), d.q, d.k, d.v, d.seqlens, d.table,
                                            w.scale, S, out, lse, None)
         assert st == fd.FD_OK, fd.fd_status_string(st)
         torch.cuda.synchronize()
-        got = host_bf16(out)
-        gl = lse.cpu().numpy().astype(np.float64)
-        assert np.all(np.isfinite(got))
-        assert np.max(np.abs(got - ref)) <= OUT_TOL
-        empty = np.isneginf(rl)
-        assert np.all(np.isneginf(gl[empty]))
-        assert np.all(np.abs(gl[~empty] - rl[~empty]) <= LSE_TOL)
+        assert torch.equal(out, ref_out), f"call {i}: out differs from fd_decode's"
+        assert torch.equal(lse, ref_lse), f"call {i}: lse differs from fd_decode's"
+        assert_close(host_bf16(out), lse.cpu().numpy().astype(np.float64), oracle_out,
+                     oracle_lse, f"{name}, call {i}")
     assert fd.fd_check_device_error() == fd.FD_OK
 
 
