@@ -18,8 +18,6 @@
 namespace {
 
 constexpr int kMaxSplits = 1024;
-// Tiles a split CTA may prefetch into L2 before its inputs are released.
-constexpr int kPrefetchTiles = 4;
 constexpr int kMaxDevices = 64;
 
 // ---------------------------------------------------------------- planner
@@ -481,6 +479,27 @@ int pick_splits(int max_len, long long units, int slots, Model model) {
   return best;
 }
 
+// Tiles each split CTA of a contiguous cache pulls into L2 before it waits on
+// the previous grid, one TMA prefetch per tile (the prefetch overlaps the
+// previous call's combine and the launch between the calls).
+// bf16: a quarter of the split's tiles, at least 2, with the tiles of the
+// CTAs resident at once (one or two per SM) kept to 64 MB of the 126 MB L2.
+// Swept on B200 over 2..16 tiles for the CodeLlama-34B heads at 16K..256K
+// tokens and S = 16 (one CTA per SM) and 32 (two): the best depth grows with
+// the split (16K: 4, 32K: 8, 64K and longer: 12..16 at S = 16; 2, 4, 6..8,
+// 8 at S = 32), and a fixed 4 cost 0.9 us at 32K, 1.4 us at 64K and 2.8 us
+// at 128K.
+// fp8 (half the bytes per tile, twice the CTAs): half the split's tiles, at
+// most 4, which the same sweep kept.
+int prefetch_tiles(int max_tiles, long long grid, int sms, bool deep, bool fp8, int D) {
+  if (fp8) return std::min(4, std::max(1, max_tiles / 2));
+  const long long resident = std::min<long long>(grid, deep ? sms : 2LL * sms);
+  const long long tile_bytes = 2LL * fd::kTile * D * 2;      // K + V tiles, bf16
+  const long long cap = std::max<long long>(2, (64LL << 20) / (std::max(resident, 1LL) * tile_bytes));
+  return static_cast<int>(std::min<long long>(std::min<long long>(max_tiles, std::max(2, max_tiles / 4)),
+                                              std::min<long long>(cap, 16)));
+}
+
 // Inputs of the sparse decode (null for the dense one).
 struct SparseArgs {
   const int8_t* k8;
@@ -590,11 +609,6 @@ fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
   a.tile_r = chunks.tiles % n_splits;
   a.scale_log2 = scale * (fp8 ? p->k_scale : 1.f) * 1.4426950408889634074f;
   a.v_scale = fp8 ? p->v_scale : 1.f;
-  // L2 prefetch ahead of the wait on the previous grid (contiguous caches):
-  // half the split's tiles, at most kPrefetchTiles.  Swept on B200 over
-  // 0..12 tiles at 4K..64K tokens, bf16 and fp8, S = 16 and 32.
-  a.prefetch_tiles =
-      (paged || sp) ? 0 : std::min(kPrefetchTiles, std::max(1, chunks.max_tiles / 2));
   a.scale = scale;
   if (sp) {
     a.k8 = sp->k8;
@@ -606,7 +620,9 @@ fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
 
   int sms = 0;
   if (device_sms(dev, &sms) != FD_OK) return FD_ERR_CUDA;
-  const bool deep = static_cast<long long>(B) * Hkv * n_splits <= sms;
+  const long long grid = static_cast<long long>(B) * Hkv * n_splits;
+  const bool deep = grid <= sms;
+  a.prefetch_tiles = (paged || sp) ? 0 : prefetch_tiles(chunks.max_tiles, grid, sms, deep, fp8, D);
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   fd_status r;

@@ -97,6 +97,17 @@ __host__ __device__ constexpr uint32_t perm16(uint32_t s) {
   return ((s & 7) >> 1) * 4 + (s >> 3) * 2 + (s & 1);
 }
 
+// Row of a warp's 16-row slice of the tile that holds the fp8 path's local
+// token t: rows 8..15 swap in pairs (8 <-> 10, 9 <-> 11, 12 <-> 14,
+// 13 <-> 15).  The eight rows of every 8-lane ldmatrix phase then sit in
+// eight different 128-byte swizzle phases (row mod 8): for K the local tokens
+// perm16(0..7) = 0, 1, 4, 5, 8, 9, 12, 13 (and perm16(8..15)), for V the
+// local tokens 0..7 and 8..15.  Without the swap, rows r and r + 8 of one K
+// phase shared a phase: one extra shared-memory wavefront per phase.  The
+// attention sum does not depend on the order of its tokens, so only the
+// addresses and the masks (which use the row) see the swap.
+__host__ __device__ constexpr uint32_t rho16(uint32_t t) { return t ^ ((t >> 3) << 1); }
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -457,14 +468,15 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
   // 128-byte swizzle phase (row mod 8).  A tile is a stack of TMA boxes of
   // 2^log2_box_rows rows, each laid out [column half][row][128 bytes].
   //
-  // FP8: row r of the score MMA is token perm16(r), so that after the P
-  // transpose the k-slots 2t, 2t+1 and 2t+8, 2t+9 of the P.V MMA are tokens
-  // 4t, 4t+1 and 4t+2, 4t+3: the order in which the byte-transposing
-  // ldmatrix delivers V (see ldmatrix_x2_trans_b8).
+  // FP8: row r of the score MMA is local token perm16(r), so that after the
+  // P transpose the k-slots 2t, 2t+1 and 2t+8, 2t+9 of the P.V MMA are local
+  // tokens 4t, 4t+1 and 4t+2, 4t+3: the order in which the byte-transposing
+  // ldmatrix delivers V (see ldmatrix_x2_trans_b8).  Local token t sits in
+  // row rho16(t) of the warp's slice.
   const uint32_t r16 = ((lane >> 3) & 1) * 8 + (lane & 7);
-  const uint32_t rowK = wr * 16 + (FP8 ? perm16(r16) : r16);
-  const uint32_t rowV = wr * 16 + (FP8 ? (lane & 15) : (lane >> 4) * 8 + (lane & 7));
-  const uint32_t x7 = lane & 7;              // swizzle phase of rowV (and of rowK if not FP8)
+  const uint32_t rowK = wr * 16 + (FP8 ? rho16(perm16(r16)) : r16);
+  const uint32_t rowV = wr * 16 + (FP8 ? rho16(lane & 15) : (lane >> 4) * 8 + (lane & 7));
+  const uint32_t xv = rowV & 7;              // swizzle phases of the two rows
   const uint32_t xk = rowK & 7;
   const uint32_t lgr = a.log2_box_rows;
   const uint32_t half_bytes = 128u << lgr;                    // one column half of a box
@@ -472,8 +484,8 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
   const uint32_t offK = (rowK >> lgr) * box_bytes + (rowK & ((1u << lgr) - 1)) * 128;
   const uint32_t offV = (rowV >> lgr) * box_bytes + (rowV & ((1u << lgr) - 1)) * 128;
   // Token rows of the C fragment held by this lane.
-  const int r_lo = wr * 16 + (FP8 ? perm16(lane >> 2) : (lane >> 2));
-  const int r_hi = wr * 16 + (FP8 ? perm16((lane >> 2) + 8) : (lane >> 2) + 8);
+  const int r_lo = wr * 16 + (FP8 ? rho16(perm16(lane >> 2)) : (lane >> 2));
+  const int r_hi = wr * 16 + (FP8 ? rho16(perm16((lane >> 2) + 8)) : (lane >> 2) + 8);
   const float sl2 = a.scale_log2;
   bool failed = false;
 
@@ -526,7 +538,7 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
 #pragma unroll
       for (int ks = 0; ks < KSTEPS; ++ks) {
         const uint32_t chunk16 = ((ks & 3) << 1) + (lane >> 4);
-        const uint32_t addr = kbase + offK + (ks >> 2) * half_bytes + ((chunk16 ^ x7) << 4);
+        const uint32_t addr = kbase + offK + (ks >> 2) * half_bytes + ((chunk16 ^ xk) << 4);
         uint32_t af[4];
         ldmatrix_x4(addr, af[0], af[1], af[2], af[3]);
 #pragma unroll
@@ -601,10 +613,13 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
     // zeroed in registers so that 0 * NaN never reaches the accumulator.
     uint32_t vmask_lo = 0xffffffffu, vmask_hi = 0xffffffffu;
     if (partial) {
-      if constexpr (FP8) {  // bytes i of a register: token 4t + i
-        const int tk = wr * 16 + 4 * (lane & 3);
-        vmask_lo = (tk < tile_valid ? 0xffu : 0u) | (tk + 1 < tile_valid ? 0xff00u : 0u) |
-                   (tk + 2 < tile_valid ? 0xff0000u : 0u) | (tk + 3 < tile_valid ? 0xff000000u : 0u);
+      if constexpr (FP8) {  // byte i of a register: local token 4t + i, in row rho16(4t + i)
+        const int t4 = 4 * (lane & 3);
+        const int base = wr * 16;
+        vmask_lo = (base + static_cast<int>(rho16(t4)) < tile_valid ? 0xffu : 0u) |
+                   (base + static_cast<int>(rho16(t4 + 1)) < tile_valid ? 0xff00u : 0u) |
+                   (base + static_cast<int>(rho16(t4 + 2)) < tile_valid ? 0xff0000u : 0u) |
+                   (base + static_cast<int>(rho16(t4 + 3)) < tile_valid ? 0xff000000u : 0u);
       } else {
         const int tk = wr * 16 + 2 * (lane & 3);
         vmask_lo = (tk < tile_valid ? 0x0000ffffu : 0u) | (tk + 1 < tile_valid ? 0xffff0000u : 0u);
@@ -619,7 +634,7 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
 #pragma unroll
       for (int dp = 0; dp < DBLK / 2; ++dp) {
         const uint32_t chunk16 = 2 * dp + (lane >> 4);
-        const uint32_t addr = vbase + offV + ((chunk16 ^ x7) << 4);
+        const uint32_t addr = vbase + offV + ((chunk16 ^ xv) << 4);
         uint32_t r[4];
         ldmatrix_x2_trans_b8(addr, r[0], r[1], r[2], r[3]);
         if (partial) {
@@ -642,7 +657,7 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
 #pragma unroll
     for (int db = 0; db < DBLK; ++db) {
       const uint32_t chunk16 = ((db & 3) << 1) + ((lane >> 3) & 1);
-      const uint32_t addr = vbase + offV + (db >> 2) * half_bytes + ((chunk16 ^ x7) << 4);
+      const uint32_t addr = vbase + offV + (db >> 2) * half_bytes + ((chunk16 ^ xv) << 4);
       uint32_t vf[4];
       ldmatrix_x4_trans(addr, vf[0], vf[1], vf[2], vf[3]);
       if (partial) {
@@ -715,11 +730,14 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
   if (!live) return;
 
   // One pass with no further barrier.  Each thread merges the CW warp
-  // states for 8 head-dim entries of one head (4 at d0 and 4 at d0 + D/2, so
-  // that a warp's 16-byte reads and writes are contiguous) and computes that
-  // head's weights itself from a few broadcast reads.  (A separate per-head
+  // states for 4 * kParts head-dim entries of one head (4 at d0, and with
+  // four consumer warps 4 more at d0 + D/2, so that a warp's 16-byte reads
+  // and writes are contiguous) and computes that head's weights itself from a
+  // few broadcast reads.  Eight consumer warps take 4 entries each, so that
+  // all 256 threads share the merge of the G = 8 heads.  (A separate per-head
   // pass behind two more barriers took about 1.5 us per CTA.)
-  constexpr int kChunks = D / 8;  // chunks of 8 entries per head
+  constexpr int kParts = CW == kConsumerWarps ? 2 : 1;
+  constexpr int kChunks = D / (4 * kParts);  // chunks of 4 * kParts entries per head
   const bool direct = n_parts == 1;
   for (int c = threadIdx.x; c < a.G * kChunks; c += CW * 32) {
     const int g = c / kChunks;
@@ -753,7 +771,7 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
     for (int w = 0; w < CW; ++w) {
       const float* src = f + L::kRedAcc + (w * NCOL + g) * L::kAccStride + d0;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      for (int h = 0; h < kParts; ++h) {
         float4 v = *reinterpret_cast<const float4*>(src + h * (D / 2));
         if constexpr (MODE == kDup) {  // columns g + 4 hold the bf16 residuals
           const float4 r = *reinterpret_cast<const float4*>(src + 4 * L::kAccStride + h * (D / 2));
@@ -772,20 +790,20 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
     if (direct) {
       if (a.out_f32) {
         float* dst = a.out_f32 + row * D + d0;
-        *reinterpret_cast<float4*>(dst) = o[0];
-        *reinterpret_cast<float4*>(dst + D / 2) = o[1];
+#pragma unroll
+        for (int h = 0; h < kParts; ++h) *reinterpret_cast<float4*>(dst + h * (D / 2)) = o[h];
       } else {
         __nv_bfloat16* dst = a.out + row * D + d0;
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
+        for (int h = 0; h < kParts; ++h)
           *reinterpret_cast<uint2*>(dst + h * (D / 2)) =
               make_uint2(pack_bf16x2(o[h].x, o[h].y), pack_bf16x2(o[h].z, o[h].w));
       }
       if (d0 == 0 && a.lse) a.lse[row] = lse_s;
     } else {
       float* dst = a.part_o + (row * a.n_splits + split) * D + d0;
-      *reinterpret_cast<float4*>(dst) = o[0];
-      *reinterpret_cast<float4*>(dst + D / 2) = o[1];
+#pragma unroll
+      for (int h = 0; h < kParts; ++h) *reinterpret_cast<float4*>(dst + h * (D / 2)) = o[h];
       if (d0 == 0) a.part_lse[row * a.n_splits + split] = lse_s;
     }
   }
