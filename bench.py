@@ -15,6 +15,17 @@ Reported (one JSON line from rank 0):
   e2e          the same metric through the C ABI from pinned host buffers,
                host<->device copies inside the timed region
   cpu_baseline the fp64 oracle on this host's cores, on a bounded sample
+  samples      the same call timed again as >= 10 samples of >= 20 calls
+               (each long enough for the clock sampler to see it): median,
+               min and max microseconds per call, and the SM clocks read
+               inside those windows
+  kernels      the split and combine kernels' shares of the call, from the
+               committed ncu launch list, and the split kernel's own time and
+               bandwidth derived from them
+  workloads    the other benchmark shapes, each as the median of >= 10
+               samples: the tiny MHA case at 1, 2, 4 and 8 splits, the varlen
+               batch, the paged cache, the peaked 256K history and the fp8
+               cache at 64K
   sweep        the same call at cache lengths 512 .. 64K
   planner      host microseconds per fd_plan_problem call (outside the timed
                region)
@@ -79,6 +90,11 @@ def parse_args():
     ap.add_argument("--crossover-filter", default=None,
                     help="with --crossover: only the shapes whose tag contains this text")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other benchmark shapes (the workloads array)")
+    ap.add_argument("--samples", type=int, default=10,
+                    help="timing samples per shape beside the declared region (at least 10 "
+                         "are taken; 0 skips them, e.g. for a profiler run)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -137,16 +153,21 @@ def ncu_traffic(workload: str, num_splits: int):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms, each
+    sample with its time stamp, so that samples can be matched to timing
+    windows of the host clock."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, device_index: int):
         import torch
         self.proc = None
         self.path = None
+        self.rows = []
         try:
             uuid = str(torch.cuda.get_device_properties(device_index).uuid)
             gid = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
@@ -167,6 +188,30 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
+    @staticmethod
+    def _parse(line):
+        parts = [p.strip() for p in line.strip().split(",")]
+        if len(parts) < 10:
+            return None
+        try:
+            t = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            util = float(parts[4]) if parts[4].replace(".", "").isdigit() else 0.0
+            return {"t": t, "sm": float(parts[1]), "max": float(parts[2]),
+                    "power": float(parts[3]), "util": util,
+                    "reasons": [ClockSampler.REASONS[i] for i in range(4)
+                                if parts[6 + i].lower() == "active"]}
+        except ValueError:
+            return None
+
+    @staticmethod
+    def summary(rows):
+        if not rows:
+            return {"samples": 0}
+        loaded = [r["sm"] for r in rows if r["util"] > 0] or [r["sm"] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": sorted({x for r in rows for x in r["reasons"]}),
+                "samples": len(rows), "power_w_max": max(r["power"] for r in rows)}
+
     def stop(self):
         if self.proc is None:
             return None
@@ -176,23 +221,15 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        rows = []
         with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.strip().split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
+            self.rows = [r for r in map(self._parse, f) if r is not None]
         os.unlink(self.path)
-        if not rows:
-            return {"samples": 0}
-        sm = [float(r[0]) for r in rows]
-        mx = [float(r[1]) for r in rows]
-        util = [float(r[3]) if r[3].replace(".", "").isdigit() else 0.0 for r in rows]
-        loaded = [s for s, u in zip(sm, util) if u > 0] or sm
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx), "reasons": reasons,
-                "samples": len(rows), "power_w_max": max(float(r[2]) for r in rows)}
+        return self.summary(self.rows)
+
+    def within(self, windows):
+        """Summary of the samples taken inside the host-time windows [(t0, t1)]."""
+        inside = [r for r in self.rows if any(t0 <= r["t"] <= t1 for t0, t1 in windows)]
+        return self.summary(inside)
 
 
 # ------------------------------------------------------------- our arm
@@ -232,8 +269,7 @@ class Call:
         else:  # the planner over the whole problem, lengths included when known
             self.S = fd.fd_plan_problem(0, self.prob, w.seqlens)
         assert self.S >= 1, fd.fd_status_string(self.S)
-        chunk = fd.fd_split_chunk(w.max_len, self.S)
-        self.s_eff = max(1, -(-w.max_len // chunk)) if w.max_len else 1
+        self.s_eff = fd.fd_effective_splits(w.max_len, self.S)
         self.out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=device)
         self.lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=device)
         self.wbytes = fd.fd_workspace_bytes(w.B, w.Hq, w.D, self.S)
@@ -303,6 +339,116 @@ def timed(torch, fn, steps, warmup, barrier=None):
     if barrier:
         barrier()
     return e0.elapsed_time(e1)  # ms
+
+
+def sampled(torch, fn, samples, min_calls=20, min_window_s=0.25):
+    """`samples` timing samples of back-to-back calls, each of at least
+    `min_calls` calls and about `min_window_s` seconds (so that the 200 ms
+    clock sampler sees every window), each timed with CUDA events on the
+    launching stream with a device synchronisation on both sides.  Returns
+    (microseconds per call of each sample, host-time windows, calls per
+    sample)."""
+    est = timed(torch, fn, min_calls, 3) * 1e3 / min_calls
+    calls = max(min_calls, int(min_window_s * 1e6 / max(est, 1e-3)))
+    per, windows = [], []
+    for _ in range(max(samples, 1)):
+        t0 = time.time()
+        ms = timed(torch, fn, calls, 0)
+        windows.append((t0, time.time()))
+        per.append(ms * 1e3 / calls)
+    return per, windows, calls
+
+
+def sample_stats(per, calls, kv_bytes, peak):
+    """Median, min and max of per-call samples, with bandwidth at the median
+    against the measured copy peak and the 8 TB/s spec."""
+    med = statistics.median(per)
+    gbs = kv_bytes / med / 1e3
+    return {"us_per_call_median": round(med, 3), "us_per_call_min": round(min(per), 3),
+            "us_per_call_max": round(max(per), 3), "samples": len(per),
+            "calls_per_sample": calls, "GB/s": round(gbs, 1),
+            "frac_measured": round(gbs / peak, 4), "frac_spec": round(gbs / SPEC_HBM_GBS, 4)}
+
+
+def workload_config(w, S, s_eff, copies, l2, world):
+    """The `config` object of a bench line: the workload, the split count and
+    how L2 is kept from serving K/V.  The reference arm reports the same."""
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+            "max_len": w.max_len, "block_size": w.block_size, "num_splits": S,
+            "effective_splits": s_eff, "kv_bytes_per_call": w.kv_bytes(),
+            "l2": f"inputs rotate over {copies} cache copies "
+                  f"({copies * (w.k.nbytes + w.v.nbytes) / 1e6:.0f} MB, L2 {l2 / 1e6:.0f} MB)",
+            "parallelism": f"replicas{world}" if world > 1 else "single"}
+
+
+def ncu_launch_shares(workload: str, num_splits: int):
+    """Shares of the split and combine kernels in the committed ncu launch
+    list (back-to-back calls, L2 not flushed between kernels), if it was
+    taken on the current device code at the same split count; else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        if j.get("source_hash") != kernel_source_hash():
+            return None
+        e = j.get("launches", {}).get(workload)
+        if e is None or int(e["num_splits"]) != num_splits:
+            return None
+        return e
+    except Exception:
+        return None
+
+
+def kernel_times(shares, us_per_call, kv_bytes, peak):
+    """The split kernel's time inside the call, as its share of the launch
+    list times the measured time per call, and its own bandwidth."""
+    if not shares:
+        return None
+    split_us = shares["split_share"] * us_per_call
+    return {"source": "ncu launch list (profiles/), shares x measured us/call",
+            "split_share": shares["split_share"], "combine_share": shares["combine_share"],
+            "split_ncu_us": shares["split_us"], "combine_ncu_us": shares["combine_us"],
+            "split_us": round(split_us, 3), "split_GB/s": round(kv_bytes / split_us / 1e3, 1),
+            "split_frac_measured": round(kv_bytes / split_us / 1e3 / peak, 4),
+            "split_frac_spec": round(kv_bytes / split_us / 1e3 / SPEC_HBM_GBS, 4)}
+
+
+# The other benchmark shapes of the default line: (workload, cache length,
+# cache type, split counts; None = the planner's).
+OTHER_WORKLOADS = (
+    ("tiny", None, "bf16", (1, 2, 4, 8)),
+    ("varlen", None, "bf16", (None,)),
+    ("paged", None, "bf16", (None,)),
+    ("peaked", None, "bf16", (None,)),
+    ("codellama34b", 65536, "fp8", (None,)),
+)
+
+
+def other_workloads(torch, fd, device, n_samples):
+    """Every other benchmark shape, each as the median of n_samples samples
+    (plus the device time from CUDA-graph replays), with its split count,
+    cache copies and the host-time windows of its samples (the caller turns
+    them into the SM clocks seen inside them once the sampler has stopped)."""
+    peak, _ = measured_peak()
+    rows = []
+    for name, L, kvd, splits in OTHER_WORKLOADS:
+        w = make_workload(name, L, 0, kv_dtype=kvd)
+        copies, l2 = copies_for(torch, w.k.nbytes + w.v.nbytes, device)
+        for S in splits:
+            call = Call(torch, fd, w, device, S, copies)
+            per, windows, calls = sampled(torch, call, n_samples)
+            g_us = timed_graph(torch, call, copies, max(1, 20 * calls // copies // 10))
+            row = {"workload": w.name, "kv": kvd, "num_splits": call.S,
+                   "effective_splits": call.s_eff, "kv_bytes_per_call": w.kv_bytes(),
+                   "copies": copies}
+            row.update(sample_stats(per, calls, w.kv_bytes(), peak))
+            row["graph_us_per_call"] = round(g_us, 3)
+            row["windows"] = windows     # replaced by the clocks seen inside them
+            rows.append(row)
+            del call
+        del w
+        torch.cuda.empty_cache()
+    return rows
 
 
 def timed_graph(torch, call, copies, reps, warmup=3):
@@ -458,7 +604,17 @@ def run_fd(args):
     sampler = ClockSampler(device.index)
     sampler.start()
     ms = timed(torch, call, args.steps, args.warmup, barrier)
+    # Beside the declared region: the same call as >= 10 samples long enough
+    # for the clock sampler (rank-local; reported by rank 0).
+    n_samples = max(args.samples, 10) if args.samples > 0 else 0
+    per, windows, calls = sampled(torch, call, n_samples) if n_samples else (None, None, None)
+    workloads = None
+    if n_samples and not args.no_workloads and rank == 0 and world == 1 \
+            and args.workload == "codellama34b" and args.kv_dtype == "bf16" and args.layout == "HND":
+        workloads = other_workloads(torch, fd, device, n_samples)
     clocks = sampler.stop()
+    for row in workloads or ():
+        row["clocks"] = sampler.within(row.pop("windows"))
     assert fd.fd_check_device_error() == 0
 
     ms = max_over_ranks(torch, ms, world, device)
@@ -473,12 +629,7 @@ def run_fd(args):
         "us_per_call": round(per_call_s * 1e6, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if w.kv_dtype == "bf16" else "e4m3 cache, f16 mma",
         "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
-                   "max_len": w.max_len, "block_size": w.block_size, "num_splits": call.S,
-                   "effective_splits": call.s_eff, "kv_bytes_per_call": kvb,
-                   "l2": f"inputs rotate over {copies} cache copies "
-                         f"({copies * (w.k.nbytes + w.v.nbytes) / 1e6:.0f} MB, L2 {l2 / 1e6:.0f} MB)",
-                   "parallelism": f"replicas{world}" if world > 1 else "single"},
+        "config": workload_config(w, call.S, call.s_eff, copies, l2, world),
         # achieved: algorithmic bytes over the whole call's event-timed duration
         # (the split kernel, the dominant one, plus the combine), so it is a
         # lower bound for the split kernel alone; traffic: the split kernel's
@@ -493,12 +644,21 @@ def run_fd(args):
         "clocks": clocks,
         "planner": planner_cost(fd, call.prob, w.seqlens),
     }
+    if n_samples:
+        stats = sample_stats(per, calls, kvb, peak)
+        stats["clocks"] = sampler.within(windows)
+        result["samples"] = stats
+        result["kernels"] = kernel_times(ncu_launch_shares(w.name, call.S),
+                                         stats["us_per_call_median"], kvb, peak)
+    if workloads is not None:
+        result["workloads"] = workloads
 
     if not args.no_e2e:
         result["e2e"] = e2e(torch, fd, call, w, device, min(args.steps, 30), 3, barrier, world)
 
-    if not args.no_sweep and args.workload == "codellama34b" and rank == 0 and world == 1:
-        result["sweep"] = sweep(torch, fd, device)
+    if not args.no_sweep and n_samples and args.workload == "codellama34b" and rank == 0 \
+            and world == 1:
+        result["sweep"] = sweep(torch, fd, device, n_samples)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
@@ -540,7 +700,7 @@ def e2e(torch, fd, call, w, device, steps, warmup, barrier, world):
             "d2h_bytes_per_step": d2h, "steps": steps}
 
 
-def sweep(torch, fd, device):
+def sweep(torch, fd, device, n_samples=10):
     from split_kv_decode_attn_b200 import workloads as wl
     peak, _ = measured_peak()
     rows = []
@@ -548,18 +708,14 @@ def sweep(torch, fd, device):
         w = wl.config(2, L=L)
         copies, _ = copies_for(torch, w.k.nbytes + w.v.nbytes, device)
         call = Call(torch, fd, w, device, None, copies)
-        steps = max(200, min(20000, int(0.3e9 / max(w.kv_bytes(), 1) * 100)))
-        ms = timed(torch, call, steps, 50)
-        per = ms / 1e3 / steps
-        gbs = w.kv_bytes() / per / 1e9
-        g_us = timed_graph(torch, call, copies, max(1, steps // copies))
+        per, _, calls = sampled(torch, call, n_samples)
+        g_us = timed_graph(torch, call, copies, max(1, 2 * calls // copies))
         g_gbs = w.kv_bytes() / (g_us * 1e-6) / 1e9
-        rows.append({"L": L, "num_splits": call.S, "effective_splits": call.s_eff,
-                     "us_per_call": round(per * 1e6, 3), "GB/s": round(gbs, 1),
-                     "frac_measured": round(gbs / peak, 4), "frac_spec": round(gbs / SPEC_HBM_GBS, 4),
-                     "graph_us_per_call": round(g_us, 3), "graph_GB/s": round(g_gbs, 1),
-                     "graph_frac_measured": round(g_gbs / peak, 4),
-                     "copies": copies, "steps": steps})
+        row = {"L": L, "num_splits": call.S, "effective_splits": call.s_eff, "copies": copies}
+        row.update(sample_stats(per, calls, w.kv_bytes(), peak))
+        row.update({"graph_us_per_call": round(g_us, 3), "graph_GB/s": round(g_gbs, 1),
+                    "graph_frac_measured": round(g_gbs / peak, 4)})
+        rows.append(row)
         del call
         torch.cuda.empty_cache()
     return rows
@@ -659,8 +815,9 @@ def run_sparse(args):
 def run_sharded(args):
     """Sequence-parallel decode of the CodeLlama-34B-shaped workload: rank r
     holds tokens [r*L/N, (r+1)*L/N) of every KV head.  A step is the local
-    partial (fd_decode_partial), the all-gather of the partial results and
-    their merge (fd_combine).  value = the whole history's K+V bytes over the
+    partial (fd_decode_partial) written into one packed buffer, one
+    all-gather of the packed buffers and their merge where they lie
+    (fd_combine_strided).  value = the whole history's K+V bytes over the
     slowest rank's time (strong scaling)."""
     import numpy as np
     import torch
@@ -695,10 +852,15 @@ def run_sharded(args):
     S = args.splits or fd.fd_plan(B, Hq, Hkv, D, hi - lo, 0)
     nbytes = fd.fd_workspace_bytes(B, Hq, D, S)
     ws = torch.empty(max(nbytes, 4) // 4, dtype=torch.float32, device=device)
-    o = torch.empty((B, Hq, D), dtype=torch.float32, device=device)
-    lse = torch.empty((B, Hq), dtype=torch.float32, device=device)
-    o_all = torch.empty((world, B, Hq, D), dtype=torch.float32, device=device)
-    l_all = torch.empty((world, B, Hq), dtype=torch.float32, device=device)
+    # This rank's partial goes straight into its packed buffer (O rows, then
+    # lse); one all-gather lays the ranks' buffers end to end, and the merge
+    # reads them where they lie.  With one rank the packed buffer is the
+    # gathered one.
+    P = sharded.packed_floats(B, Hq, D)
+    send = torch.empty(P, dtype=torch.float32, device=device)
+    parts = torch.empty(world * P, dtype=torch.float32, device=device) if world > 1 else send
+    o, lse = sharded.unpack(send, B, Hq, D)
+    rows = B * Hq
     out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=device)
     lse_out = torch.empty((B, Hq), dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device).cuda_stream
@@ -711,12 +873,10 @@ def run_sharded(args):
         assert st == 0, fd.fd_status_string(st)
         if world > 1:
             import torch.distributed as dist
-            dist.all_gather_into_tensor(o_all, o)
-            dist.all_gather_into_tensor(l_all, lse)
-        else:
-            o_all[0].copy_(o)
-            l_all[0].copy_(lse)
-        st = fd.fd_combine(world, B, Hq, D, o_all, l_all, out, lse_out, stream)
+            dist.all_gather_into_tensor(parts, send)
+        base = parts.data_ptr()
+        st = fd.fd_combine_strided(world, B, Hq, D, base, P, base + 4 * rows * D, P, out,
+                                   lse_out, stream)
         assert st == 0, fd.fd_status_string(st)
 
     ms = max_over_ranks(torch, timed(torch, step, args.steps, args.warmup, barrier), world, device)
@@ -752,7 +912,7 @@ def crossover(args):
     call's own cost; eager calls below ~2K tokens are bound by the host's
     launch work), with cache copies rotated past L2.  Shapes: the CodeLlama-34B
     head shape (Hq=64, Hkv=8, D=128) at B=1 over L = 512..128K, at B = 2..40
-    over L = 2K..64K, and at B = 64 and 256 over L = 512..8K, bf16 and fp8
+    over L = 2K..64K, and at B = 64 and 256 over L = 512..64K and 512..16K, bf16 and fp8
     caches; G=4; the varlen, paged and peaked workloads.  One JSON line per shape on stdout, with the planner's pick
     (fd_plan_problem) and its regret against the fastest measured count."""
     import torch
@@ -806,7 +966,9 @@ def crossover(args):
                     [s for s in (1, 2, 3, 4, 6, 8, 12, 16, 24, 32) if s <= L // 64],
                     f"B{B}-L{L}-{kvd}")
     # Large batches: B * Hkv = 512 and 2048 CTAs at S = 1 already fill the device.
-    for B, Ls in ((64, (512, 2048, 8192)), (256, (512, 2048, 4096))):
+    # Up to 64K tokens at B = 64 and 16K at B = 256 (17 GB of cache each).
+    for B, Ls in ((64, (512, 2048, 8192, 16384, 32768, 65536)),
+                  (256, (512, 2048, 4096, 16384))):
         for L in Ls:
             run(lambda B=B, L=L: wl.make_problem(B, 64, 8, 128, L, wl.CONFIG_SEED_BASE + 200 + B,
                                                  name=f"B{B}-L{L}"),
@@ -820,6 +982,25 @@ def crossover(args):
 
 
 # ------------------------------------------------------- reference arm
+
+def reference_config(w, world):
+    """The repo arm's `config` for the same workload, so that the two lines
+    name the same problem: the split count is what the planner (host code)
+    picks for it, and the cache copies are those the repo arm rotates.  The
+    oracle itself neither splits nor rotates anything."""
+    import torch
+    import split_kv_decode_attn_b200 as fd
+    sms, l2 = 148, 126 * 1024 * 1024
+    if torch.cuda.is_available():
+        props = torch.cuda.get_device_properties(0)
+        sms, l2 = props.multi_processor_count, props.L2_cache_size
+    prob = fd.make_problem(w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size, w.num_blocks,
+                           w.max_blocks_per_seq, w.kv_layout, w.kv_dtype_code, w.k_scale,
+                           w.v_scale)
+    S = fd.fd_plan_problem(sms, prob, w.seqlens)
+    copies = max(2, math.ceil(4 * l2 / max(w.k.nbytes + w.v.nbytes, 1)))
+    return workload_config(w, S, fd.fd_effective_splits(w.max_len, S), copies, l2, world)
+
 
 def run_reference(args):
     """The fp64 CPU oracle timed as the reference arm, on this host's cores.
@@ -861,8 +1042,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
-                   "max_len": w.max_len},
+        "config": reference_config(w, world),
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
                          "sample": f"each step: all {w.Hq} query heads of one sequence over a "
                                    f"{n_tok}-token window of its history, {threads} threads"},
