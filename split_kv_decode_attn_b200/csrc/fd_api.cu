@@ -331,27 +331,38 @@ fd_status cached_cache_map(CUtensorMap* tm, const MapKey& key) {
 
 // --------------------------------------------------------------- launches
 
-// Stages of the split kernel's ring: about 96 KB, two CTAs per SM.  DEEP
-// (bf16, D = 128, a grid of at most one CTA per SM): the CTA has its SM to
-// itself and runs eight consumer warps over a 6-stage ring (192 KB; the
-// sparse decode, whose scan stages hold 32 KB of codes, 4 stages).
-template <int D, bool FP8, bool DEEP, bool SPARSE>
+// How a split CTA holds its SM (bf16, D = 128; every other case shares):
+//   kShared     two CTAs per SM: four consumer warps, 3 stages (96 KB)
+//   kDeepLong   one CTA per SM (grid <= SMs), splits of more than 64 tiles:
+//               eight consumer warps, 4 stages (128 KB)
+//   kDeepShort  one CTA per SM, splits of at most 64 tiles: eight consumer
+//               warps, 6 stages (192 KB)
+// Measured on one B200 with the CodeLlama-34B heads at S = 16 (interleaved
+// runs, eager us): 6 stages against 4, 32K 22.55 vs 23.18, 64K 40.67 vs
+// 41.53; but 128K 79.6 vs 77.8 and 256K 150.0 vs 149.3.  The sparse decode
+// (32 KB scan stages) keeps 4 stages at one CTA per SM.
+enum Ring { kShared = 0, kDeepLong = 1, kDeepShort = 2 };
+constexpr int kDeepShortMaxTiles = 64;
+
+template <int D, bool FP8, int RING, bool SPARSE>
 constexpr int split_stages() {
-  return (D == 128 && !FP8) ? (DEEP ? (SPARSE ? 4 : 6) : 3) : 6;
+  if (D != 128 || FP8) return 6;
+  if (RING == kShared) return 3;
+  return (RING == kDeepShort && !SPARSE) ? 6 : 4;
 }
 
-template <bool DEEP, bool SPARSE>
+template <int RING>
 constexpr int split_consumer_warps() {
-  return DEEP ? fd::kWideConsumerWarps : fd::kConsumerWarps;
+  return RING == kShared ? fd::kConsumerWarps : fd::kWideConsumerWarps;
 }
 
-template <int D, int NB, int MODE, bool PAGED, bool FP8 = false, bool DEEP = false,
+template <int D, int NB, int MODE, bool PAGED, bool FP8 = false, int RING = kShared,
           bool SPARSE = false>
 fd_status launch_split(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tc,
                        const fd::SplitArgs& a, int n_splits, int Hkv, int B,
                        cudaStream_t stream) {
-  constexpr int STAGES = split_stages<D, FP8, DEEP, SPARSE>();
-  constexpr int CW = split_consumer_warps<DEEP, SPARSE>();
+  constexpr int STAGES = split_stages<D, FP8, RING, SPARSE>();
+  constexpr int CW = split_consumer_warps<RING>();
   using L = fd::SplitSmem<D, NB, STAGES, FP8, SPARSE, CW>;
   auto kern = fd::fd_split_kernel<D, NB, MODE, PAGED, STAGES, FP8, SPARSE, CW>;
   // The shared-memory opt-in belongs to the device's context; remember the
@@ -385,8 +396,8 @@ template <int D>
 fd_status launch_combine(const fd::SplitArgs& a, int B, cudaStream_t stream) {
   cudaLaunchConfig_t cfg{};
   const int rows = B * a.Hq;
-  cfg.gridDim = dim3(static_cast<unsigned>((rows + 3) / 4));
-  cfg.blockDim = dim3(128);
+  cfg.gridDim = dim3(static_cast<unsigned>((rows + fd::kCombineWarps - 1) / fd::kCombineWarps));
+  cfg.blockDim = dim3(fd::kCombineWarps * 32);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -398,20 +409,20 @@ fd_status launch_combine(const fd::SplitArgs& a, int B, cudaStream_t stream) {
 }
 
 // Launches the split kernel and, with several splits, the combine kernel.
-// deep: the grid has at most one CTA per SM, so a deeper ring costs no
-// occupancy (bf16, D = 128 only; measured 5 % faster at 16K tokens, S = 16).
+// ring: how the CTAs hold their SMs (Ring; bf16, D = 128 only).
 // sparse: the low-bit scan and top-delta selection run first (contiguous
 // bf16 caches only).
 template <int D, int NB, int MODE, bool PAGED, bool FP8 = false>
 fd_status launch_call(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tc,
-                      const fd::SplitArgs& a, int n_splits, int Hkv, int B, bool deep,
+                      const fd::SplitArgs& a, int n_splits, int Hkv, int B, int ring,
                       bool sparse, cudaStream_t s) {
   fd_status r = FD_ERR_UNSUPPORTED;
   if constexpr (!PAGED && !FP8) {
     if (sparse) {
       if constexpr (D == 128) {
-        r = deep ? launch_split<D, NB, MODE, PAGED, FP8, true, true>(tk, tv, tc, a, n_splits, Hkv, B, s)
-                 : launch_split<D, NB, MODE, PAGED, FP8, false, true>(tk, tv, tc, a, n_splits, Hkv, B, s);
+        r = ring != kShared
+                ? launch_split<D, NB, MODE, PAGED, FP8, kDeepLong, true>(tk, tv, tc, a, n_splits, Hkv, B, s)
+                : launch_split<D, NB, MODE, PAGED, FP8, kShared, true>(tk, tv, tc, a, n_splits, Hkv, B, s);
         if (r == FD_OK && n_splits > 1) r = launch_combine<D>(a, B, s);
       }
       return r;
@@ -419,11 +430,15 @@ fd_status launch_call(const CUtensorMap& tk, const CUtensorMap& tv, const CUtens
   }
   if (sparse) return FD_ERR_UNSUPPORTED;
   if constexpr (D == 128 && !FP8) {
-    r = deep ? launch_split<D, NB, MODE, PAGED, FP8, true>(tk, tv, tc, a, n_splits, Hkv, B, s)
-             : launch_split<D, NB, MODE, PAGED, FP8, false>(tk, tv, tc, a, n_splits, Hkv, B, s);
+    if (ring == kDeepShort)
+      r = launch_split<D, NB, MODE, PAGED, FP8, kDeepShort>(tk, tv, tc, a, n_splits, Hkv, B, s);
+    else if (ring == kDeepLong)
+      r = launch_split<D, NB, MODE, PAGED, FP8, kDeepLong>(tk, tv, tc, a, n_splits, Hkv, B, s);
+    else
+      r = launch_split<D, NB, MODE, PAGED, FP8, kShared>(tk, tv, tc, a, n_splits, Hkv, B, s);
   } else {
-    (void)deep;
-    r = launch_split<D, NB, MODE, PAGED, FP8, false>(tk, tv, tc, a, n_splits, Hkv, B, s);
+    (void)ring;
+    r = launch_split<D, NB, MODE, PAGED, FP8, kShared>(tk, tv, tc, a, n_splits, Hkv, B, s);
   }
   if (r == FD_OK && n_splits > 1) r = launch_combine<D>(a, B, s);
   return r;
@@ -435,21 +450,21 @@ fd_status dispatch_split_fp8(int G, const CUtensorMap& tk, const CUtensorMap& tv
                              const fd::SplitArgs& a, int n_splits, int Hkv, int B,
                              cudaStream_t s) {
   if (G <= 8)
-    return launch_call<128, 1, fd::kHi, PAGED, true>(tk, tv, tk, a, n_splits, Hkv, B, false,
+    return launch_call<128, 1, fd::kHi, PAGED, true>(tk, tv, tk, a, n_splits, Hkv, B, kShared,
                                                      false, s);
-  return launch_call<128, 2, fd::kHi, PAGED, true>(tk, tv, tk, a, n_splits, Hkv, B, false, false,
-                                                   s);
+  return launch_call<128, 2, fd::kHi, PAGED, true>(tk, tv, tk, a, n_splits, Hkv, B, kShared,
+                                                   false, s);
 }
 
 template <int D, bool PAGED>
 fd_status dispatch_split(int G, const CUtensorMap& tk, const CUtensorMap& tv,
                          const CUtensorMap& tc, const fd::SplitArgs& a, int n_splits, int Hkv,
-                         int B, bool deep, bool sparse, cudaStream_t s) {
+                         int B, int ring, bool sparse, cudaStream_t s) {
   if (G <= 4)
-    return launch_call<D, 1, fd::kDup, PAGED>(tk, tv, tc, a, n_splits, Hkv, B, deep, sparse, s);
+    return launch_call<D, 1, fd::kDup, PAGED>(tk, tv, tc, a, n_splits, Hkv, B, ring, sparse, s);
   if (G == 8)
-    return launch_call<D, 1, fd::kHiLo, PAGED>(tk, tv, tc, a, n_splits, Hkv, B, deep, sparse, s);
-  return launch_call<D, 2, fd::kHiLo, PAGED>(tk, tv, tc, a, n_splits, Hkv, B, deep, sparse, s);
+    return launch_call<D, 1, fd::kHiLo, PAGED>(tk, tv, tc, a, n_splits, Hkv, B, ring, sparse, s);
+  return launch_call<D, 2, fd::kHiLo, PAGED>(tk, tv, tc, a, n_splits, Hkv, B, ring, sparse, s);
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -622,6 +637,7 @@ fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
   if (device_sms(dev, &sms) != FD_OK) return FD_ERR_CUDA;
   const long long grid = static_cast<long long>(B) * Hkv * n_splits;
   const bool deep = grid <= sms;
+  const int ring = !deep ? kShared : chunks.max_tiles <= kDeepShortMaxTiles ? kDeepShort : kDeepLong;
   a.prefetch_tiles = (paged || sp) ? 0 : prefetch_tiles(chunks.max_tiles, grid, sms, deep, fp8, D);
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -630,12 +646,12 @@ fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
     r = paged ? dispatch_split_fp8<true>(G, tk, tv, a, n_splits, Hkv, B, s)
               : dispatch_split_fp8<false>(G, tk, tv, a, n_splits, Hkv, B, s);
   else if (D == 128)
-    r = paged ? dispatch_split<128, true>(G, tk, tv, tk, a, n_splits, Hkv, B, deep, false, s)
-              : dispatch_split<128, false>(G, tk, tv, sp ? tc : tk, a, n_splits, Hkv, B, deep,
+    r = paged ? dispatch_split<128, true>(G, tk, tv, tk, a, n_splits, Hkv, B, ring, false, s)
+              : dispatch_split<128, false>(G, tk, tv, sp ? tc : tk, a, n_splits, Hkv, B, ring,
                                            sp != nullptr, s);
   else
-    r = paged ? dispatch_split<64, true>(G, tk, tv, tk, a, n_splits, Hkv, B, deep, false, s)
-              : dispatch_split<64, false>(G, tk, tv, tk, a, n_splits, Hkv, B, deep, false, s);
+    r = paged ? dispatch_split<64, true>(G, tk, tv, tk, a, n_splits, Hkv, B, ring, false, s)
+              : dispatch_split<64, false>(G, tk, tv, tk, a, n_splits, Hkv, B, ring, false, s);
   return r;
 }
 
@@ -824,8 +840,8 @@ fd_status fd_combine_strided(int R, int B, int Hq, int D, const float* part_o, s
   const fd_status arch = device_is_sm100(dev);
   if (arch != FD_OK) return arch;
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>((rows + 3) / 4));
-  cfg.blockDim = dim3(128);
+  cfg.gridDim = dim3(static_cast<unsigned>((rows + fd::kCombineWarps - 1) / fd::kCombineWarps));
+  cfg.blockDim = dim3(fd::kCombineWarps * 32);
   cfg.stream = reinterpret_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

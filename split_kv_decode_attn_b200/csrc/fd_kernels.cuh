@@ -35,6 +35,7 @@ constexpr int kTileWarps = 4;       // consumer warps per tile, 16 tokens each
 constexpr int kConsumerWarps = 4;   // consumer warps of a CTA sized for two CTAs per SM
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kCtasPerSm = 2;       // occupancy the split kernel is sized for
+constexpr int kCombineWarps = 4;    // rows (one per warp) per combine CTA
 // A CTA alone on its SM runs two sets of four consumer warps, which take the
 // even and the odd tiles: one warp per SM sub-partition is bound by the
 // latency of its tile loop, two hide it.
@@ -1053,8 +1054,8 @@ __global__ void __launch_bounds__(split_threads<CW>(), CW == kConsumerWarps ? kC
 }
 
 template <int D>
-__global__ void __launch_bounds__(128) fd_combine_kernel(const SplitArgs a, int B) {
-  const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+__global__ void __launch_bounds__(kCombineWarps * 32) fd_combine_kernel(const SplitArgs a, int B) {
+  const int row = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   // The lengths may be read before the wait: the split kernel, the grid this
   // one depends on, does not write them, and this grid launches only after
@@ -1088,13 +1089,13 @@ __global__ void __launch_bounds__(128) fd_combine_kernel(const SplitArgs a, int 
 // packed buffer per part when both strides are the part's size).  One warp
 // per row.
 template <int D>
-__global__ void __launch_bounds__(128) fd_merge_kernel(const float* part_o, const float* part_lse,
+__global__ void __launch_bounds__(kCombineWarps * 32) fd_merge_kernel(const float* part_o, const float* part_lse,
                                                        int R, int rows, size_t o_stride,
                                                        size_t l_stride, __nv_bfloat16* out,
                                                        float* lse) {
   grid_dependency_wait();
   grid_dependents_launch();
-  const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int row = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
   combine_row<D>(part_o + static_cast<size_t>(row) * D, part_lse + row, R, o_stride, l_stride,
