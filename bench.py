@@ -715,6 +715,10 @@ def sweep(torch, fd, device, n_samples=10):
         row.update(sample_stats(per, calls, w.kv_bytes(), peak))
         row.update({"graph_us_per_call": round(g_us, 3), "graph_GB/s": round(g_gbs, 1),
                     "graph_frac_measured": round(g_gbs / peak, 4)})
+        kt = kernel_times(ncu_launch_shares(w.name, call.S), row["us_per_call_median"],
+                          w.kv_bytes(), peak)
+        if kt:
+            row["kernels"] = kt
         rows.append(row)
         del call
         torch.cuda.empty_cache()
