@@ -925,7 +925,7 @@ def crossover(args):
     torch.cuda.set_device(0)
     device = torch.device("cuda", 0)
     fd.load_library()
-    ladder = (1, 2, 3, 4, 6, 8, 12, 16, 20, 24, 28, 32, 40, 48, 64)
+    ladder = (1, 2, 3, 4, 6, 8, 12, 16, 18, 20, 24, 28, 32, 40, 48, 64)
 
     def run(make, Ss, tag):
         """make: builds the workload (only for the shapes that are run)."""
@@ -981,7 +981,11 @@ def crossover(args):
         run(lambda kvd=kvd: make_workload("varlen", None, 0, kv_dtype=kvd), [1, 2, 3, 4, 6, 8],
             f"varlen-{kvd}")
     run(lambda: make_workload("paged", None, 0), [1, 2, 3, 4, 6, 8], "paged-bf16")
+    run(lambda: make_workload("paged", None, 0, kv_dtype="fp8"), [2, 3, 4, 6, 8, 9, 12],
+        "paged-fp8")
     run(lambda: make_workload("peaked", None, 0), [8, 12, 16, 20, 24, 32, 48, 64], "peaked-bf16")
+    run(lambda: make_workload("peaked", None, 0, kv_dtype="fp8"), [16, 18, 24, 32, 48],
+        "peaked-fp8")
     assert fd.fd_check_device_error() == 0
 
 

@@ -38,24 +38,28 @@ constexpr int kMaxDevices = 64;
 //   kCtaTokPerUs       tokens per microsecond of one CTA
 //   kCtaDeepTokPerUs   the same for a bf16 D = 128 grid of at most one CTA
 //                      per SM, which runs the deeper ring
-//   kCtaFp8TokPerUs    the same for an fp8 cache
+//   kCtaFp8TokPerUs    the same for an fp8 cache, two CTAs per SM
+//   kCtaFp8DeepTokPerUs  an fp8 CTA alone on its SM (grid <= SMs), with eight
+//                      consumer warps
 //   kCtaPagedTokPerUs  alone on an SM when pages hold fewer than 64 tokens
 //                      (one TMA box per page instead of one per tile) ...
 //   kCtaPagedSharedTokPerUs  ... and two to an SM (bf16 or fp8)
 //   kCtaFixedUs        per-CTA fixed cost within a wave
 //   kCombineUs         device time added by a call with several splits (the
 //                      combine kernel after its dependency) ...
-//   kCombinePer16Us    ... plus this per 16 splits merged
+//   kCombinePer32Us    ... plus this per 32 splits merged (one L2 round trip
+//                      per batch of 32 partial rows)
 struct PlanModel {
   static constexpr double kHbmGBs = 6500.0;
   static constexpr double kCtaTokPerUs = 90.0;
   static constexpr double kCtaDeepTokPerUs = 100.0;
   static constexpr double kCtaFp8TokPerUs = 100.0;
+  static constexpr double kCtaFp8DeepTokPerUs = 180.0;
   static constexpr double kCtaPagedTokPerUs = 50.0;
   static constexpr double kCtaPagedSharedTokPerUs = 80.0;
   static constexpr double kCtaFixedUs = 0.3;
   static constexpr double kCombineUs = 1.0;
-  static constexpr double kCombinePer16Us = 2.0;
+  static constexpr double kCombinePer32Us = 2.0;
 };
 
 // How a call cuts the history: T = ceil(max_len / 64) tiles into S = min(S
@@ -91,7 +95,7 @@ struct PlanShape {
   int Hkv;
   double token_bytes;  // K + V bytes of one token of one KV head
   bool small_pages;    // pages of fewer than 64 tokens
-  bool deep_ring;      // bf16, D = 128: a grid of <= num_sms CTAs gets the deep ring
+  bool deep_ring;      // D = 128: a grid of <= num_sms CTAs gets the deep ring
   bool fp8;            // fp8 E4M3 cache
 };
 
@@ -102,7 +106,9 @@ double wave_time_us(const PlanShape& ps, double tokens, double k, double grid) {
   double own = PlanModel::kCtaTokPerUs;
   if (ps.small_pages)
     own = k <= ps.num_sms ? PlanModel::kCtaPagedTokPerUs : PlanModel::kCtaPagedSharedTokPerUs;
-  else if (ps.fp8) own = PlanModel::kCtaFp8TokPerUs;
+  else if (ps.fp8)
+    own = ps.deep_ring && grid <= ps.num_sms ? PlanModel::kCtaFp8DeepTokPerUs
+                                             : PlanModel::kCtaFp8TokPerUs;
   else if (ps.deep_ring && grid <= ps.num_sms) own = PlanModel::kCtaDeepTokPerUs;
   return tokens / std::min(hbm_tok, own) + PlanModel::kCtaFixedUs;
 }
@@ -124,7 +130,7 @@ double model_time_us(const PlanShape& ps, double n_ctas, double tokens, double m
   if (rem > 0) waves += wave_time_us(ps, mean, rem, grid);
   const double longest = wave_time_us(ps, max_cta, std::min(n_ctas, slots), grid);
   double t = std::max(waves, longest);
-  if (s_eff > 1) t += PlanModel::kCombineUs + PlanModel::kCombinePer16Us * std::ceil(s_eff / 16.0);
+  if (s_eff > 1) t += PlanModel::kCombineUs + PlanModel::kCombinePer32Us * std::ceil(s_eff / 32.0);
   return t;
 }
 
@@ -331,22 +337,26 @@ fd_status cached_cache_map(CUtensorMap* tm, const MapKey& key) {
 
 // --------------------------------------------------------------- launches
 
-// How a split CTA holds its SM (bf16, D = 128; every other case shares):
-//   kShared     two CTAs per SM: four consumer warps, 3 stages (96 KB)
+// How a split CTA holds its SM (D = 128; D = 64 always shares):
+//   kShared     two CTAs per SM: four consumer warps; bf16 3 stages (96 KB),
+//               fp8 6 stages of 16 KB (96 KB)
 //   kDeepLong   one CTA per SM (grid <= SMs), splits of more than 64 tiles:
-//               eight consumer warps, 4 stages (128 KB)
+//               eight consumer warps; bf16 4 stages (128 KB), fp8 8 (128 KB)
 //   kDeepShort  one CTA per SM, splits of at most 64 tiles: eight consumer
-//               warps, 6 stages (192 KB)
+//               warps; bf16 6 stages (192 KB), fp8 12 (192 KB)
 // Measured on one B200 with the CodeLlama-34B heads at S = 16 (interleaved
-// runs, eager us): 6 stages against 4, 32K 22.55 vs 23.18, 64K 40.67 vs
-// 41.53; but 128K 79.6 vs 77.8 and 256K 150.0 vs 149.3.  The sparse decode
-// (32 KB scan stages) keeps 4 stages at one CTA per SM.
+// runs, eager us): bf16 6 stages against 4, 32K 22.55 vs 23.18, 64K 40.67 vs
+// 41.53; but 128K 79.6 vs 77.8 and 256K 150.0 vs 149.3.  fp8 at S = 18 (one
+// CTA per SM) against S = 32 (two per SM on most SMs): 32K 15.0 vs 15.55,
+// 64K 24.1 vs 24.75, 128K 43.3 vs 45.4, 256K 79.9 vs 82.7.  The sparse
+// decode (32 KB scan stages) keeps 4 stages at one CTA per SM.
 enum Ring { kShared = 0, kDeepLong = 1, kDeepShort = 2 };
 constexpr int kDeepShortMaxTiles = 64;
 
 template <int D, bool FP8, int RING, bool SPARSE>
 constexpr int split_stages() {
-  if (D != 128 || FP8) return 6;
+  if (FP8) return RING == kShared ? 6 : (RING == kDeepShort ? 12 : 8);
+  if (D != 128) return 6;
   if (RING == kShared) return 3;
   return (RING == kDeepShort && !SPARSE) ? 6 : 4;
 }
@@ -429,7 +439,7 @@ fd_status launch_call(const CUtensorMap& tk, const CUtensorMap& tv, const CUtens
     }
   }
   if (sparse) return FD_ERR_UNSUPPORTED;
-  if constexpr (D == 128 && !FP8) {
+  if constexpr (D == 128) {
     if (ring == kDeepShort)
       r = launch_split<D, NB, MODE, PAGED, FP8, kDeepShort>(tk, tv, tc, a, n_splits, Hkv, B, s);
     else if (ring == kDeepLong)
@@ -447,12 +457,12 @@ fd_status launch_call(const CUtensorMap& tk, const CUtensorMap& tv, const CUtens
 // fp8 caches (D = 128): f16 contraction, bf16(p) residuals not needed.
 template <bool PAGED>
 fd_status dispatch_split_fp8(int G, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const fd::SplitArgs& a, int n_splits, int Hkv, int B,
+                             const fd::SplitArgs& a, int n_splits, int Hkv, int B, int ring,
                              cudaStream_t s) {
   if (G <= 8)
-    return launch_call<128, 1, fd::kHi, PAGED, true>(tk, tv, tk, a, n_splits, Hkv, B, kShared,
+    return launch_call<128, 1, fd::kHi, PAGED, true>(tk, tv, tk, a, n_splits, Hkv, B, ring,
                                                      false, s);
-  return launch_call<128, 2, fd::kHi, PAGED, true>(tk, tv, tk, a, n_splits, Hkv, B, kShared,
+  return launch_call<128, 2, fd::kHi, PAGED, true>(tk, tv, tk, a, n_splits, Hkv, B, ring,
                                                    false, s);
 }
 
@@ -643,8 +653,8 @@ fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   fd_status r;
   if (fp8)
-    r = paged ? dispatch_split_fp8<true>(G, tk, tv, a, n_splits, Hkv, B, s)
-              : dispatch_split_fp8<false>(G, tk, tv, a, n_splits, Hkv, B, s);
+    r = paged ? dispatch_split_fp8<true>(G, tk, tv, a, n_splits, Hkv, B, ring, s)
+              : dispatch_split_fp8<false>(G, tk, tv, a, n_splits, Hkv, B, ring, s);
   else if (D == 128)
     r = paged ? dispatch_split<128, true>(G, tk, tv, tk, a, n_splits, Hkv, B, ring, false, s)
               : dispatch_split<128, false>(G, tk, tv, sp ? tc : tk, a, n_splits, Hkv, B, ring,
@@ -663,8 +673,7 @@ int plan_impl(int num_sms, int B, int Hkv, int D, int max_len, int block_size, i
   // planning cost for large batches).
   if (static_cast<long long>(B) * Hkv >= 2LL * num_sms * fd::kCtasPerSm) return 1;
   const PlanShape ps{num_sms, B, Hkv, 2.0 * D * elem_bytes,
-                     block_size > 0 && block_size < fd::kTile, elem_bytes == 2 && D == 128,
-                     elem_bytes == 1};
+                     block_size > 0 && block_size < fd::kTile, D == 128, elem_bytes == 1};
   const long long units = static_cast<long long>(B) * Hkv;
   const int slots = num_sms * fd::kCtasPerSm;
   if (seqlens)

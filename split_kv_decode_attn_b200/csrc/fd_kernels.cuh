@@ -33,7 +33,6 @@ namespace fd {
 constexpr int kTile = 64;           // tokens per pipeline stage
 constexpr int kTileWarps = 4;       // consumer warps per tile, 16 tokens each
 constexpr int kConsumerWarps = 4;   // consumer warps of a CTA sized for two CTAs per SM
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kCtasPerSm = 2;       // occupancy the split kernel is sized for
 constexpr int kCombineWarps = 4;    // rows (one per warp) per combine CTA
 // A CTA alone on its SM runs two sets of four consumer warps, which take the
