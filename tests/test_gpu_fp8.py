@@ -50,6 +50,22 @@ def test_fp8_group_sizes_and_ragged_lengths(G):
         assert_close(got, gl, ref, rl, f"fp8 G={G} S={S}")
 
 
+@pytest.mark.parametrize("G", [1, 8, 16])
+def test_fp8_long_splits_at_one_cta_per_sm_ragged(G):
+    """fp8 splits of more than 64 tiles on a grid of at most one CTA per SM
+    (eight consumer warps, 8-stage ring), ragged lengths and NaN codes past
+    every length; and splits of at most 64 tiles (12-stage ring)."""
+    Hkv = 2
+    lens = [0, 1, 4097, 5000, 9000]
+    w = wl.make_problem(len(lens), G * Hkv, Hkv, 128, 9000, seed=310 + G, seqlens=lens,
+                        nan_pad=True, kv_dtype="fp8")
+    d = OnDevice(w)
+    ref, rl = reference(w)
+    for S in (1, 2, 3):     # 141, 71 and 47 tiles per split
+        got, gl, _ = run_gpu(d, S)
+        assert_close(got, gl, ref, rl, f"fp8 long splits G={G} S={S}")
+
+
 @pytest.mark.parametrize("layout", ["HND", "NHD"])
 @pytest.mark.parametrize("bs", [16, 64, 256])
 def test_fp8_paged_matches_contiguous_bit_for_bit(bs, layout):

@@ -101,6 +101,22 @@ def test_group_sizes_and_ragged_lengths(G, D):
         assert_close(got, gl, ref, rl, f"G={G} D={D} S={S}")
 
 
+@pytest.mark.parametrize("G", [1, 4, 8, 16])
+def test_long_splits_at_one_cta_per_sm_ragged(G):
+    """Splits of more than 64 tiles on a grid of at most one CTA per SM: the
+    eight consumer warps over the shorter ring, with ragged lengths, an
+    empty sequence and NaN padding past every length."""
+    Hkv = 2
+    lens = [0, 1, 4097, 5000, 9000]
+    w = wl.make_problem(len(lens), G * Hkv, Hkv, 128, 9000, seed=150 + G, seqlens=lens,
+                        nan_pad=True)
+    d = OnDevice(w)
+    ref, rl = reference(w)
+    for S in (1, 2):        # 141 and 71 tiles per split, 10 and 20 CTAs
+        got, gl, _ = run_gpu(d, S)
+        assert_close(got, gl, ref, rl, f"long splits G={G} S={S}")
+
+
 def test_all_sequences_empty():
     w = wl.make_problem(3, 16, 2, 128, 500, seed=5, seqlens=[0, 0, 0])
     d = OnDevice(w)
