@@ -81,6 +81,22 @@ typedef enum fd_kv_dtype {
   FD_KV_FP8_E4M3 = 1  /* OCP fp8 e4m3 (bias 7, max 448, no inf); value = scale * code */
 } fd_kv_dtype;
 
+/* Tensor-core path of an fp8 cache.
+ *   FD_FP8_MMA_SYNC     the default: e4m3 codes converted to f16 in registers,
+ *                       both contractions on mma.sync with fp32 accumulation.
+ *   FD_FP8_MMA_TCGEN05  kind::f8f6f4 tcgen05 MMAs on the codes as the TMA left
+ *                       them in shared memory, accumulators in tensor memory;
+ *                       q and the softmax weights enter as sums of e4m3 codes
+ *                       (q exactly, the weights to 12 significant bits). Taken
+ *                       where G is 2, 4 or 8 and the grid has at most one CTA
+ *                       per SM; other calls run the default path. Measured
+ *                       slower on B200 (CodeLlama-34B heads, 64K tokens:
+ *                       40.8 against 24.2 us per call). */
+typedef enum fd_fp8_mma {
+  FD_FP8_MMA_SYNC = 0,
+  FD_FP8_MMA_TCGEN05 = 1
+} fd_fp8_mma;
+
 /* Shape of one decode-attention call.
  *   B           sequences in the batch (1 .. 65535)
  *   Hq, Hkv     query heads and KV heads (Hkv .. 65535, Hq % Hkv == 0)
@@ -96,8 +112,11 @@ typedef enum fd_kv_dtype {
  *   k_scale, v_scale
  *               fp8 caches: the real K and V are k_scale * code and
  *               v_scale * code (finite, > 0). Ignored for bf16 caches.
- *               An fp8 cache needs D = 128, and the contraction runs on f16
- *               tensor cores: q must be finite in f16 (|q| < 65504). */
+ *               An fp8 cache needs D = 128; on the default path the
+ *               contraction runs on f16 tensor cores, so q must be finite
+ *               in f16 (|q| < 65504).
+ *   fp8_mma     an fd_fp8_mma value (FD_FP8_MMA_SYNC when zero-initialised);
+ *               ignored for bf16 caches. */
 typedef struct fd_problem {
   int32_t B;
   int32_t Hq;
@@ -111,6 +130,7 @@ typedef struct fd_problem {
   int32_t kv_dtype;
   float k_scale;
   float v_scale;
+  int32_t fp8_mma;
 } fd_problem;
 
 /* Split-count planner.

@@ -49,6 +49,8 @@ FD_LAYOUT_HND = 0  # cache [.., Hkv, tokens, D]
 FD_LAYOUT_NHD = 1  # cache [.., tokens, Hkv, D]
 FD_KV_BF16 = 0       # bf16 cache
 FD_KV_FP8_E4M3 = 1   # fp8 e4m3 cache, real value = scale * code
+FD_FP8_MMA_SYNC = 0     # fp8: codes converted to f16, mma.sync (default)
+FD_FP8_MMA_TCGEN05 = 1  # fp8: tcgen05 kind::f8f6f4 on the codes in shared memory
 
 
 class fd_problem(ctypes.Structure):
@@ -57,7 +59,7 @@ class fd_problem(ctypes.Structure):
                 ("block_size", ctypes.c_int32), ("num_blocks", ctypes.c_int32),
                 ("max_blocks_per_seq", ctypes.c_int32), ("kv_layout", ctypes.c_int32),
                 ("kv_dtype", ctypes.c_int32), ("k_scale", ctypes.c_float),
-                ("v_scale", ctypes.c_float)]
+                ("v_scale", ctypes.c_float), ("fp8_mma", ctypes.c_int32)]
 
 
 _lib = None
@@ -266,9 +268,10 @@ def fd_selftest_device_timeout(limit_us: int, stream=None) -> int:
 # ---- convenience wrapper -----------------------------------------------------
 
 def make_problem(B, Hq, Hkv, D, max_len, block_size=0, num_blocks=0, max_blocks_per_seq=0,
-                 kv_layout=FD_LAYOUT_HND, kv_dtype=FD_KV_BF16, k_scale=1.0, v_scale=1.0):
+                 kv_layout=FD_LAYOUT_HND, kv_dtype=FD_KV_BF16, k_scale=1.0, v_scale=1.0,
+                 fp8_mma=0):
     return fd_problem(B, Hq, Hkv, D, max_len, block_size, num_blocks, max_blocks_per_seq,
-                      kv_layout, kv_dtype, k_scale, v_scale)
+                      kv_layout, kv_dtype, k_scale, v_scale, fp8_mma)
 
 
 def _check(t, name, dtypes, shape=None):

@@ -402,6 +402,37 @@ fd_status launch_split(const CUtensorMap& tk, const CUtensorMap& tv, const CUten
   return FD_OK;
 }
 
+// The fp8 split kernel on tcgen05 (D = 128, G in {2, 4, 8}, one CTA per SM).
+template <bool PAGED, int STAGES, int G>
+fd_status launch_split_tc(const CUtensorMap& tk, const CUtensorMap& tv, const fd::SplitArgs& a,
+                          int n_splits, int Hkv, int B, cudaStream_t stream) {
+  using L = fd::TcSmem<STAGES>;
+  auto kern = fd::fd_split_tc_kernel<PAGED, STAGES, G>;
+  static std::atomic<unsigned long long> attr_ctx[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FD_ERR_CUDA;
+  const unsigned long long ctx = current_context_id();
+  if (ctx == 0 || attr_ctx[dev].load() != ctx) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             L::kDynamicBytes) != cudaSuccess)
+      return FD_ERR_CUDA;
+    attr_ctx[dev].store(ctx);
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(n_splits), static_cast<unsigned>(Hkv),
+                     static_cast<unsigned>(B));
+  cfg.blockDim = dim3(fd::kTcThreads);
+  cfg.dynamicSmemBytes = L::kDynamicBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, tk, tv, a) != cudaSuccess) return FD_ERR_CUDA;
+  return FD_OK;
+}
+
 template <int D>
 fd_status launch_combine(const fd::SplitArgs& a, int B, cudaStream_t stream) {
   cudaLaunchConfig_t cfg{};
@@ -454,11 +485,30 @@ fd_status launch_call(const CUtensorMap& tk, const CUtensorMap& tv, const CUtens
   return r;
 }
 
-// fp8 caches (D = 128): f16 contraction, bf16(p) residuals not needed.
+// fp8 caches (D = 128).  mma.sync: codes converted to f16 in registers, f16
+// contraction, bf16(p) residuals not needed.  tcgen05: the tcgen05 kernel
+// where it applies (G in {2, 4, 8}, one CTA per SM).
 template <bool PAGED>
 fd_status dispatch_split_fp8(int G, const CUtensorMap& tk, const CUtensorMap& tv,
                              const fd::SplitArgs& a, int n_splits, int Hkv, int B, int ring,
-                             cudaStream_t s) {
+                             bool tcgen05, cudaStream_t s) {
+  if (tcgen05 && (G == 2 || G == 4 || G == 8) && ring != kShared) {
+    // One CTA per SM: the tcgen05 kernel, with the rings of the mma.sync one.
+    constexpr int kShort = split_stages<128, true, kDeepShort, false>();
+    constexpr int kLong = split_stages<128, true, kDeepLong, false>();
+    fd_status r;
+    if (G == 8)
+      r = ring == kDeepShort ? launch_split_tc<PAGED, kShort, 8>(tk, tv, a, n_splits, Hkv, B, s)
+                             : launch_split_tc<PAGED, kLong, 8>(tk, tv, a, n_splits, Hkv, B, s);
+    else if (G == 4)
+      r = ring == kDeepShort ? launch_split_tc<PAGED, kShort, 4>(tk, tv, a, n_splits, Hkv, B, s)
+                             : launch_split_tc<PAGED, kLong, 4>(tk, tv, a, n_splits, Hkv, B, s);
+    else
+      r = ring == kDeepShort ? launch_split_tc<PAGED, kShort, 2>(tk, tv, a, n_splits, Hkv, B, s)
+                             : launch_split_tc<PAGED, kLong, 2>(tk, tv, a, n_splits, Hkv, B, s);
+    if (r == FD_OK && n_splits > 1) r = launch_combine<128>(a, B, s);
+    return r;
+  }
   if (G <= 8)
     return launch_call<128, 1, fd::kHi, PAGED, true>(tk, tv, tk, a, n_splits, Hkv, B, ring,
                                                      false, s);
@@ -553,6 +603,7 @@ fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
   }
   if (p->kv_layout != FD_LAYOUT_HND && p->kv_layout != FD_LAYOUT_NHD) return FD_ERR_INVALID_ARGUMENT;
   if (p->kv_dtype != FD_KV_BF16 && p->kv_dtype != FD_KV_FP8_E4M3) return FD_ERR_INVALID_ARGUMENT;
+  if (p->fp8_mma != FD_FP8_MMA_SYNC && p->fp8_mma != FD_FP8_MMA_TCGEN05) return FD_ERR_INVALID_ARGUMENT;
   const bool fp8 = p->kv_dtype == FD_KV_FP8_E4M3;
   if (fp8) {
     if (p->D != 128) return FD_ERR_UNSUPPORTED;
@@ -652,9 +703,10 @@ fd_status decode_impl(const fd_problem* p, const void* q, const void* k_cache,
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   fd_status r;
+  const bool tcgen05 = p->fp8_mma == FD_FP8_MMA_TCGEN05;
   if (fp8)
-    r = paged ? dispatch_split_fp8<true>(G, tk, tv, a, n_splits, Hkv, B, ring, s)
-              : dispatch_split_fp8<false>(G, tk, tv, a, n_splits, Hkv, B, ring, s);
+    r = paged ? dispatch_split_fp8<true>(G, tk, tv, a, n_splits, Hkv, B, ring, tcgen05, s)
+              : dispatch_split_fp8<false>(G, tk, tv, a, n_splits, Hkv, B, ring, tcgen05, s);
   else if (D == 128)
     r = paged ? dispatch_split<128, true>(G, tk, tv, tk, a, n_splits, Hkv, B, ring, false, s)
               : dispatch_split<128, false>(G, tk, tv, sp ? tc : tk, a, n_splits, Hkv, B, ring,

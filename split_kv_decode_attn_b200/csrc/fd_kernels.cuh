@@ -24,6 +24,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cstdint>
 
 #include "fd_ptx.cuh"
@@ -389,6 +390,95 @@ __device__ __forceinline__ bool sparse_scan_consumer(const SplitArgs& a, uint32_
 // split's result, which goes to `out` (the sequence has one split) or to the
 // global partials (several splits).  Warp w takes tokens 16 (w mod 4) ..
 // +15 of every (CW / 4)-th tile, starting at tile w / 4.
+// The last step of a split: merge the CW consumer warps' states (running
+// maximum and sum per head in log2 units, unnormalised accumulator rows),
+// which the warps left in shared memory at L::kRedM, L::kRedL and
+// L::kRedAcc, into the split's partial output and log-sum-exp (or the final
+// result when the sequence has a single split).
+template <int D, int NB, int MODE, int CW, class L>
+__device__ __forceinline__ void split_merge(const SplitArgs& a, const float* f, int b, int h0,
+                                            int split, int n_parts) {
+  constexpr int NCOL = L::kNcol;
+  // One pass with no further barrier.  Each thread merges the CW warp
+  // states for 4 * kParts head-dim entries of one head (4 at d0, and with
+  // four consumer warps 4 more at d0 + D/2, so that a warp's 16-byte reads
+  // and writes are contiguous) and computes that head's weights itself from a
+  // few broadcast reads.  Eight consumer warps take 4 entries each, so that
+  // all 256 threads share the merge of the G = 8 heads.  (A separate per-head
+  // pass behind two more barriers took about 1.5 us per CTA.)
+  constexpr int kParts = CW == kConsumerWarps ? 2 : 1;
+  constexpr int kChunks = D / (4 * kParts);  // chunks of 4 * kParts entries per head
+  const bool direct = n_parts == 1;
+  for (int c = threadIdx.x; c < a.G * kChunks; c += CW * 32) {
+    const int g = c / kChunks;
+    const int d0 = (c - g * kChunks) * 4;
+    float mw[CW];
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < CW; ++w) {
+      mw[w] = f[L::kRedM + w * NCOL + g];
+      M = fmaxf(M, mw[w]);
+    }
+    float wt[CW];
+    float lse_s = -INFINITY;
+    if (M == -INFINITY) {  // no token in this split
+#pragma unroll
+      for (int w = 0; w < CW; ++w) wt[w] = 0.f;
+    } else {
+      float Ls = 0.f;
+#pragma unroll
+      for (int w = 0; w < CW; ++w) {
+        wt[w] = ex2(mw[w] - M);
+        Ls += wt[w] * f[L::kRedL + w * NCOL + g];
+      }
+      const float inv = a.v_scale / Ls;  // an fp8 V cache is dequantised here
+#pragma unroll
+      for (int w = 0; w < CW; ++w) wt[w] *= inv;
+      lse_s = (M + log2f(Ls)) * 0.69314718055994530942f;
+    }
+    float4 o[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+#pragma unroll
+    for (int w = 0; w < CW; ++w) {
+      const float* src = f + L::kRedAcc + (w * NCOL + g) * L::kAccStride + d0;
+#pragma unroll
+      for (int h = 0; h < kParts; ++h) {
+        float4 v = *reinterpret_cast<const float4*>(src + h * (D / 2));
+        if constexpr (MODE == kDup) {  // columns g + 4 hold the bf16 residuals
+          const float4 r = *reinterpret_cast<const float4*>(src + 4 * L::kAccStride + h * (D / 2));
+          v.x += r.x;
+          v.y += r.y;
+          v.z += r.z;
+          v.w += r.w;
+        }
+        o[h].x += wt[w] * v.x;
+        o[h].y += wt[w] * v.y;
+        o[h].z += wt[w] * v.z;
+        o[h].w += wt[w] * v.w;
+      }
+    }
+    const size_t row = static_cast<size_t>(b) * a.Hq + h0 + g;
+    if (direct) {
+      if (a.out_f32) {
+        float* dst = a.out_f32 + row * D + d0;
+#pragma unroll
+        for (int h = 0; h < kParts; ++h) *reinterpret_cast<float4*>(dst + h * (D / 2)) = o[h];
+      } else {
+        __nv_bfloat16* dst = a.out + row * D + d0;
+#pragma unroll
+        for (int h = 0; h < kParts; ++h)
+          *reinterpret_cast<uint2*>(dst + h * (D / 2)) =
+              make_uint2(pack_bf16x2(o[h].x, o[h].y), pack_bf16x2(o[h].z, o[h].w));
+      }
+      if (d0 == 0 && a.lse) a.lse[row] = lse_s;
+    } else {
+      float* dst = a.part_o + (row * a.n_splits + split) * D + d0;
+#pragma unroll
+      for (int h = 0; h < kParts; ++h) *reinterpret_cast<float4*>(dst + h * (D / 2)) = o[h];
+      if (d0 == 0) a.part_lse[row * a.n_splits + split] = lse_s;
+    }
+  }
+}
+
 template <int D, int NB, int MODE, int STAGES, bool FP8, bool SPARSE, int CW = kConsumerWarps>
 __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* smem,
                                                 uint32_t smem_base, uint32_t bar_full,
@@ -729,83 +819,97 @@ __device__ __forceinline__ void split_consumers(const SplitArgs& a, uint8_t* sme
   named_barrier_sync(1, CW * 32);
   if (!live) return;
 
-  // One pass with no further barrier.  Each thread merges the CW warp
-  // states for 4 * kParts head-dim entries of one head (4 at d0, and with
-  // four consumer warps 4 more at d0 + D/2, so that a warp's 16-byte reads
-  // and writes are contiguous) and computes that head's weights itself from a
-  // few broadcast reads.  Eight consumer warps take 4 entries each, so that
-  // all 256 threads share the merge of the G = 8 heads.  (A separate per-head
-  // pass behind two more barriers took about 1.5 us per CTA.)
-  constexpr int kParts = CW == kConsumerWarps ? 2 : 1;
-  constexpr int kChunks = D / (4 * kParts);  // chunks of 4 * kParts entries per head
-  const bool direct = n_parts == 1;
-  for (int c = threadIdx.x; c < a.G * kChunks; c += CW * 32) {
-    const int g = c / kChunks;
-    const int d0 = (c - g * kChunks) * 4;
-    float mw[CW];
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < CW; ++w) {
-      mw[w] = f[L::kRedM + w * NCOL + g];
-      M = fmaxf(M, mw[w]);
-    }
-    float wt[CW];
-    float lse_s = -INFINITY;
-    if (M == -INFINITY) {  // no token in this split
-#pragma unroll
-      for (int w = 0; w < CW; ++w) wt[w] = 0.f;
-    } else {
-      float Ls = 0.f;
-#pragma unroll
-      for (int w = 0; w < CW; ++w) {
-        wt[w] = ex2(mw[w] - M);
-        Ls += wt[w] * f[L::kRedL + w * NCOL + g];
+  split_merge<D, NB, MODE, CW, L>(a, f, b, h0, split, n_parts);
+}
+
+// The producer warp of a split CTA: streams the split's K/V tiles (or the
+// listed ones) into the ring, one stage per tile, after it_base earlier ring
+// uses.  Stage s holds its K tile at s * STAGE_STRIDE and its V tile
+// V_OFFSET bytes further.  Contiguous caches take one TMA box per tensor and tile; paged caches
+// one box per page, the page ids read from the block table 32 at a time.
+// Every lane waits (the decision is made warp-uniform); lane 0 issues.
+// Before returning it waits until no copy is still landing in shared memory.
+template <bool PAGED, bool SPARSE, int STAGES, int STAGE_STRIDE, int V_OFFSET, int HALVES>
+__device__ __forceinline__ void split_producer(const SplitArgs& a, const CUtensorMap* tmK,
+                                               const CUtensorMap* tmV, uint32_t smem_base,
+                                               uint32_t bar_full, uint32_t bar_empty,
+                                               volatile int* cta_error, int lane, int b, int kvh,
+                                               int start, int n, int n_work, int it_base,
+                                               const uint16_t* list) {
+  const uint64_t policy = policy_evict_first();
+  int issued = it_base;   // ring uses so far (the sparse scan's stages)
+  bool ok = true;
+  if constexpr (!PAGED) {
+    for (int it = 0; it < n_work; ++it) {
+      const int ig = it_base + it;
+      const int s = ig % STAGES, k = ig / STAGES;
+      if (k > 0) ok = mbar_wait(bar_empty + 8 * s, (k - 1) & 1, kWaitLimitNs);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      if (lane == 0) {
+        const int t0 = start + (SPARSE ? static_cast<int>(list[it]) : it) * kTile;
+        const uint32_t dk = smem_base + s * STAGE_STRIDE;
+        const uint32_t dv = dk + V_OFFSET;
+        mbar_arrive_expect_tx(bar_full + 8 * s, 2 * kTile * 128 * HALVES);
+        tma_load_5d(dk, tmK, bar_full + 8 * s, 0, kvh, t0, 0, b, policy);
+        tma_load_5d(dv, tmV, bar_full + 8 * s, 0, kvh, t0, 0, b, policy);
       }
-      const float inv = a.v_scale / Ls;  // an fp8 V cache is dequantised here
-#pragma unroll
-      for (int w = 0; w < CW; ++w) wt[w] *= inv;
-      lse_s = (M + log2f(Ls)) * 0.69314718055994530942f;
+      ++issued;
+      __syncwarp();
     }
-    float4 o[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+  } else {
+    const int bs = a.block_size, lbs = a.log2_block_size;
+    const int rows = bs < kTile ? bs : kTile;            // rows per TMA box
+    const int pages_per_tile = bs < kTile ? kTile / bs : 1;
+    const int n_pages = (n + bs - 1) >> lbs;
+    const int32_t* bt = a.block_table + static_cast<size_t>(b) * a.max_blocks_per_seq;
+    // A window of 32 page ids, one per lane, plus the next window in flight.
+    int win = start >> lbs;
+    int cur = (win + lane < n_pages) ? __ldg(bt + win + lane) : 0;
+    int nxt = (win + 32 + lane < n_pages) ? __ldg(bt + win + 32 + lane) : 0;
+    for (int it = 0; it < n_work; ++it) {
+      const int s = it % STAGES, k = it / STAGES;
+      if (k > 0) ok = mbar_wait(bar_empty + 8 * s, (k - 1) & 1, kWaitLimitNs);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      const int t0 = start + it * kTile;
+      const int pg = t0 >> lbs;
+      if (pg >= win + 32) {
+        win += 32;
+        cur = nxt;
+        nxt = (win + 32 + lane < n_pages) ? __ldg(bt + win + 32 + lane) : 0;
+      }
+      const int row0 = bs > kTile ? (t0 & (bs - 1)) : 0;
+      const int valid_pages = min(pages_per_tile, n_pages - pg);
+      const uint32_t dk = smem_base + s * STAGE_STRIDE;
+      const uint32_t dv = dk + V_OFFSET;
+      int pid[8];
 #pragma unroll
-    for (int w = 0; w < CW; ++w) {
-      const float* src = f + L::kRedAcc + (w * NCOL + g) * L::kAccStride + d0;
+      for (int j = 0; j < 8; ++j) pid[j] = __shfl_sync(0xffffffffu, cur, (pg - win + j) & 31);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar_full + 8 * s,
+                              valid_pages * rows * 128 * HALVES * 2);
 #pragma unroll
-      for (int h = 0; h < kParts; ++h) {
-        float4 v = *reinterpret_cast<const float4*>(src + h * (D / 2));
-        if constexpr (MODE == kDup) {  // columns g + 4 hold the bf16 residuals
-          const float4 r = *reinterpret_cast<const float4*>(src + 4 * L::kAccStride + h * (D / 2));
-          v.x += r.x;
-          v.y += r.y;
-          v.z += r.z;
-          v.w += r.w;
+        for (int j = 0; j < 8; ++j) {
+          if (j < valid_pages) {
+            // page j of the tile: both column halves of `rows` rows
+            const uint32_t off = j * rows * 128 * HALVES;
+            tma_load_5d(dk + off, tmK, bar_full + 8 * s, 0, kvh, row0, 0, pid[j], policy);
+            tma_load_5d(dv + off, tmV, bar_full + 8 * s, 0, kvh, row0, 0, pid[j], policy);
+          }
         }
-        o[h].x += wt[w] * v.x;
-        o[h].y += wt[w] * v.y;
-        o[h].z += wt[w] * v.z;
-        o[h].w += wt[w] * v.w;
       }
+      ++issued;
+      __syncwarp();
     }
-    const size_t row = static_cast<size_t>(b) * a.Hq + h0 + g;
-    if (direct) {
-      if (a.out_f32) {
-        float* dst = a.out_f32 + row * D + d0;
-#pragma unroll
-        for (int h = 0; h < kParts; ++h) *reinterpret_cast<float4*>(dst + h * (D / 2)) = o[h];
-      } else {
-        __nv_bfloat16* dst = a.out + row * D + d0;
-#pragma unroll
-        for (int h = 0; h < kParts; ++h)
-          *reinterpret_cast<uint2*>(dst + h * (D / 2)) =
-              make_uint2(pack_bf16x2(o[h].x, o[h].y), pack_bf16x2(o[h].z, o[h].w));
-      }
-      if (d0 == 0 && a.lse) a.lse[row] = lse_s;
-    } else {
-      float* dst = a.part_o + (row * a.n_splits + split) * D + d0;
-#pragma unroll
-      for (int h = 0; h < kParts; ++h) *reinterpret_cast<float4*>(dst + h * (D / 2)) = o[h];
-      if (d0 == 0) a.part_lse[row * a.n_splits + split] = lse_s;
-    }
+  }
+  if (!ok && lane == 0) {
+    raise_device_error(1u);
+    *cta_error = 1;
+  }
+  // No copy may still be landing in shared memory when the CTA retires.
+  if (lane == 0) {
+    for (int it = issued > STAGES ? issued - STAGES : 0; it < issued; ++it)
+      if (!mbar_wait(bar_full + 8 * (it % STAGES), (it / STAGES) & 1, kWaitLimitNs))
+        raise_device_error(2u);
   }
 }
 
@@ -967,88 +1071,500 @@ __global__ void __launch_bounds__(split_threads<CW>(), CW == kConsumerWarps ? kC
 
   if (warp == CW) {
     // ------------------------------------------------------------- producer
-    // Every lane waits (the decision is made warp-uniform); lane 0 issues.
-    const uint64_t policy = policy_evict_first();
-    int issued = it_base;   // ring uses so far (the sparse scan's stages)
-    bool ok = true;
-    if constexpr (!PAGED) {
-      for (int it = 0; it < n_work; ++it) {
-        const int ig = it_base + it;
-        const int s = ig % STAGES, k = ig / STAGES;
-        if (k > 0) ok = mbar_wait(bar_empty + 8 * s, (k - 1) & 1, kWaitLimitNs);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        if (lane == 0) {
-          const int t0 = start + (SPARSE ? static_cast<int>(list[it]) : it) * kTile;
-          const uint32_t dk = smem_base + s * L::kStageBytes;
-          const uint32_t dv = dk + L::kTileBytes;
-          mbar_arrive_expect_tx(bar_full + 8 * s, L::kStageBytes);
-          tma_load_5d(dk, &tmK, bar_full + 8 * s, 0, kvh, t0, 0, b, policy);
-          tma_load_5d(dv, &tmV, bar_full + 8 * s, 0, kvh, t0, 0, b, policy);
-        }
-        ++issued;
-        __syncwarp();
-      }
-    } else {
-      const int bs = a.block_size, lbs = a.log2_block_size;
-      const int rows = bs < kTile ? bs : kTile;            // rows per TMA box
-      const int pages_per_tile = bs < kTile ? kTile / bs : 1;
-      const int n_pages = (n + bs - 1) >> lbs;
-      const int32_t* bt = a.block_table + static_cast<size_t>(b) * a.max_blocks_per_seq;
-      // A window of 32 page ids, one per lane, plus the next window in flight.
-      int win = start >> lbs;
-      int cur = (win + lane < n_pages) ? __ldg(bt + win + lane) : 0;
-      int nxt = (win + 32 + lane < n_pages) ? __ldg(bt + win + 32 + lane) : 0;
-      for (int it = 0; it < n_work; ++it) {
-        const int s = it % STAGES, k = it / STAGES;
-        if (k > 0) ok = mbar_wait(bar_empty + 8 * s, (k - 1) & 1, kWaitLimitNs);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        const int t0 = start + it * kTile;
-        const int pg = t0 >> lbs;
-        if (pg >= win + 32) {
-          win += 32;
-          cur = nxt;
-          nxt = (win + 32 + lane < n_pages) ? __ldg(bt + win + 32 + lane) : 0;
-        }
-        const int row0 = bs > kTile ? (t0 & (bs - 1)) : 0;
-        const int valid_pages = min(pages_per_tile, n_pages - pg);
-        const uint32_t dk = smem_base + s * L::kStageBytes;
-        const uint32_t dv = dk + L::kTileBytes;
-        int pid[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) pid[j] = __shfl_sync(0xffffffffu, cur, (pg - win + j) & 31);
-        if (lane == 0) {
-          mbar_arrive_expect_tx(bar_full + 8 * s,
-                                valid_pages * rows * 128 * L::kHalves * 2);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (j < valid_pages) {
-              // page j of the tile: both column halves of `rows` rows
-              const uint32_t off = j * rows * 128 * L::kHalves;
-              tma_load_5d(dk + off, &tmK, bar_full + 8 * s, 0, kvh, row0, 0, pid[j], policy);
-              tma_load_5d(dv + off, &tmV, bar_full + 8 * s, 0, kvh, row0, 0, pid[j], policy);
-            }
-          }
-        }
-        ++issued;
-        __syncwarp();
-      }
-    }
-    if (!ok && lane == 0) {
-      raise_device_error(1u);
-      *cta_error = 1;
-    }
-    // No copy may still be landing in shared memory when the CTA retires.
-    if (lane == 0) {
-      for (int it = issued > STAGES ? issued - STAGES : 0; it < issued; ++it)
-        if (!mbar_wait(bar_full + 8 * (it % STAGES), (it / STAGES) & 1, kWaitLimitNs))
-          raise_device_error(2u);
-    }
+    split_producer<PAGED, SPARSE, STAGES, L::kStageBytes, L::kTileBytes, L::kHalves>(
+        a, &tmK, &tmV, smem_base, bar_full, bar_empty, cta_error, lane, b, kvh, start, n,
+        n_work, it_base, list);
   } else {
     // ------------------------------------------------------------- consumers
     split_consumers<D, NB, MODE, STAGES, FP8, SPARSE, CW>(a, smem, smem_base, bar_full, bar_empty,
                                                       cta_error, warp, lane, b, h0, split,
                                                       start, end, n_work, n_parts, list,
                                                       it_base);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// fp8 split kernel on the fifth-generation tensor cores (tcgen05).
+//
+// Same work split, producer and merge as fd_split_kernel with an fp8 cache,
+// but the two contractions are kind::f8f6f4 MMAs that read the e4m3 K and V
+// tiles straight from the TMA-swizzled ring: no code is converted in
+// registers.  Tensor memory keeps the accumulator rows of warp j of a
+// warpgroup in lanes 32j .. 32j+31, the lanes that warp may read.
+//
+// A tcgen05 MMA costs its issuing thread about the same time whatever its
+// size when it is this small, so the scores are taken four tiles at a time:
+// the ring keeps its K tiles apart from its V tiles, four consecutive K
+// tiles are one 256-row operand, and
+//  S = Q K^T  (M = 64, N = 256 tokens, K = 128; rows 16j .. 16j+15 in lanes
+//    32j .. 32j+15): the A rows 16j + r of every j hold the same 2G rows of
+//    q as e4m3 pairs, so warp j reads the scores of tokens 16j .. 16j+15 of
+//    each tile for all heads from its own lanes.  The warps copy their two
+//    tiles' scores to registers first, which frees S for the next four.
+//  O += P V  (M = 128, N = 128 = D, K = 64 tokens; row i in lane i): warp
+//    j's 3G rows 32j + r of P are non-zero only in its own 16 tokens, so
+//    rows 32j .. 32j+31 of O sum that warp's tokens alone, under that warp's
+//    running maximum.
+//
+// A bf16 value x is split exactly into two e4m3 codes, x sigma = x1 + x2 / 16
+// (sigma a power of two that brings max |x| to [128, 256)); q rows r < G hold
+// x1 of head r and rows G + r hold x2.  The softmax weights p <= 2^8 take
+// three codes, p = p1 + p2 / 16 + p3 / 256 (12 significant bits, like an f16
+// weight; two codes, 8 bits, moved the log-sum-exp of a dominant token by up
+// to 2^-8), in P rows r, G + r and 2G + r, and the running sum adds the
+// split values, so O and l see the same weights.
+// A warp rescales its O rows only when its maximum grows by more than 2^8;
+// until then the weights stay relative to the older maximum.
+//
+// Warps: 0-7 softmax (two warpgroups that take alternate tiles, each with
+// its own O in tensor memory), 8 the TMA producer, 9 the MMA issuer.
+constexpr int kTcSoftmaxWarps = 8;
+constexpr int kTcProducerWarp = kTcSoftmaxWarps;
+constexpr int kTcMmaWarp = kTcSoftmaxWarps + 1;
+constexpr int kTcThreads = (kTcSoftmaxWarps + 2) * 32;
+constexpr int kTcMaxG = 8;                   // 3G rows of P per warp, at most 32
+constexpr int kTcQuad = 4;                   // tiles per score MMA
+constexpr uint32_t kTcCols = 512;            // TMEM columns: S of four tiles at 0 (256),
+constexpr uint32_t kTcOCol = 256;            // O of warpgroup g at 256 + 128 g
+constexpr float kTcRescaleLog2 = 8.f;        // weights up to 2^8 before a rescale
+
+template <int STAGES>
+struct TcSmem {
+  static_assert(STAGES % kTcQuad == 0, "four consecutive K tiles are contiguous");
+  static constexpr int kTileBytes = kTile * 128;          // 64 token rows of 128 codes
+  static constexpr int kHalves = 1;
+  static constexpr int kKRing = 0;                        // STAGES K tiles
+  static constexpr int kVRing = STAGES * kTileBytes;      // STAGES V tiles
+  static constexpr int kQOffset = 2 * STAGES * kTileBytes;  // 64 x 128 e4m3, 128-byte swizzle
+  static constexpr int kPOffset = kQOffset + 64 * 128;    // two 128 x 64 e4m3, 8x16-byte cores
+  static constexpr int kPBytes = 128 * 64;
+  static constexpr int kBarOffset = kPOffset + 2 * kPBytes;
+  static constexpr int kSFull = kBarOffset + 2 * STAGES * 8;  // scores of a quad ready
+  static constexpr int kSFree = kSFull + 8;                   // scores of a quad copied out
+  static constexpr int kPFull = kSFree + 8;                   // per warpgroup: P written
+  static constexpr int kODone = kPFull + 16;                  // per warpgroup: P.V done
+  static constexpr int kMmaDone = kODone + 16;                // every MMA done
+  static constexpr int kTmemSlot = kMmaDone + 8;
+  static constexpr int kErrorOffset = kTmemSlot + 4;
+  static constexpr int kQExpOffset = kErrorOffset + 4;        // int per head
+  static constexpr int kBytes = kQExpOffset + 4 * kTcMaxG;
+  static constexpr int kDynamicBytes = kBytes + 1024;         // room to align to 1 KB
+  // Epilogue scratch over the drained ring, in the layout split_merge reads.
+  static constexpr int kNcol = 8;
+  static constexpr int kAccStride = 128 + 4;
+  static constexpr int kRedAcc = 0;
+  static constexpr int kRedM = kRedAcc + kTcSoftmaxWarps * kNcol * kAccStride;
+  static constexpr int kRedL = kRedM + kTcSoftmaxWarps * kNcol;
+  static constexpr int kScratchFloats = kRedL + kTcSoftmaxWarps * kNcol;
+  static_assert(kScratchFloats * 4 <= kQOffset, "epilogue scratch must fit the ring");
+  static_assert(kDynamicBytes <= 227 * 1024, "shared memory per CTA");
+};
+
+// Byte offset of (row, byte k) in the 128 x 64 P operand: 8-row x 16-byte core
+// matrices, 128 bytes apart along k and 512 bytes apart along the rows.
+__device__ __forceinline__ uint32_t tc_p_offset(uint32_t row, uint32_t k) {
+  return (row >> 3) * 512 + (k >> 4) * 128 + (row & 7) * 16 + (k & 15);
+}
+
+// Two floats to an e4m3 pair (round to nearest even, saturating), x in the
+// low byte, and the values it holds.
+__device__ __forceinline__ uint32_t tc_e4m3x2(float x, float y, float& xq, float& yq) {
+  const __nv_fp8x2_storage_t c = __nv_cvt_float2_to_fp8x2(make_float2(x, y), __NV_SATFINITE, __NV_E4M3);
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(c, __NV_E4M3);
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+  xq = f.x;
+  yq = f.y;
+  return static_cast<uint32_t>(c);
+}
+
+template <bool PAGED, int STAGES, int G>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    fd_split_tc_kernel(const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const SplitArgs a) {
+  using L = TcSmem<STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t smem_base = smem_u32(smem);
+  const uint32_t bar_full = smem_base + L::kBarOffset;
+  const uint32_t bar_empty = bar_full + STAGES * 8;
+  const uint32_t s_full = smem_base + L::kSFull;
+  const uint32_t s_free = smem_base + L::kSFree;
+  const uint32_t p_full = smem_base + L::kPFull;
+  const uint32_t o_done = smem_base + L::kODone;
+  const uint32_t mma_done = smem_base + L::kMmaDone;
+  volatile int* cta_error = reinterpret_cast<volatile int*>(smem + L::kErrorOffset);
+  int* qexp = reinterpret_cast<int*>(smem + L::kQExpOffset);
+
+  const int split = blockIdx.x;
+  const int kvh = blockIdx.y;
+  const int b = blockIdx.z;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);   // released by the commit of the tile's P.V
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, kTcSoftmaxWarps);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(p_full + 8 * g, 4);      // the four warps of the warpgroup
+      mbar_init(o_done + 8 * g, 1);
+    }
+    mbar_init(mma_done, 1);
+    *cta_error = 0;
+    fence_mbar_init();
+  }
+  if (warp == kTcProducerWarp && lane == 0) {
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmV);
+  }
+  if constexpr (!PAGED) {
+    if (warp == kTcProducerWarp && lane < a.prefetch_tiles) {
+      const int tile0 = split_first_tile(a, split);
+      const int t0 = (tile0 + lane) * kTile;
+      if (tile0 + lane < split_first_tile(a, split + 1) && t0 < a.max_len) {
+        tma_prefetch_l2_5d(&tmK, 0, kvh, t0, 0, b);
+        tma_prefetch_l2_5d(&tmV, 0, kvh, t0, 0, b);
+      }
+    }
+  }
+  if (warp == kTcMmaWarp) {
+    tmem_alloc(smem_base + L::kTmemSlot, kTcCols);
+    tmem_relinquish();
+  }
+  tcgen05_fence_before();
+  __syncthreads();
+  tcgen05_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::kTmemSlot);
+
+  grid_dependency_wait();
+
+  const int n = seq_length(a.seqlens, b, a.max_len);
+  const int start = split_first_tile(a, split) * kTile;
+  const int end = min(split_first_tile(a, split + 1) * kTile, n);
+  static_assert(G == 2 || G == 4 || G == 8, "group sizes of the tcgen05 kernel");
+  const int h0 = kvh * G;
+  const int n_tiles = start < end ? (end - start + kTile - 1) / kTile : 0;
+  const int n_quads = (n_tiles + kTcQuad - 1) / kTcQuad;
+  const int n_parts = (a.n_splits == 1 || (n + kTile - 1) / kTile <= a.tile_q) ? 1 : 2;
+
+  if (n_tiles == 0) {
+    if (split == 0) {  // an empty sequence: out = 0, lse = -inf
+      const size_t base = (static_cast<size_t>(b) * a.Hq + h0) * 128;
+      for (int i = threadIdx.x; i < G * 128; i += kTcThreads) {
+        if (a.out_f32)
+          a.out_f32[base + i] = 0.f;
+        else
+          a.out[base + i] = __float2bfloat16_rn(0.f);
+      }
+      if (a.lse && threadIdx.x < G) a.lse[static_cast<size_t>(b) * a.Hq + h0 + threadIdx.x] = -INFINITY;
+    }
+  } else {
+    if (warp < kTcSoftmaxWarps) {
+      // Zero the q and P operands (24 KB: 96 bytes per thread) ...
+      uint4* z = reinterpret_cast<uint4*>(smem + L::kQOffset);
+#pragma unroll
+      for (int i = 0; i < 6; ++i) z[threadIdx.x * 6 + i] = make_uint4(0u, 0u, 0u, 0u);
+      named_barrier_sync(1, kTcSoftmaxWarps * 32);
+      // ... then warp g < G writes head g's pair into rows 16j + g and
+      // 16j + G + g of every j; lane l holds head-dim entries 4l .. 4l+3.
+      const int g = warp;
+      if (g < G) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(
+            a.q + (static_cast<size_t>(b) * a.Hq + h0 + g) * 128 + 4 * lane);
+        const __nv_bfloat162 q01 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+        const __nv_bfloat162 q23 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+        float x[4] = {__low2float(q01), __high2float(q01), __low2float(q23), __high2float(q23)};
+        float mx = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        int e = 0;
+        frexpf(mx, &e);                  // mx = f 2^e, f in [0.5, 1); 0 for mx = 0
+        float r[4];
+        for (int i = 0; i < 4; ++i) x[i] = ldexpf(x[i], 8 - e);   // exact
+        float x1[4], x2[4];
+        const uint32_t c01 = tc_e4m3x2(x[0], x[1], x1[0], x1[1]);
+        const uint32_t c23 = tc_e4m3x2(x[2], x[3], x1[2], x1[3]);
+        for (int i = 0; i < 4; ++i) r[i] = (x[i] - x1[i]) * 16.f;   // exact
+        const uint32_t d01 = tc_e4m3x2(r[0], r[1], x2[0], x2[1]);
+        const uint32_t d23 = tc_e4m3x2(r[2], r[3], x2[2], x2[3]);
+        const uint32_t w1 = c01 | (c23 << 16);
+        const uint32_t w2 = d01 | (d23 << 16);
+        const uint32_t chunk = static_cast<uint32_t>(lane) >> 2;
+        const uint32_t within = (static_cast<uint32_t>(lane) & 3) * 4;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t r1 = 16 * j + g, r2 = 16 * j + G + g;
+          *reinterpret_cast<uint32_t*>(smem + L::kQOffset + r1 * 128 + ((chunk ^ (r1 & 7)) << 4) + within) = w1;
+          *reinterpret_cast<uint32_t*>(smem + L::kQOffset + r2 * 128 + ((chunk ^ (r2 & 7)) << 4) + within) = w2;
+        }
+        if (lane == 0) qexp[g] = e;
+      }
+      fence_proxy_async_smem();
+    }
+    __syncthreads();
+
+    if (warp == kTcProducerWarp) {
+      split_producer<PAGED, false, STAGES, L::kTileBytes, L::kVRing - L::kKRing, L::kHalves>(
+          a, &tmK, &tmV, smem_base + L::kKRing, bar_full, bar_empty, cta_error, lane, b, kvh,
+          start, n, n_tiles, 0, nullptr);
+    } else if (warp == kTcMmaWarp) {
+      if (lane == 0) {
+        constexpr uint32_t kIdS = idesc_e4m3_f32(64, kTcQuad * kTile, false, false);
+        constexpr uint32_t kIdPV = idesc_e4m3_f32(128, 128, false, true);
+        const uint32_t qaddr = smem_base + L::kQOffset;
+        bool ok = true;
+        // The scores of quad q (tiles 4q .. 4q+3, stages 4q mod STAGES ..),
+        // once its tiles have landed; tiles past the split give columns
+        // nobody reads.
+        auto issue_scores = [&](int q) -> bool {
+          const int t_end = min(kTcQuad * q + kTcQuad, n_tiles);
+          for (int t = kTcQuad * q; t < t_end; ++t)
+            if (!mbar_wait(bar_full + 8 * (t % STAGES), (t / STAGES) & 1, kWaitLimitNs)) return false;
+          tcgen05_fence_after();
+          const uint32_t kaddr = smem_base + L::kKRing + ((kTcQuad * q) % STAGES) * L::kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_e4m3(tmem, smem_desc(qaddr + 32 * kk, 16, 1024, 2),
+                     smem_desc(kaddr + 32 * kk, 16, 1024, 2), kIdS, kk > 0);
+          tcgen05_commit(s_full);
+          return true;
+        };
+        ok = issue_scores(0);
+        for (int i = 0; ok && i < n_tiles; ++i) {
+          const int grp = i & 1, k = i >> 1;
+          if (!mbar_wait(p_full + 8 * grp, k & 1, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tcgen05_fence_after();
+          const int s = i % STAGES;
+          const uint32_t vaddr = smem_base + L::kVRing + s * L::kTileBytes;
+          const uint32_t paddr = smem_base + L::kPOffset + grp * L::kPBytes;
+          const uint32_t d = tmem + kTcOCol + grp * 128;
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk)
+            mma_e4m3(d, smem_desc(paddr + 256 * kk, 128, 512, 0),
+                     smem_desc(vaddr + 4096 * kk, 0, 1024, 2), kIdPV, k > 0 || kk > 0);
+          tcgen05_commit(o_done + 8 * grp);
+          tcgen05_commit(bar_empty + 8 * s);
+          // After the first P.V of a quad, the next quad's scores: every
+          // softmax warp has copied this quad's out of S by then.
+          const int q = i / kTcQuad;
+          if (i == kTcQuad * q && q + 1 < n_quads) {
+            if (!mbar_wait(s_free, q & 1, kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
+            ok = issue_scores(q + 1);
+          }
+        }
+        if (!ok) {
+          raise_device_error(1u);
+          *cta_error = 1;
+        }
+        // Nothing may still run on the tensor cores when TMEM is released.
+        tcgen05_commit(mma_done);
+        if (!mbar_wait(mma_done, 0, kWaitLimitNs)) raise_device_error(2u);
+      }
+      __syncwarp();
+    } else {
+      // ----------------------------------------------------------- softmax
+      // After the load, lane r holds S row r (code r / G of head r mod G)
+      // for the warp's 16 tokens; the scores are then spread so that lane l
+      // holds tokens m TPL .. m TPL + TPL - 1 of head h = l mod G (m = l / G),
+      // and every lane does a share of the exponentials and weight codes.
+      constexpr int TPL = G / 2;                            // tokens per lane
+      const int grp = warp >> 2, j = warp & 3;
+      const uint32_t lane_base = static_cast<uint32_t>(32 * j) << 16;
+      const uint32_t s_tm = tmem + lane_base + 16 * j;      // + 64 per tile of the quad
+      const uint32_t o_tm = tmem + lane_base + kTcOCol + grp * 128;
+      const int h = lane % G, m = lane / G;
+      const float sl2 = ldexpf(a.scale_log2, qexp[h] - 8);
+      uint8_t* pbuf = smem + L::kPOffset + grp * L::kPBytes;
+      // This lane's P bytes: code T of head h, tokens 16j + m TPL ...
+      uint32_t poff[3];
+#pragma unroll
+      for (int T = 0; T < 3; ++T) poff[T] = tc_p_offset(32 * j + T * G + h, 16 * j + m * TPL);
+      float m_run = -INFINITY, l_run = 0.f;                 // per head (l: this lane's share)
+      bool failed = false;
+      int k = 0;                                            // tiles of this warpgroup so far
+      for (int q = 0; q < n_quads && !failed; ++q) {
+        // This warpgroup's tiles of the quad: 4q + grp and 4q + grp + 2.
+        if (!__all_sync(0xffffffffu, mbar_wait(s_full, q & 1, kWaitLimitNs))) {
+          failed = true;
+          break;
+        }
+        tcgen05_fence_after();
+        uint32_t raw[2][16];
+        tmem_ld16(s_tm + grp * kTile, raw[0]);
+        tmem_ld16(s_tm + (grp + 2) * kTile, raw[1]);
+        tmem_wait_ld();
+        tcgen05_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int i = kTcQuad * q + grp + 2 * u;
+          if (i >= n_tiles) break;
+          const int tile_valid = min(kTile, end - (start + i * kTile));
+          float t[TPL];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float v1 = __shfl_sync(0xffffffffu, __uint_as_float(raw[u][c]), h);
+            const float v2 = __shfl_sync(0xffffffffu, __uint_as_float(raw[u][c]), G + h);
+            if (c / TPL == m) t[c % TPL] = (v1 + v2 * 0.0625f) * sl2;
+          }
+          float mx = -INFINITY;
+#pragma unroll
+          for (int x = 0; x < TPL; ++x) {
+            if (16 * j + m * TPL + x >= tile_valid) t[x] = -INFINITY;
+            mx = fmaxf(mx, t[x]);
+          }
+#pragma unroll
+          for (int off = G; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+          const float m_new = fmaxf(m_run, mx);
+          const bool rescale = k > 0 && m_new > m_run + kTcRescaleLog2;
+          const float al = rescale ? ex2(m_run - m_new) : 1.f;
+          if (k == 0 || rescale) m_run = m_new;
+          l_run *= al;
+          const float mu = m_run == -INFINITY ? 0.f : m_run;
+          // p = p1 + p2 / 16 + p3 / 256, each code e4m3; the residuals are
+          // exact in fp32.
+          uint32_t w[3] = {0u, 0u, 0u};
+          float lsum = 0.f;
+#pragma unroll
+          for (int x = 0; x < TPL; x += 2) {
+            const float p0 = ex2(t[x] - mu);
+            const float p1 = TPL > 1 ? ex2(t[x + 1] - mu) : 0.f;
+            float a0, a1, b0, b1, d0, d1;
+            const uint32_t c1 = tc_e4m3x2(p0, p1, a0, a1);
+            const float r0 = p0 - a0, r1 = p1 - a1;
+            const uint32_t c2 = tc_e4m3x2(r0 * 16.f, r1 * 16.f, b0, b1);
+            const float e0 = r0 - b0 * 0.0625f, e1 = r1 - b1 * 0.0625f;
+            const uint32_t c3 = tc_e4m3x2(e0 * 256.f, e1 * 256.f, d0, d1);
+            lsum += ((a0 + a1) + (b0 + b1) * 0.0625f) + (d0 + d1) * 0.00390625f;
+            w[0] |= c1 << (8 * x);
+            w[1] |= c2 << (8 * x);
+            w[2] |= c3 << (8 * x);
+          }
+          // P.V of this warpgroup's previous tile must be done before its P
+          // buffer is rewritten or O is rescaled.
+          if (k > 0) {
+            if (!__all_sync(0xffffffffu, mbar_wait(o_done + 8 * grp, (k - 1) & 1, kWaitLimitNs))) {
+              failed = true;
+              break;
+            }
+            tcgen05_fence_after();
+          }
+          if (__any_sync(0xffffffffu, rescale)) {
+            // Lane r holds O row r, whose head is r mod G: this lane's own.
+#pragma unroll 1
+            for (int cc = 0; cc < 8; ++cc) {
+              uint32_t o[16];
+              tmem_ld16(o_tm + 16 * cc, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * al);
+              tmem_st16(o_tm + 16 * cc, o);
+            }
+            tmem_wait_st();
+          }
+          l_run += lsum;
+#pragma unroll
+          for (int T = 0; T < 3; ++T) {
+            if constexpr (TPL == 4) {
+              *reinterpret_cast<uint32_t*>(pbuf + poff[T]) = w[T];
+            } else if constexpr (TPL == 2) {
+              *reinterpret_cast<uint16_t*>(pbuf + poff[T]) = static_cast<uint16_t>(w[T]);
+            } else {
+              pbuf[poff[T]] = static_cast<uint8_t>(w[T]);
+            }
+          }
+          if (tile_valid < kTile) {
+            // Rows past the sequence may hold anything (NaN included): zero
+            // this warp's invalid V rows so that 0 * NaN never reaches O.
+            // The wait on the stage's phase, already complete, orders its
+            // copies before these writes.
+            if (!__all_sync(0xffffffffu, mbar_wait(bar_full + 8 * (i % STAGES), (i / STAGES) & 1,
+                                                   kWaitLimitNs))) {
+              failed = true;
+              break;
+            }
+            uint8_t* vt = smem + L::kVRing + (i % STAGES) * L::kTileBytes;
+            const int rr = 16 * j + (lane >> 1);
+            if (rr >= tile_valid) {
+              uint4* dst = reinterpret_cast<uint4*>(vt + rr * 128 + (lane & 1) * 64);
+#pragma unroll
+              for (int c = 0; c < 4; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+            }
+          }
+          fence_proxy_async_smem();
+          tcgen05_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(p_full + 8 * grp);
+          ++k;
+        }
+      }
+      // The last P.V of this warpgroup.
+      if (!failed && k > 0 &&
+          !__all_sync(0xffffffffu, mbar_wait(o_done + 8 * grp, (k - 1) & 1, kWaitLimitNs)))
+        failed = true;
+      tcgen05_fence_after();
+      grid_dependents_launch();
+      if (failed && lane == 0) {
+        raise_device_error(1u);
+        *cta_error = 1;
+      }
+      // Both warpgroups are past their last MMA, so the ring holds the
+      // scratch: per warp and head the O row (the three weight terms summed),
+      // the running maximum and sum.
+      named_barrier_sync(1, kTcSoftmaxWarps * 32);
+      float* f = reinterpret_cast<float*>(smem);
+      const bool live = !*cta_error;
+      // Sum the lanes' shares of each head's running sum.
+#pragma unroll
+      for (int off = G; off < 32; off <<= 1) l_run += __shfl_xor_sync(0xffffffffu, l_run, off);
+      const bool head_lane = lane < G;
+      if (live) {
+        float* dst = f + L::kRedAcc + (warp * L::kNcol + h) * L::kAccStride;
+#pragma unroll 1
+        for (int cc = 0; cc < 8; ++cc) {
+          uint32_t o[16];
+          if (k > 0) {
+            tmem_ld16(o_tm + 16 * cc, o);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) o[c] = 0u;
+          }
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float v = __uint_as_float(o[c]);
+            const float v2 = __shfl_down_sync(0xffffffffu, v, G);
+            const float v3 = __shfl_down_sync(0xffffffffu, v, 2 * G);
+            if (head_lane) dst[16 * cc + c] = v + (v2 * 0.0625f + v3 * 0.00390625f);
+          }
+        }
+        if (head_lane) {
+          f[L::kRedM + warp * L::kNcol + h] = m_run;
+          f[L::kRedL + warp * L::kNcol + h] = l_run;
+        }
+      }
+      named_barrier_sync(1, kTcSoftmaxWarps * 32);
+      if (live) split_merge<128, 1, kHi, kTcSoftmaxWarps, L>(a, f, b, h0, split, n_parts);
+    }
+  }
+
+  // Release the tensor memory once every warp is past its last use.
+  tcgen05_fence_before();
+  __syncthreads();
+  if (warp == kTcMmaWarp) {
+    tcgen05_fence_after();
+    tmem_dealloc(tmem, kTcCols);
   }
 }
 

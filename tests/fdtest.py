@@ -52,8 +52,9 @@ def host_bf16(x) -> np.ndarray:
 class OnDevice:
     """Device copies of a workload's tensors."""
 
-    def __init__(self, w: wl.Workload):
+    def __init__(self, w: wl.Workload, fp8_mma: int = 0):
         self.w = w
+        self.fp8_mma = fp8_mma
         self.q = dev_bf16(w.q)
         up = dev_bf16 if w.kv_dtype == "bf16" else dev_u8
         self.k = up(w.k)
@@ -65,7 +66,7 @@ class OnDevice:
         w = self.w
         return fd.make_problem(w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size, w.num_blocks,
                                w.max_blocks_per_seq, w.kv_layout, w.kv_dtype_code, w.k_scale,
-                               w.v_scale)
+                               w.v_scale, self.fp8_mma)
 
     def plan(self) -> int:
         """The split count the benchmark uses: fd_plan_problem over the whole

@@ -267,6 +267,13 @@ def test_decode_rejects_bad_paging():
     assert decode(P(bs=12, nb=64, mb=64), table=0x60000) == fd.FD_ERR_UNSUPPORTED
 
 
+def test_decode_rejects_unknown_fp8_mma():
+    for bad in (2, -1):
+        prob = P()
+        prob.fp8_mma = bad
+        assert decode(prob) == fd.FD_ERR_INVALID_ARGUMENT
+
+
 def test_decode_rejects_unknown_layout():
     prob = P()
     prob.kv_layout = 2
@@ -277,8 +284,9 @@ def test_decode_rejects_unknown_layout():
 
 def test_problem_struct_matches_header():
     import ctypes
-    # ten int32 fields and two floats, in the order of fd_problem in include/fd.h
-    assert ctypes.sizeof(fd.fd_problem) == 12 * 4
+    # ten int32 fields, two floats and one more int32, in the order of
+    # fd_problem in include/fd.h
+    assert ctypes.sizeof(fd.fd_problem) == 13 * 4
     names = [f[0] for f in fd.fd_problem._fields_]
     text = open(os.path.join(ROOT, "include", "fd.h")).read()
     body = text[text.index("typedef struct fd_problem {"):text.index("} fd_problem;")]
@@ -445,3 +453,14 @@ def test_static_workspace_size_matches_header():
     expr = m.group(1).strip()
     value = eval(re.sub(r"(\d+)[uUlL]+", r"\1", expr), {"__builtins__": {}})
     assert value == fd.FD_STATIC_WORKSPACE_BYTES
+
+
+def test_enum_values_match_header():
+    """The binding's enum constants are the header's enumerator values."""
+    import re
+    text = open(os.path.join(ROOT, "include", "fd.h")).read()
+    for name in ("FD_LAYOUT_HND", "FD_LAYOUT_NHD", "FD_KV_BF16", "FD_KV_FP8_E4M3",
+                 "FD_FP8_MMA_SYNC", "FD_FP8_MMA_TCGEN05"):
+        m = re.search(rf"\b{name}\s*=\s*(\d+)", text)
+        assert m, f"{name} is not an enumerator of fd.h"
+        assert int(m.group(1)) == getattr(fd, name), name
