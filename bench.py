@@ -78,6 +78,8 @@ def parse_args():
     ap.add_argument("--splits", type=int, default=None, help="override the planner's split count")
     ap.add_argument("--kv-dtype", choices=["bf16", "fp8"], default="bf16",
                     help="cache element type (fp8: e4m3 codes with per-tensor scales)")
+    ap.add_argument("--fp8-mma", choices=["mma_sync", "tcgen05"], default="mma_sync",
+                    help="tensor-core path of an fp8 cache (fd_problem.fp8_mma)")
     ap.add_argument("--layout", choices=["HND", "NHD"], default="HND",
                     help="cache dimension order (heads outside tokens, or tokens outside heads)")
     ap.add_argument("--shard-sequence", action="store_true",
@@ -252,7 +254,7 @@ class Call:
     """Device buffers and a bound fd_decode call for one workload; `copies`
     rotating cache copies keep L2 from serving K/V."""
 
-    def __init__(self, torch, fd, w, device, num_splits=None, copies=1):
+    def __init__(self, torch, fd, w, device, num_splits=None, copies=1, fp8_mma=0):
         self.torch, self.fd, self.w = torch, fd, w
         self.q = dev_bf16(torch, w.q, device)
         k = host_cache(torch, w.k).to(device)
@@ -263,7 +265,7 @@ class Call:
         self.table = None if w.block_table is None else torch.from_numpy(w.block_table).to(device)
         self.prob = fd.make_problem(w.B, w.Hq, w.Hkv, w.D, w.max_len, w.block_size, w.num_blocks,
                                     w.max_blocks_per_seq, w.kv_layout, w.kv_dtype_code,
-                                    w.k_scale, w.v_scale)
+                                    w.k_scale, w.v_scale, fp8_mma)
         if num_splits:
             self.S = num_splits
         else:  # the planner over the whole problem, lengths included when known
@@ -599,7 +601,11 @@ def run_fd(args):
     w = make_workload(args.workload, args.L, rank, layout=args.layout, kv_dtype=args.kv_dtype)
     kvb = w.kv_bytes()
     copies, l2 = copies_for(torch, (w.k.nbytes + w.v.nbytes), device)
-    call = Call(torch, fd, w, device, args.splits, copies)
+    tcgen05 = w.kv_dtype == "fp8" and args.fp8_mma == "tcgen05"
+    call = Call(torch, fd, w, device, args.splits, copies,
+                fd.FD_FP8_MMA_TCGEN05 if tcgen05 else fd.FD_FP8_MMA_SYNC)
+    # ncu records are per kernel: the tcgen05 path has its own entries
+    ncu_name = w.name + ("-tcgen05" if tcgen05 else "")
 
     sampler = ClockSampler(device.index)
     sampler.start()
@@ -627,9 +633,12 @@ def run_fd(args):
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
         "us_per_call": round(per_call_s * 1e6, 3), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16" if w.kv_dtype == "bf16" else "e4m3 cache, f16 mma",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.kv_dtype == "bf16" else
+                 ("e4m3 cache, e4m3 tcgen05 mma" if tcgen05 else "e4m3 cache, f16 mma"),
         "data": "synthetic",
-        "config": workload_config(w, call.S, call.s_eff, copies, l2, world),
+        "config": dict(workload_config(w, call.S, call.s_eff, copies, l2, world),
+                       **({"fp8_mma": args.fp8_mma} if w.kv_dtype == "fp8" else {})),
         # achieved: algorithmic bytes over the whole call's event-timed duration
         # (the split kernel, the dominant one, plus the combine), so it is a
         # lower bound for the split kernel alone; traffic: the split kernel's
@@ -638,7 +647,8 @@ def run_fd(args):
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                      "frac_of_spec_8tbs": round(achieved / SPEC_HBM_GBS, 4),
-                     "traffic": ncu_traffic(w.name, call.S), "traffic_kernel": "fd_split_kernel",
+                     "traffic": ncu_traffic(ncu_name, call.S),
+                     "traffic_kernel": "fd_split_tc_kernel" if tcgen05 else "fd_split_kernel",
                      "algorithmic_bytes": kvb},
         "gpu_launches": args.steps * call.launches_per_call,
         "clocks": clocks,
@@ -648,7 +658,7 @@ def run_fd(args):
         stats = sample_stats(per, calls, kvb, peak)
         stats["clocks"] = sampler.within(windows)
         result["samples"] = stats
-        result["kernels"] = kernel_times(ncu_launch_shares(w.name, call.S),
+        result["kernels"] = kernel_times(ncu_launch_shares(ncu_name, call.S),
                                          stats["us_per_call_median"], kvb, peak)
     if workloads is not None:
         result["workloads"] = workloads
