@@ -353,7 +353,7 @@ def _check_problem_sizes(problem: fd_problem, q, k_cache):
 def decode(q, k_cache, v_cache, seqlens=None, block_table=None, *, max_len: Optional[int] = None,
            kv_layout: int = FD_LAYOUT_HND, scale: Optional[float] = None,
            num_splits: Optional[int] = None, out=None, lse=None, workspace=None, stream=None,
-           k_scale: float = 1.0, v_scale: float = 1.0):
+           k_scale: float = 1.0, v_scale: float = 1.0, fp8_mma: int = FD_FP8_MMA_SYNC):
     """Decode attention on torch CUDA tensors.
 
     q [B, Hq, D] bf16.  Caches: bf16, or E4M3 codes (torch.uint8 or
@@ -363,9 +363,11 @@ def decode(q, k_cache, v_cache, seqlens=None, block_table=None, *, max_len: Opti
     [B, max_len, Hkv, D] or paged [num_blocks, block_size, Hkv, D].  Paged
     caches come with block_table [B, max_blocks] int32.  seqlens [B] int32
     or None.  Returns (out [B, Hq, D] bf16, lse [B, Hq] fp32).  num_splits
-    defaults to fd_plan_problem's choice.  Raises ValueError for tensors of
-    the wrong dtype, shape or device, or not contiguous, before anything is
-    launched, and FdError for a failing status."""
+    defaults to fd_plan_problem's choice.  fp8_mma picks the tensor-core path
+    of an fp8 cache (FD_FP8_MMA_SYNC or FD_FP8_MMA_TCGEN05).  Raises
+    ValueError for tensors of the wrong dtype, shape or device, or not
+    contiguous, before anything is launched, and FdError for a failing
+    status."""
     import torch
     _check_decode_args(q, k_cache, v_cache, seqlens, block_table, kv_layout, max_len, out, lse,
                        workspace)
@@ -380,7 +382,7 @@ def decode(q, k_cache, v_cache, seqlens=None, block_table=None, *, max_len: Opti
             _, L, Hkv, _ = k_cache.shape
         max_len = L if max_len is None else max_len
         prob = make_problem(B, Hq, Hkv, D, max_len, kv_layout=kv_layout, kv_dtype=kv_dtype,
-                            k_scale=k_scale, v_scale=v_scale)
+                            k_scale=k_scale, v_scale=v_scale, fp8_mma=fp8_mma)
     else:
         if kv_layout == FD_LAYOUT_HND:
             nb, Hkv, bs, _ = k_cache.shape
@@ -390,7 +392,7 @@ def decode(q, k_cache, v_cache, seqlens=None, block_table=None, *, max_len: Opti
         mbps = block_table.shape[1]
         max_len = mbps * bs if max_len is None else max_len
         prob = make_problem(B, Hq, Hkv, D, max_len, bs, nb, mbps, kv_layout, kv_dtype, k_scale,
-                            v_scale)
+                            v_scale, fp8_mma)
     if scale is None:
         scale = 1.0 / (D ** 0.5)
     if num_splits is None:

@@ -208,3 +208,22 @@ def test_fp8_tcgen05_path_runs_its_own_arithmetic():
         res[m] = (got, gl)
     a, b = res[fd.FD_FP8_MMA_SYNC], res[fd.FD_FP8_MMA_TCGEN05]
     assert not (np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1]))
+
+
+def test_fp8_decode_wrapper(mma):
+    """The torch-level decode() on uint8 code tensors, with the path chosen
+    by its fp8_mma argument, against the oracle."""
+    import torch
+    w = wl.make_problem(2, 16, 2, 128, 3000, seed=399, seqlens=[3000, 1700], kv_dtype="fp8")
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q = torch.from_numpy(w.q.view(np.int16)).to(dev).view(torch.bfloat16)
+    k = torch.from_numpy(w.k).to(dev)
+    v = torch.from_numpy(w.v).to(dev)
+    sl = torch.from_numpy(w.seqlens).to(dev)
+    out, lse = fd.decode(q, k, v, sl, scale=w.scale, num_splits=6, k_scale=w.k_scale,
+                         v_scale=w.v_scale, fp8_mma=mma)
+    torch.cuda.synchronize()
+    assert fd.fd_check_device_error() == fd.FD_OK
+    got = wl.bf16_bits_to_f64(out.view(torch.int16).cpu().numpy().view(np.uint16))
+    ref, rl = reference(w)
+    assert_close(got, lse.cpu().numpy().astype(np.float64), ref, rl, f"fp8 decode() mma={mma}")
