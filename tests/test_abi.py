@@ -274,6 +274,17 @@ def test_decode_rejects_unknown_fp8_mma():
         assert decode(prob) == fd.FD_ERR_INVALID_ARGUMENT
 
 
+def test_fp8_mma_values_pass_validation_for_every_cache_type():
+    # Both paths are valid values for a bf16 cache (where the field is
+    # ignored) and an fp8 one: the call gets as far as the workspace check,
+    # which comes after every argument check and before any device call, so
+    # nothing is launched on these placeholder pointers.
+    for kv_dtype in (fd.FD_KV_BF16, fd.FD_KV_FP8_E4M3):
+        for mma in (fd.FD_FP8_MMA_SYNC, fd.FD_FP8_MMA_TCGEN05):
+            prob = fd.make_problem(1, 8, 8, 128, 512, kv_dtype=kv_dtype, fp8_mma=mma)
+            assert decode(prob, S=2, ws=None, wsb=0) == fd.FD_ERR_WORKSPACE
+
+
 def test_decode_rejects_unknown_layout():
     prob = P()
     prob.kv_layout = 2
